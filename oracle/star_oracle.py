@@ -1,0 +1,327 @@
+"""Plain, slow, fp64 CPU oracle for the Star Attention two-phase attention path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or
+links this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA path; it takes plain NumPy arrays (the exact bf16 inputs
+upcast to float64) and returns float64 results.
+
+Sources (page title, then section / step / equation):
+
+* [P2] "Star Attention: Efficient LLM Inference over Long Sequences"
+  (paper-graph-ui analysis page), section 3.4 "Detailed, Sentence-Based
+  Technical Breakdown":
+    - "The Attention Decomposition" -- the causal softmax-attention equation
+      with scale 1/sqrt(d);
+    - "Phase 1: Context Encoding with Anchor Blocks", Steps 1-5 (partition,
+      anchor augmentation with preserved positions, blockwise-local causal
+      attention, anchor KV discard);
+    - "Phase 2: Query Encoding and Token Generation with Distributed Softmax",
+      Steps 3 (local A_h, s_h), the partition identity, Step 5 (log-sum-exp
+      aggregation) and Step 7 (only the query region grows).
+* [P3] "NVIDIA/Star-Attention" (README mirror), section "Two Phases of Star
+  Attention": Phase 1 bullets (segmentation, anchor prefix, non-anchor KV kept)
+  and Phase 2 bullets (A_h, s_h, s_global, A_global).
+
+Readings where the pages are silent or garbled (each is listed in the design doc):
+
+* the anchor is the first ``b_a`` context tokens, ``0 <= b_a <= b``;
+* block 0 is plain causal attention over its own rows, blocks i >= 1 see the
+  whole anchor plus their own block causally; only block rows are outputs;
+* the last block may be short;
+* ``s_h`` is carried as a natural-log log-sum-exp over the *scaled* logits;
+  the merge is ``s = log sum_h exp(s_h)``, ``A = sum_h exp(s_h - s) A_h``
+  (algebraically the README's ``s_h / s_global`` weights); the garbled
+  log-space update printed in [P2] Step 5 is not followed;
+* grouped-query heads map contiguously: q head ``h`` reads kv head
+  ``h // (Hq // Hkv)``;
+* a query row ``r`` sees query-region rows ``0..r``; a decode token is
+  appended to the query region first and then attends to it (itself included).
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+library routines (torch scaled-dot-product attention in float64,
+``scipy.special.logsumexp``), closed forms and brute force.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+# ---------------------------------------------------------------------------
+# Phase 1, Step 1: partition of the context into blocks.
+# ---------------------------------------------------------------------------
+def block_table(L: int, b: int) -> list[tuple[int, int]]:
+    """Blocks ``c_1..c_n`` of a context of ``L`` tokens with block size ``b``.
+
+    [P2] Phase 1 Step 1: ``n = ceil(L / b)`` contiguous blocks, the last one
+    possibly shorter.  Returns ``[(start, length), ...]``.
+    """
+    if L < 0 or b < 1:
+        raise ValueError("need L >= 0 and b >= 1")
+    n = -(-L // b)
+    return [(i * b, min((i + 1) * b, L) - i * b) for i in range(n)]
+
+
+# ---------------------------------------------------------------------------
+# Phase 1, Steps 2-4: the explicit Star mask.
+# ---------------------------------------------------------------------------
+def star_mask_rows(L: int, b: int, b_a: int, rows) -> np.ndarray:
+    """Rows ``rows`` of the explicit Star-Attention context mask, bool [R, L].
+
+    ``M[t, j]`` is True iff context token ``t`` attends to token ``j`` in
+    phase 1 ([P2] Phase 1 Steps 2 and 4, [P3] Phase 1 bullets):
+
+    * ``j <= t`` (causal), and
+    * ``j`` lies in the same block as ``t``, or ``t`` lies in a block
+      ``i >= 1`` and ``j`` is an anchor token (``j < b_a``).
+
+    The anchor keeps its original positions (Step 2), so with pre-rotated
+    inputs its keys are literally rows ``0..b_a-1`` of the context K/V.
+    """
+    if not (0 <= b_a <= b):
+        raise ValueError("need 0 <= b_a <= b")
+    t = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.arange(L, dtype=np.int64)[None, :]
+    causal = j <= t
+    same_block = (j // b) == (t // b)
+    anchor = ((t // b) >= 1) & (j < b_a)
+    return causal & (same_block | anchor)
+
+
+def star_mask(L: int, b: int, b_a: int) -> np.ndarray:
+    """The full ``L x L`` Star mask (small ``L`` only)."""
+    return star_mask_rows(L, b, b_a, np.arange(L))
+
+
+# ---------------------------------------------------------------------------
+# The attention equation ([P2] "The Attention Decomposition").
+# ---------------------------------------------------------------------------
+def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                     mask: np.ndarray, scale: float):
+    """Softmax attention of rows ``q`` [R, D] over keys ``k``/``v`` [N, D].
+
+    Only keys with ``mask[r, j]`` True take part.  Returns ``(O [R, D],
+    LSE [R])`` in float64, where ``LSE = log sum_j exp(scale * q.k_j)`` over
+    the visible keys (natural log of the scaled logits) and ``O`` is the
+    softmax-weighted mean of the visible values.  A row with no visible key
+    gets ``O = 0`` and ``LSE = -inf``.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    x = scale * (q @ k.T)
+    x = np.where(mask, x, NEG_INF)
+    m = x.max(axis=1, initial=NEG_INF)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(x - m_safe[:, None])
+    ssum = e.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        lse = np.where(empty, NEG_INF, m_safe + np.log(ssum))
+        o = np.where(empty[:, None], 0.0, (e @ v) / ssum[:, None])
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Phase 1: context encoding.
+# ---------------------------------------------------------------------------
+def ctx_encode(Q: np.ndarray, K: np.ndarray, V: np.ndarray, b: int, b_a: int,
+               scale: float, rows=None):
+    """Phase-1 outputs for Q [B, Hq, L, D], K/V [B, Hkv, L, D] (float64).
+
+    For every context token ``t`` and q head ``h`` (kv head ``h // G``), the
+    output is softmax attention over the tokens the Star mask lets ``t`` see
+    ([P2] Phase 1 Step 4).  ``rows`` restricts the computation to the given
+    token indices (the others are left as NaN); the result for a row does not
+    depend on which other rows are computed.
+
+    Returns ``(O [B, Hq, L, D], LSE [B, Hq, L])``.
+    """
+    Bn, Hq, L, D = Q.shape
+    Hkv = K.shape[1]
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    rows = np.arange(L) if rows is None else np.asarray(rows, np.int64)
+    O = np.full((Bn, Hq, L, D), np.nan)
+    LSE = np.full((Bn, Hq, L), np.nan)
+    if len(rows) == 0:
+        return O, LSE
+    mask = star_mask_rows(L, b, b_a, rows)
+    # Only the union of visible columns is needed; gather them once.
+    cols = np.nonzero(mask.any(axis=0))[0]
+    sub = mask[:, cols]
+    for bi in range(Bn):
+        for h in range(Hq):
+            g = h // G
+            o, lse = masked_attention(Q[bi, h, rows], K[bi, g, cols],
+                                      V[bi, g, cols], sub, scale)
+            O[bi, h, rows] = o
+            LSE[bi, h, rows] = lse
+    return O, LSE
+
+
+def cache_segments(K: np.ndarray, V: np.ndarray, b: int):
+    """Per-block KV-cache segments kept after phase 1.
+
+    [P2] Phase 1 Step 5 / [P3] Phase 1 last bullet: block ``i`` keeps only
+    the K/V of its own tokens; the anchor's K/V is discarded, so every
+    context token is cached exactly once.  Returns a list of
+    ``(start, length, K_seg [B, Hkv, len, D], V_seg [B, Hkv, len, D])``.
+    Works on any dtype (bit-exact comparisons use the raw bf16 bits).
+    """
+    L = K.shape[2]
+    return [(s, n, K[:, :, s:s + n], V[:, :, s:s + n])
+            for (s, n) in block_table(L, b)]
+
+
+# ---------------------------------------------------------------------------
+# Phase 2: local partials, their merge, query prefill and decode.
+# ---------------------------------------------------------------------------
+def local_partial(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                  mask: np.ndarray | None = None):
+    """One partition's local attention ``A_h`` and its log-sum-exp ``s_h``.
+
+    [P2] Phase 2 Step 3 / [P3] Phase 2: ``A_h`` is the softmax attention of
+    ``q`` [R, D] over this partition's keys only; ``s_h`` (carried here in
+    log space) is ``log sum_k exp(q.k / sqrt(d))`` over the same keys.  An
+    empty partition gives ``A_h = 0``, ``s_h = -inf``.
+    """
+    if mask is None:
+        mask = np.ones((q.shape[0], k.shape[0]), dtype=bool)
+    return masked_attention(q, k, v, mask, scale)
+
+
+def lse_merge(A: np.ndarray, s: np.ndarray):
+    """Merge partials ``A [P, R, D]``, ``s [P, R]`` into ``(A [R, D], s [R])``.
+
+    [P3] Phase 2: ``s_global = sum_h s_h`` and ``A_global = sum_h (s_h /
+    s_global) A_h`` with raw exponent sums; written here in log space as
+    [P2] Step 5 intends: ``s = log sum_h exp(s_h)`` and
+    ``A = sum_h exp(s_h - s) A_h``.  The maximum is subtracted before
+    exponentiating; partitions with ``s_h = -inf`` contribute nothing.
+    """
+    A = np.asarray(A, np.float64)
+    s = np.asarray(s, np.float64)
+    m = s.max(axis=0)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    w = np.exp(s - m_safe[None])                  # exp(s_h - m), 0 for -inf
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s_glob = np.where(empty, NEG_INF, m_safe + np.log(tot))
+        coef = np.where(empty[None], 0.0, np.exp(s - np.where(empty, 0.0, s_glob)[None]))
+    A_glob = np.einsum("pr,prd->rd", coef, A)
+    return A_glob, s_glob
+
+
+def _context_keys(segments, bi, g):
+    """Concatenation of every context segment's cache for (batch, kv head)."""
+    ks = [seg[2][bi, g] for seg in segments]
+    vs = [seg[3][bi, g] for seg in segments]
+    return np.concatenate(ks, axis=0), np.concatenate(vs, axis=0)
+
+
+def query_attend(q_rows: np.ndarray, segments, qk_region: np.ndarray,
+                 qv_region: np.ndarray, visible_q: np.ndarray, scale: float):
+    """Exact global attention of phase-2 rows over the whole cache.
+
+    ``q_rows`` [B, Hq, R, D]; ``segments`` from :func:`cache_segments`;
+    ``qk_region``/``qv_region`` [B, Hkv, Nq, D] is the query region's cache
+    (query and generated tokens, [P2] Phase 2 Step 7); row ``r`` sees every
+    context token and the first ``visible_q[r]`` query-region rows.
+
+    This is the definition the distributed softmax reproduces exactly
+    ([P2] Phase 2, the partition identity): one softmax over
+    ``[context cache || query region]``.  Returns ``(O, LSE)`` float64.
+    """
+    Bn, Hq, R, D = q_rows.shape
+    Hkv = qk_region.shape[1]
+    G = Hq // Hkv
+    Nq = qk_region.shape[2]
+    O = np.zeros((Bn, Hq, R, D))
+    LSE = np.zeros((Bn, Hq, R))
+    for bi in range(Bn):
+        for g in range(Hkv):
+            kc, vc = _context_keys(segments, bi, g)
+            k_all = np.concatenate([kc, qk_region[bi, g]], axis=0)
+            v_all = np.concatenate([vc, qv_region[bi, g]], axis=0)
+            Lc = kc.shape[0]
+            mask = np.ones((R, Lc + Nq), dtype=bool)
+            mask[:, Lc:] = np.arange(Nq)[None, :] < np.asarray(visible_q)[:, None]
+            for h in range(g * G, (g + 1) * G):
+                o, lse = masked_attention(q_rows[bi, h], k_all, v_all, mask, scale)
+                O[bi, h] = o
+                LSE[bi, h] = lse
+    return O, LSE
+
+
+def query_prefill(Qq, Kq, Vq, segments, qk_region, qv_region, q_len0: int,
+                  scale: float):
+    """Phase-2 query prefill.
+
+    Appends ``Kq``/``Vq`` [B, Hkv, lq, D] to the query region (which held
+    ``q_len0`` rows) and attends each query row ``r`` to all context segments
+    plus query-region rows ``0..q_len0 + r``.  Returns ``(O, LSE, qk_region,
+    qv_region)`` with the regions updated (copies).
+    """
+    lq = Qq.shape[2]
+    qk = qk_region.copy()
+    qv = qv_region.copy()
+    qk[:, :, q_len0:q_len0 + lq] = Kq
+    qv[:, :, q_len0:q_len0 + lq] = Vq
+    vis = q_len0 + np.arange(lq) + 1
+    O, LSE = query_attend(Qq, segments, qk, qv, vis, scale)
+    return O, LSE, qk, qv
+
+
+def decode_step(q, k, v, segments, qk_region, qv_region, q_len: int,
+                scale: float):
+    """One phase-2 generation step for q [B, Hq, 1, D], k/v [B, Hkv, 1, D].
+
+    [P2] Phase 2 Step 7: the new token's K/V is appended to the query region
+    only (at row ``q_len``), then the token attends to every context token
+    and query-region rows ``0..q_len`` (itself included).
+    """
+    qk = qk_region.copy()
+    qv = qv_region.copy()
+    qk[:, :, q_len] = k[:, :, 0]
+    qv[:, :, q_len] = v[:, :, 0]
+    O, LSE = query_attend(q, segments, qk, qv, np.array([q_len + 1]), scale)
+    return O, LSE, qk, qv
+
+
+def phase2_partials(q_rows, segments, qk_region, qv_region, visible_q, scale):
+    """Second, independent form of phase 2: per-segment partials + merge.
+
+    Each context segment ``h`` gives ``(A_h, s_h)`` ([P2] Phase 2 Step 3); the
+    query region is one more partition with its causal visibility; the
+    partials are merged with :func:`lse_merge` ([P2] Step 5).  Used only to
+    check the partition identity against :func:`query_attend`.
+    """
+    Bn, Hq, R, D = q_rows.shape
+    Hkv = qk_region.shape[1]
+    G = Hq // Hkv
+    Nq = qk_region.shape[2]
+    O = np.zeros((Bn, Hq, R, D))
+    LSE = np.zeros((Bn, Hq, R))
+    qmask = np.arange(Nq)[None, :] < np.asarray(visible_q)[:, None]
+    for bi in range(Bn):
+        for h in range(Hq):
+            g = h // G
+            As, ss = [], []
+            for seg in segments:
+                a, s = local_partial(q_rows[bi, h], seg[2][bi, g], seg[3][bi, g], scale)
+                As.append(a)
+                ss.append(s)
+            a, s = local_partial(q_rows[bi, h], qk_region[bi, g], qv_region[bi, g],
+                                 scale, qmask)
+            As.append(a)
+            ss.append(s)
+            o, lse = lse_merge(np.stack(As), np.stack(ss))
+            O[bi, h] = o
+            LSE[bi, h] = lse
+    return O, LSE

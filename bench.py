@@ -1,0 +1,385 @@
+"""Benchmark of the Star Attention two-phase hot path on B200.
+
+One step = the whole path over one synthetic batch of the Llama-3.1-8B
+attention shape at 32K context (H_q=32, H_kv=8, D=128, b = b_a = 8192, 4
+blocks; 64 query tokens, 32 decode steps): phase-1 context encoding, phase-2
+query prefill, and every decode step.
+
+Reported (one JSON line from rank 0):
+  value      -- phase-1 context-encode tokens/s (B*L / encode time), all ranks
+  decode     -- phase-2 decode tokens/s and its HBM roofline
+  roofline   -- phase-1 kernel against the measured bf16 dense peak
+  e2e        -- the same metric through the public API with pinned-host
+                inputs copied in and results copied out inside the timed region
+  cpu_baseline -- the fp64 oracle on a bounded sample, extrapolated
+
+L2 is flushed (a 256 MB write) before every timed kernel region; the flush is
+outside the CUDA-event brackets.  Multi-GPU runs are independent replicas
+(the single-GPU path has no exchange step): value = all ranks' tokens / the
+slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this path
+has) on a bounded sample of the same workload and prints the same line with
+"impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "8b-32k"
+METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roofline"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def phase1_flops(w):
+    """Algorithmic flops of phase 1: 4*D per visible (query, key) pair of block rows."""
+    pairs = 0
+    for i in range(w.n_blocks):
+        n = min(w.b, w.L - i * w.b)
+        pairs += n * (n + 1) // 2 + (w.b_a * n if i > 0 else 0)
+    return 4 * w.D * w.Hq * w.B * pairs, pairs
+
+
+def decode_bytes(w, t):
+    """Algorithmic bytes of decode step t: the K and V of every cached row."""
+    return w.B * w.Hkv * (w.L + w.lq + t + 1) * w.D * 2 * 2
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"star_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(w, x, budget_s=12.0):
+    """Time the fp64 oracle on sampled phase-1 rows and phase-2 decode rows.
+
+    Returns (ctx tok/s, decode tok/s, sample description, threads).  Phase-1
+    time is extrapolated to the whole layer by visible (query, key) pairs; the
+    decode time by the number of heads sampled.
+    """
+    import numpy as np
+    from oracle import star_oracle as so
+    rng = np.random.default_rng(0)
+    _, total_pairs = phase1_flops(w)
+    total_pairs *= w.Hq * w.B
+    g = 0
+    hs = slice(0, w.G)
+    Qc, Kc, Vc = x["Qc"][0:1, hs], x["Kc"][0:1, g:g + 1], x["Vc"][0:1, g:g + 1]
+    t_p1 = 0.0
+    pairs = 0
+    nrows = 0
+    blocks = so.block_table(w.L, w.b)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s * 0.6:
+        i = int(rng.integers(0, len(blocks)))
+        s, n = blocks[i]
+        rows = np.sort(rng.integers(s, s + n, size=16))
+        a = time.perf_counter()
+        so.ctx_encode(Qc, Kc, Vc, w.b, w.b_a, w.scale, rows=rows)
+        t_p1 += time.perf_counter() - a
+        vis = (rows - s + 1) + (w.b_a if i > 0 else 0)
+        pairs += int(vis.sum()) * w.G
+        nrows += len(rows)
+    ctx_time = t_p1 * total_pairs / pairs
+    # decode: one step of one kv group against the full cache, extrapolated to all heads
+    kc, vc = so._f64(Kc), so._f64(Vc)
+    segs = so.cache_segments(kc, vc, w.b)
+    qk = so._f64(x["Kq"][0:1, g:g + 1])
+    qv = so._f64(x["Vq"][0:1, g:g + 1])
+    a = time.perf_counter()
+    steps = 0
+    while steps < 2 or time.perf_counter() - a < budget_s * 0.2:
+        so.query_attend(x["Qq"][0:1, hs, :1], segs, qk, qv, np.array([1]), w.scale)
+        steps += 1
+    t_dec = (time.perf_counter() - a) / steps * (w.Hkv * w.B)
+    threads = _blas_threads()
+    sample = (f"phase 1: {nrows} rows x {w.G} heads of kv group 0 "
+              f"(extrapolated by visible (q,k) pairs to {w.B}x{w.Hq} heads x {w.L} rows); "
+              f"decode: {steps} one-token steps of kv group 0 vs the {w.L}-token cache "
+              f"(x{w.B * w.Hkv} kv groups)")
+    return w.B * w.L / ctx_time, 1.0 / t_dec, sample, threads
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from block_sparse_long_phase_b200 import workloads as wl
+    w = wl.get(WORKLOAD)
+    x = wl.make_inputs(w, "cpu", with_decode=False)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, x, budget_s=min(per_step, 4.0))
+    vals, decs = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, d, sample, threads = cpu_oracle_sample(w, x, budget_s=per_step)
+        vals.append(v)
+        decs.append(d)
+    el = time.perf_counter() - t0
+    v = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "ctx tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
+                   "block": w.b, "anchor": w.b_a, "lq": w.lq, "decode_steps": w.T},
+        "decode": {"value": statistics.median(decs), "unit": "decode tok/s"},
+        "cpu_baseline": {"value": v, "unit": "ctx tok/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "ctx tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del torch
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="star", choices=["star", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    w = wl.get(args.workload)
+    x = wl.make_inputs(w, dev)
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+    O = torch.empty((w.B, w.Hq, w.L, w.D), dtype=torch.bfloat16, device=dev)
+    LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    Oq = torch.empty((w.B, w.Hq, w.lq, w.D), dtype=torch.bfloat16, device=dev)
+    LSEq = torch.empty((w.B, w.Hq, w.lq), dtype=torch.float32, device=dev)
+    od = torch.empty((w.T, w.B, w.Hq, 1, w.D), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((w.T, w.B, w.Hq), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(times):
+        flush.fill_(1.0)
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"], O, LSE)
+        e1.record(stream)
+        flush.fill_(2.0)
+        e2, e3 = ev(), ev()
+        e2.record(stream)
+        cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"], Oq, LSEq)
+        e3.record(stream)
+        dec = []
+        for t in range(w.T):
+            flush.fill_(3.0)
+            a, b = ev(), ev()
+            a.record(stream)
+            cache.star_decode_step(x["qd"][t], x["kd"][t], x["vd"][t], od[t], lsed[t])
+            b.record(stream)
+            dec.append((a, b))
+        times.append(((e0, e1), (e2, e3), dec))
+
+    for _ in range(args.warmup):
+        step([])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = Clocks(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter()
+    times = []
+    for _ in range(args.steps):
+        step(times)
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    enc_ms = [a.elapsed_time(b) for (a, b), _, _ in times]
+    pre_ms = [a.elapsed_time(b) for _, (a, b), _ in times]
+    dec_ms = [[a.elapsed_time(b) for a, b in d] for _, _, d in times]
+    step_ms = [e + p + sum(d) for e, p, d in zip(enc_ms, pre_ms, dec_ms)]
+    enc_total = sum(enc_ms)
+    dec_total = sum(sum(d) for d in dec_ms)
+    tot = torch.tensor([enc_total, dec_total, sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
+    enc_total, dec_total, step_total = tot.tolist()
+
+    # ---- end to end through the public API (pinned host buffers) ----------------
+    e2e = None
+    if not args.no_e2e:
+        hx = {k: v.cpu().pin_memory() for k, v in x.items() if k in ("Qc", "Kc", "Vc")}
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        hL = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
+        dx = {k: torch.empty_like(x[k]) for k in hx}
+        e2e_ms = []
+        for it in range(args.warmup + args.steps):
+            flush.fill_(4.0)
+            a, b = ev(), ev()
+            a.record(stream)
+            for k in hx:
+                dx[k].copy_(hx[k], non_blocking=True)
+            cache.star_ctx_encode(dx["Qc"], dx["Kc"], dx["Vc"], O, LSE)
+            hO.copy_(O, non_blocking=True)
+            hL.copy_(LSE, non_blocking=True)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= args.warmup:
+                e2e_ms.append(a.elapsed_time(b))
+        t = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        h2d = sum(v.numel() * v.element_size() for v in hx.values())
+        d2h = hO.numel() * 2 + hL.numel() * 4
+        e2e = {"value": world * w.B * w.L * args.steps / (t.item() / 1e3), "unit": "ctx tok/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "what": "H2D of Q,K,V from pinned host + star_ctx_encode + D2H of O,LSE"}
+
+    pk = peaks()
+    flops, _ = phase1_flops(w)
+    enc_avg_s = enc_total / args.steps / 1e3
+    achieved_tf = flops / enc_avg_s / 1e12
+    dbytes = sum(decode_bytes(w, t) for t in range(w.T))
+    dec_avg_s = dec_total / args.steps / 1e3
+    achieved_gbs = dbytes / dec_avg_s / 1e9
+    value = world * w.B * w.L / enc_avg_s
+    line = {
+        "metric": METRIC, "value": value, "unit": "ctx tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
+                   "block": w.b, "anchor": w.b_a, "lq": w.lq, "decode_steps": w.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (256 MB write) before every timed kernel region"},
+        "decode": {"value": world * w.B * w.T / dec_avg_s, "unit": "decode tok/s",
+                   "us_per_step": dec_avg_s / w.T * 1e6,
+                   "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"],
+                                "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
+                                "traffic": None, "peak_source": pk["source"]}},
+        "prefill_ms": sum(pre_ms) / args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"], "traffic": None,
+                     "kernel": "phase-1 context encode", "flops_per_launch": flops,
+                     "peak_source": pk["source"] + " burst bf16 dense"},
+        "clocks": clk,
+        "gpu_launches": args.steps * (1 + 2 + w.T),
+        "wall_s_timed_region": wall,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, d, sample, threads = cpu_oracle_sample(w, x)
+        line["cpu_baseline"] = {"value": v, "unit": "ctx tok/s", "cores": threads, "kind": "oracle",
+                                "sample": sample, "decode_value": d}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    cache.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

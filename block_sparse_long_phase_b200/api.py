@@ -1,0 +1,190 @@
+"""Thin PyTorch binding of libstar: argument marshalling only.
+
+Every step of the path runs in libstar's kernels; this module checks tensor
+shapes and dtypes, allocates outputs with torch (device memory is PyTorch's),
+and passes raw pointers and torch's current CUDA stream through the C ABI.
+The names follow the C entry points.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _abi
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, shape, dtype, name):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libstar has no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+@dataclass
+class Segment:
+    k: int          # device pointer
+    v: int
+    start: int
+    len: int
+    cap: int
+
+
+class StarCache:
+    """A Star Attention KV cache: per-block context segments + query region.
+
+    Wraps ``star_cache_create``; the cache lives on the current CUDA device.
+    """
+
+    def __init__(self, B, Hq, Hkv, D, L, block, anchor, q_cap, scale=0.0):
+        if not torch.cuda.is_available():
+            raise RuntimeError("libstar needs a CUDA device; there is no CPU fallback")
+        self.lib = _abi.load()
+        self.params = _abi.StarParams(B, Hq, Hkv, D, L, block, anchor, q_cap, float(scale))
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        h = ctypes.c_void_p()
+        _abi.check(self.lib.star_cache_create(ctypes.byref(self.params), ctypes.byref(h)))
+        self.handle = h
+        self.B, self.Hq, self.Hkv, self.D, self.L = B, Hq, Hkv, D, L
+        self.block, self.anchor, self.q_cap = block, anchor, q_cap
+
+    # -- lifetime ------------------------------------------------------------
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            _abi.check(self.lib.star_cache_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # -- introspection -------------------------------------------------------
+    @property
+    def num_segments(self) -> int:
+        return self.lib.star_cache_num_segments(self.handle)
+
+    def segment(self, i: int) -> Segment:
+        k, v = ctypes.c_void_p(), ctypes.c_void_p()
+        s, n, c = ctypes.c_longlong(), ctypes.c_longlong(), ctypes.c_longlong()
+        _abi.check(self.lib.star_cache_segment(self.handle, i, ctypes.byref(k), ctypes.byref(v),
+                                               ctypes.byref(s), ctypes.byref(n), ctypes.byref(c)))
+        return Segment(k.value, v.value, s.value, n.value, c.value)
+
+    def segment_tensors(self, i: int):
+        """(K, V) views of segment ``i`` as bf16 tensors [B, Hkv, cap, D]."""
+        seg = self.segment(i)
+        n = self.B * self.Hkv * seg.cap * self.D
+        out = []
+        for p in (seg.k, seg.v):
+            t = _tensor_from_ptr(p, n, self.device).view(self.B, self.Hkv, seg.cap, self.D)
+            out.append(t)
+        return out[0], out[1], seg
+
+    @property
+    def q_len(self) -> int:
+        return self.segment(self.num_segments - 1).len
+
+    def reset_query(self):
+        _abi.check(self.lib.star_cache_reset_query(self.handle))
+
+    # -- the hot path --------------------------------------------------------
+    def star_ctx_encode(self, Q, K, V, O=None, LSE=None):
+        B, Hq, Hkv, D, L = self.B, self.Hq, self.Hkv, self.D, self.L
+        _need(Q, (B, Hq, L, D), torch.bfloat16, "Q")
+        _need(K, (B, Hkv, L, D), torch.bfloat16, "K")
+        _need(V, (B, Hkv, L, D), torch.bfloat16, "V")
+        if O is None:
+            O = torch.empty((B, Hq, L, D), dtype=torch.bfloat16, device=Q.device)
+        if LSE is None:
+            LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
+        _need(O, (B, Hq, L, D), torch.bfloat16, "O")
+        _need(LSE, (B, Hq, L), torch.float32, "LSE")
+        _abi.check(self.lib.star_ctx_encode(self.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                            _ptr(LSE), _stream(Q.device)))
+        return O, LSE
+
+    def star_query_prefill(self, Q, K, V, O=None, LSE=None):
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        lq = Q.shape[2]
+        _need(Q, (B, Hq, lq, D), torch.bfloat16, "Q")
+        _need(K, (B, Hkv, lq, D), torch.bfloat16, "K")
+        _need(V, (B, Hkv, lq, D), torch.bfloat16, "V")
+        if O is None:
+            O = torch.empty((B, Hq, lq, D), dtype=torch.bfloat16, device=Q.device)
+        if LSE is None:
+            LSE = torch.empty((B, Hq, lq), dtype=torch.float32, device=Q.device)
+        _need(O, (B, Hq, lq, D), torch.bfloat16, "O")
+        _need(LSE, (B, Hq, lq), torch.float32, "LSE")
+        _abi.check(self.lib.star_query_prefill(self.handle, lq, _ptr(Q), _ptr(K), _ptr(V),
+                                               _ptr(O), _ptr(LSE), _stream(Q.device)))
+        return O, LSE
+
+    def star_decode_step(self, q, k, v, o=None, lse=None):
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        _need(q, (B, Hq, 1, D), torch.bfloat16, "q")
+        _need(k, (B, Hkv, 1, D), torch.bfloat16, "k")
+        _need(v, (B, Hkv, 1, D), torch.bfloat16, "v")
+        if o is None:
+            o = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
+        if lse is None:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        _need(o, (B, Hq, 1, D), torch.bfloat16, "o")
+        _need(lse, (B, Hq), torch.float32, "lse")
+        _abi.check(self.lib.star_decode_step(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                             _ptr(lse), _stream(q.device)))
+        return o, lse
+
+
+def star_lse_merge(A: torch.Tensor, s: torch.Tensor, out_A=None, out_s=None):
+    """Merge partials A [P, R, D], s [P, R] (float32, CUDA) -> ([R, D], [R])."""
+    lib = _abi.load()
+    P, R, D = A.shape
+    _need(A, (P, R, D), torch.float32, "A")
+    _need(s, (P, R), torch.float32, "s")
+    if out_A is None:
+        out_A = torch.empty((R, D), dtype=torch.float32, device=A.device)
+    if out_s is None:
+        out_s = torch.empty((R,), dtype=torch.float32, device=A.device)
+    _need(out_A, (R, D), torch.float32, "out_A")
+    _need(out_s, (R,), torch.float32, "out_s")
+    _abi.check(lib.star_lse_merge(P, R, D, _ptr(A), _ptr(s), _ptr(out_A), _ptr(out_s),
+                                  _stream(A.device)))
+    return out_A, out_s
+
+
+def _tensor_from_ptr(ptr: int, n_elems: int, device) -> torch.Tensor:
+    """A bf16 view of ``n_elems`` elements of device memory owned by libstar."""
+
+    class _CudaArray:
+        def __init__(self):
+            self.__cuda_array_interface__ = {
+                "shape": (n_elems,), "typestr": "<u2", "data": (ptr, False), "version": 3,
+                "strides": None,
+            }
+
+    t = torch.as_tensor(_CudaArray(), device=device)
+    return t.view(torch.bfloat16)

@@ -1,0 +1,334 @@
+// C ABI of libstar: argument validation, the segmented KV cache, work plans
+// and kernel launches.  Declarations and contracts: include/star_attention.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../../include/star_attention.h"
+#include "star_internal.h"
+
+using star::bf16;
+
+struct star_cache {
+  star_params p;
+  star::CacheView view;
+  star::Scratch scratch;
+  long long q_len;          // query-region rows in use (host-side; calls are stream-ordered)
+  int device;
+  int num_sms;
+  void* block;              // the one cudaMalloc holding everything below
+  int4* ctx_work;           // phase-1 work list, longest first
+  int n_ctx_work;
+};
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(STAR_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long round_up(long long x, long long m) { return (x + m - 1) / m * m; }
+
+constexpr int kTileRows = 64;
+
+// ---- phase-2 plans --------------------------------------------------------
+star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
+  const star::CacheView& v = c->view;
+  star::PrefillPlan pl{};
+  pl.row_tiles = (int)((v.G * (long long)lq + kTileRows - 1) / kTileRows);
+  const long long bg = (long long)v.B * v.Hkv;
+  const long long target = 2LL * c->num_sms * 2;  // ~2 waves of 2 CTAs per SM
+  long long want = std::max(1LL, (target + bg * pl.row_tiles - 1) / (bg * pl.row_tiles));
+  long long chunk_len = std::max<long long>(256, round_up((v.L + want - 1) / want, kTileRows));
+  for (;;) {
+    int n = 0;
+    for (int s = 0; s < v.n_seg; ++s) n += (int)((star::seg_len(v, s) + chunk_len - 1) / chunk_len);
+    if (n + 1 <= star::kMaxPrefillChunks) break;
+    chunk_len *= 2;
+  }
+  int n = 0;
+  for (int s = 0; s < v.n_seg; ++s) {
+    const long long len = star::seg_len(v, s);
+    for (long long st = 0; st < len; st += chunk_len) {
+      pl.chunk[n].seg = s;
+      pl.chunk[n].start = (int)st;
+      pl.chunk[n].len = (int)std::min(chunk_len, len - st);
+      ++n;
+    }
+  }
+  pl.chunk[n].seg = -1;
+  pl.chunk[n].start = 0;
+  pl.chunk[n].len = (int)(len0 + lq);
+  pl.n_chunks = n + 1;
+  return pl;
+}
+
+star::DecodePlan plan_decode(const star_cache* c, long long len0) {
+  const star::CacheView& v = c->view;
+  const long long total = v.L + len0 + 1;
+  const long long bg = (long long)v.B * v.Hkv;
+  long long cph = std::max(1LL, (2LL * c->num_sms) / bg);
+  long long rows = round_up((total + cph - 1) / cph, 64);
+  cph = (total + rows - 1) / rows;
+  star::DecodePlan pl;
+  pl.chunks_per_head = (int)cph;
+  pl.chunk_rows = rows;
+  return pl;
+}
+
+// Phase-1 work list: (b*Hq + h, block, q tile), sorted by the number of K/V
+// tiles each item streams, longest first, so the tail of the grid is short.
+std::vector<int4> plan_ctx(const star_params& p) {
+  std::vector<int4> w;
+  const long long n = (p.L + p.block - 1) / p.block;
+  struct Item { long long cost; int4 v; };
+  std::vector<Item> items;
+  for (int blk = 0; blk < n; ++blk) {
+    const long long bs = (long long)blk * p.block;
+    const long long len = std::min<long long>(p.block, p.L - bs);
+    const long long tiles = (len + kTileRows - 1) / kTileRows;
+    const long long anchor_tiles = blk > 0 ? (p.anchor + kTileRows - 1) / kTileRows : 0;
+    for (int qt = 0; qt < tiles; ++qt)
+      for (int b = 0; b < p.B; ++b)
+        for (int h = 0; h < p.Hq; ++h)
+          items.push_back({anchor_tiles + qt + 1, make_int4(b * p.Hq + h, blk, qt, 0)});
+  }
+  std::stable_sort(items.begin(), items.end(),
+                   [](const Item& a, const Item& b) { return a.cost > b.cost; });
+  w.reserve(items.size());
+  for (auto& it : items) w.push_back(it.v);
+  return w;
+}
+
+int validate_params(const star_params* p) {
+  if (!p) return fail(STAR_EINVAL, "params is NULL");
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1) return fail(STAR_EINVAL, "B, Hq, Hkv must be >= 1");
+  if (p->Hq % p->Hkv) return fail(STAR_EINVAL, "Hq (%d) must be a multiple of Hkv (%d)", p->Hq, p->Hkv);
+  if (p->D != 64 && p->D != 128) return fail(STAR_EUNSUPPORTED, "head dim %d not in {64, 128}", p->D);
+  if (p->Hq / p->Hkv > 16) return fail(STAR_EUNSUPPORTED, "group size %d > 16", p->Hq / p->Hkv);
+  if (p->L < 1) return fail(STAR_EINVAL, "context length must be >= 1");
+  if (p->block < 1) return fail(STAR_EINVAL, "block size must be >= 1");
+  if (p->anchor < 0 || p->anchor > p->block)
+    return fail(STAR_EINVAL, "anchor %d must satisfy 0 <= b_a <= b (%d)", p->anchor, p->block);
+  if (p->q_cap < 1) return fail(STAR_EINVAL, "q_cap must be >= 1");
+  if (p->L + p->q_cap + 1 > 0x7fffffffLL) return fail(STAR_EINVAL, "L + q_cap too large");
+  if ((p->L + p->block - 1) / p->block > 0x7fff) return fail(STAR_EINVAL, "too many blocks");
+  return STAR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* star_last_error(void) { return g_err; }
+const char* star_version(void) { return "libstar 0.1 (sm_100a)"; }
+
+int star_cache_create(const star_params* p, star_cache** out) {
+  if (!out) return fail(STAR_EINVAL, "out is NULL");
+  *out = nullptr;
+  int rc = validate_params(p);
+  if (rc) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10) return fail(STAR_EUNSUPPORTED, "device is sm_%d%d, need sm_100", prop.major, prop.minor);
+
+  star_cache* c = new star_cache();
+  c->p = *p;
+  if (c->p.scale <= 0.f) c->p.scale = 1.0f / sqrtf((float)p->D);
+  c->device = dev;
+  c->num_sms = prop.multiProcessorCount;
+  star::CacheView& v = c->view;
+  v.B = p->B; v.Hq = p->Hq; v.Hkv = p->Hkv; v.D = p->D; v.G = p->Hq / p->Hkv;
+  v.L = p->L; v.b = p->block; v.b_a = p->anchor;
+  v.n_seg = (int)((p->L + p->block - 1) / p->block);
+  v.q_cap = p->q_cap;
+
+  // Scratch sizing: the largest prefill plan over every lq the query region
+  // admits, and the decode plan at the fullest query region.
+  long long partA = 0, partS = 0;
+  for (int lq = 1; lq <= p->q_cap; ++lq) {
+    star::PrefillPlan pl = plan_prefill(c, lq, 0);
+    const long long rows = (long long)v.B * v.Hkv * pl.n_chunks * v.G * lq;
+    partA = std::max(partA, rows * v.D);
+    partS = std::max(partS, rows);
+  }
+  for (long long len0 = 0; len0 < p->q_cap; len0 += std::max(1, p->q_cap / 64)) {
+    star::DecodePlan pl = plan_decode(c, len0);
+    const long long rows = (long long)v.B * v.Hkv * pl.chunks_per_head * v.G;
+    partA = std::max(partA, rows * v.D);
+    partS = std::max(partS, rows);
+  }
+  {
+    star::DecodePlan pl = plan_decode(c, p->q_cap - 1);
+    const long long rows = (long long)v.B * v.Hkv * pl.chunks_per_head * v.G;
+    partA = std::max(partA, rows * v.D);
+    partS = std::max(partS, rows);
+  }
+  std::vector<int4> work = plan_ctx(c->p);
+  c->n_ctx_work = (int)work.size();
+
+  const long long kv_ctx = (long long)p->B * p->Hkv * p->L * p->D;        // elements
+  const long long kv_q = (long long)p->B * p->Hkv * p->q_cap * p->D;
+  const long long n_tickets = (long long)p->B * p->Hkv;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = (off + bytes + 255) & ~size_t(255); return o; };
+  const size_t o_ck = take(kv_ctx * 2), o_cv = take(kv_ctx * 2);
+  const size_t o_qk = take(kv_q * 2), o_qv = take(kv_q * 2);
+  const size_t o_pa = take(partA * 4), o_ps = take(partS * 4);
+  const size_t o_t = take(n_tickets * 4);
+  const size_t o_w = take(work.size() * sizeof(int4));
+  e = cudaMalloc(&c->block, off);
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(STAR_ENOMEM, "cudaMalloc(%zu bytes): %s", off, cudaGetErrorString(e));
+  }
+  char* base = static_cast<char*>(c->block);
+  v.ctxK = reinterpret_cast<bf16*>(base + o_ck);
+  v.ctxV = reinterpret_cast<bf16*>(base + o_cv);
+  v.qK = reinterpret_cast<bf16*>(base + o_qk);
+  v.qV = reinterpret_cast<bf16*>(base + o_qv);
+  c->scratch.partA = reinterpret_cast<float*>(base + o_pa);
+  c->scratch.partS = reinterpret_cast<float*>(base + o_ps);
+  c->scratch.tickets = reinterpret_cast<unsigned*>(base + o_t);
+  c->scratch.partA_elems = partA;
+  c->scratch.partS_elems = partS;
+  c->scratch.n_tickets = (int)n_tickets;
+  c->ctx_work = reinterpret_cast<int4*>(base + o_w);
+  e = cudaMemset(c->scratch.tickets, 0, n_tickets * 4);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(c->ctx_work, work.data(), work.size() * sizeof(int4), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(c->block);
+    delete c;
+    return cuda_fail(e, "cache initialisation");
+  }
+  c->q_len = 0;
+  *out = c;
+  g_err[0] = 0;
+  return STAR_OK;
+}
+
+int star_cache_destroy(star_cache* c) {
+  if (!c) return STAR_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t f = cudaFree(c->block);
+  delete c;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  if (f != cudaSuccess) return cuda_fail(f, "cudaFree");
+  return STAR_OK;
+}
+
+int star_cache_num_segments(const star_cache* c) { return c ? c->view.n_seg + 1 : 0; }
+
+int star_cache_segment(const star_cache* c, int seg, void** k, void** v, long long* start,
+                       long long* len, long long* cap) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  const star::CacheView& w = c->view;
+  if (seg < 0 || seg > w.n_seg) return fail(STAR_EINVAL, "segment %d out of range", seg);
+  if (seg == w.n_seg) {
+    if (k) *k = w.qK;
+    if (v) *v = w.qV;
+    if (start) *start = w.L;
+    if (len) *len = c->q_len;
+    if (cap) *cap = w.q_cap;
+    return STAR_OK;
+  }
+  const long long off = (long long)seg * w.B * w.Hkv * (long long)w.b * w.D;
+  if (k) *k = w.ctxK + off;
+  if (v) *v = w.ctxV + off;
+  if (start) *start = (long long)seg * w.b;
+  if (len) *len = star::seg_len(w, seg);
+  if (cap) *cap = star::seg_len(w, seg);
+  return STAR_OK;
+}
+
+int star_cache_reset_query(star_cache* c) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  c->q_len = 0;
+  return STAR_OK;
+}
+
+int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
+                    float* LSE, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  cudaError_t e = star::launch_ctx_encode_mma(
+      c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+      static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work,
+      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
+  c->q_len = 0;
+  return STAR_OK;
+}
+
+int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K, const void* V,
+                       void* O, float* LSE, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (lq < 1) return fail(STAR_EINVAL, "lq must be >= 1");
+  if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (c->q_len + lq > c->view.q_cap)
+    return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, c->view.q_cap);
+  star::PrefillPlan pl = plan_prefill(c, lq, c->q_len);
+  cudaError_t e = star::launch_query_prefill_mma(
+      c->view, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
+      static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
+      c->scratch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_query_prefill launch");
+  c->q_len += lq;
+  return STAR_OK;
+}
+
+int star_decode_step(star_cache* c, const void* q, const void* k, const void* v, void* o,
+                     float* lse, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (!q || !k || !v || !o || !lse) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (c->q_len + 1 > c->view.q_cap)
+    return fail(STAR_ENOSPC, "query region full: %lld rows, q_cap %d", c->q_len, c->view.q_cap);
+  star::DecodePlan pl = plan_decode(c, c->q_len);
+  cudaError_t e = star::launch_decode_step(
+      c->view, c->p.scale, (int)c->q_len, static_cast<const bf16*>(q),
+      static_cast<const bf16*>(k), static_cast<const bf16*>(v), static_cast<bf16*>(o), lse, pl,
+      c->scratch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_decode_step launch");
+  c->q_len += 1;
+  return STAR_OK;
+}
+
+int star_lse_merge(int P, long long R, int D, const float* A, const float* s, float* out_A,
+                   float* out_s, void* stream) {
+  if (P < 1 || R < 0 || D < 1 || D > 1024) return fail(STAR_EINVAL, "need P >= 1, R >= 0, 1 <= D <= 1024");
+  if (R == 0) return STAR_OK;
+  if (!A || !s || !out_A || !out_s) return fail(STAR_EINVAL, "NULL tensor pointer");
+  cudaError_t e = star::launch_lse_merge(P, R, D, A, s, out_A, out_s, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_lse_merge launch");
+  return STAR_OK;
+}
+
+}  // extern "C"

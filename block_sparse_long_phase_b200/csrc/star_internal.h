@@ -1,0 +1,94 @@
+// Host/device view of a star_cache shared by the libstar kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace star {
+
+typedef __nv_bfloat16 bf16;
+
+// Geometry of the per-block KV cache.  Context segment i holds rows
+// [i*b, i*b + len_i) of every (batch, kv head), laid out [B][Hkv][len_i][D];
+// segments are back to back, so segment i starts i*B*Hkv*b*D elements in.
+struct CacheView {
+  int B, Hq, Hkv, D, G;
+  long long L;
+  int b, b_a, n_seg;
+  int q_cap;
+  bf16* ctxK;
+  bf16* ctxV;
+  bf16* qK;  // query region [B][Hkv][q_cap][D]
+  bf16* qV;
+};
+
+__host__ __device__ inline long long seg_len(const CacheView& c, int seg) {
+  long long s = (long long)seg * c.b;
+  long long r = c.L - s;
+  return r < c.b ? r : c.b;
+}
+
+// Element offset of context row `row` (absolute token index) of (batch bb,
+// kv head g) inside the segmented context cache.
+__host__ __device__ inline long long ctx_row_offset(const CacheView& c, int bb, int g,
+                                                    long long row) {
+  int seg = (int)(row / c.b);
+  long long off = row - (long long)seg * c.b;
+  long long len = seg_len(c, seg);
+  long long base = (long long)seg * c.B * c.Hkv * (long long)c.b * c.D;
+  return base + (((long long)bb * c.Hkv + g) * len + off) * c.D;
+}
+
+// Element offset of query-region row `row` of (bb, g).
+__host__ __device__ inline long long q_row_offset(const CacheView& c, int bb, int g,
+                                                  long long row) {
+  return (((long long)bb * c.Hkv + g) * c.q_cap + row) * c.D;
+}
+
+// Scratch owned by the cache for phase-2 partials.
+struct Scratch {
+  float* partA;        // partial outputs A_h
+  float* partS;        // partial log-sum-exp s_h
+  unsigned* tickets;   // per (batch, kv head) arrival counters, kept at 0 between calls
+  long long partA_elems;
+  long long partS_elems;
+  int n_tickets;
+};
+
+// ---- launchers (defined in the .cu files) --------------------------------
+cudaError_t launch_ctx_encode_mma(const CacheView& c, float scale, const bf16* Q, const bf16* K,
+                                  const bf16* V, bf16* O, float* LSE, const int4* work,
+                                  int n_work, cudaStream_t st);
+
+struct PrefillChunk {
+  int seg;     // context segment, or -1 for the query region
+  int start;   // first row inside the segment
+  int len;     // rows
+};
+constexpr int kMaxPrefillChunks = 96;
+
+struct PrefillPlan {
+  int n_chunks;
+  int row_tiles;   // ceil(G*lq / 64)
+  PrefillChunk chunk[kMaxPrefillChunks];
+};
+
+cudaError_t launch_query_prefill_mma(const CacheView& c, float scale, int lq, int len0,
+                                     const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
+                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
+                                     cudaStream_t st);
+
+struct DecodePlan {
+  int chunks_per_head;   // split-KV chunks per (batch, kv head)
+  long long chunk_rows;  // keys per chunk (multiple of 64)
+};
+
+cudaError_t launch_decode_step(const CacheView& c, float scale, int len0, const bf16* q,
+                               const bf16* k, const bf16* v, bf16* o, float* lse,
+                               const DecodePlan& plan, const Scratch& s, cudaStream_t st);
+
+cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,
+                             float* outA, float* outS, cudaStream_t st);
+
+}  // namespace star

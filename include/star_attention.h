@@ -1,0 +1,144 @@
+/*
+ * star_attention.h -- C ABI of libstar, the B200 (sm_100a) Star Attention
+ * two-phase attention hot path for one GPU.
+ *
+ * Sources (page title, then section):
+ *  [P2] "Star Attention: Efficient LLM Inference over Long Sequences"
+ *       (paper-graph-ui analysis page), section 3.4 "Detailed, Sentence-Based
+ *       Technical Breakdown": "Phase 1: Context Encoding with Anchor Blocks"
+ *       Steps 1-5 and "Phase 2: Query Encoding and Token Generation with
+ *       Distributed Softmax" Steps 3, 5 and 7 with the partition identity.
+ *  [P3] "NVIDIA/Star-Attention" (README mirror), "Two Phases of Star
+ *       Attention": Phase 1 and Phase 2 bullets.
+ *
+ * The pages' "hosts" are logical context blocks on one device: block i's KV
+ * lives in its own cache segment, the query region (query and generated
+ * tokens) is one more segment, and the distributed softmax of phase 2 runs
+ * on-chip.
+ *
+ * Conventions for every call below
+ *  - All tensor pointers are DEVICE pointers owned by the caller, except the
+ *    cache segments, which belong to the star_cache.  Tensors are dense,
+ *    row-major, 16-byte aligned; bf16 is IEEE bfloat16 (uint16 bits).
+ *  - Q/K/V are already rotated (RoPE applied by the caller).  Because the
+ *    anchor keeps its original positions ([P2] Phase 1 Step 2), the anchor's
+ *    keys and values are rows 0..b_a-1 of the context K/V: no copy is made.
+ *  - Grouped-query attention: q head h reads kv head h / (Hq / Hkv).
+ *  - LSE values are natural-log log-sum-exp of the SCALED logits
+ *    (scale * q.k), float32.
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t passed
+ *    as void*, NULL = legacy default stream).  Calls on one cache must be
+ *    issued in order from one host thread on one stream.
+ *  - No call allocates device memory except star_cache_create.
+ *  - Return value: STAR_OK (0) or a negative STAR_E* code; shape and argument
+ *    errors are caught on the host before anything is launched and leave the
+ *    cache unchanged.  star_last_error() gives a one-line description of the
+ *    last failure in the calling thread.
+ */
+#ifndef STAR_ATTENTION_H
+#define STAR_ATTENTION_H
+
+#if defined(__GNUC__)
+#define STAR_API __attribute__((visibility("default")))
+#else
+#define STAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STAR_OK            0
+#define STAR_EINVAL       -1   /* bad shape, ratio, b_a > b, null or misaligned pointer */
+#define STAR_ENOSPC       -2   /* query region full (q_cap reached)                      */
+#define STAR_ECUDA        -3   /* CUDA runtime / launch error                            */
+#define STAR_EUNSUPPORTED -4   /* head_dim not 64/128, device not sm_100                 */
+#define STAR_ENOMEM       -5   /* cudaMalloc failed in star_cache_create                 */
+
+/* Problem statement of one attention layer ([P2] Phase 1 Step 1, Phase 2
+ * Step 3).  B sequences with identical shapes and independent caches. */
+typedef struct {
+  int B;            /* batch, >= 1                                          */
+  int Hq;           /* query heads, a multiple of Hkv                       */
+  int Hkv;          /* key/value heads                                      */
+  int D;            /* head dim: 64 or 128                                  */
+  long long L;      /* context length, >= 1                                 */
+  int block;        /* block size b >= 1; n = ceil(L / b) blocks            */
+  int anchor;       /* anchor size b_a, 0 <= b_a <= b (0 = no anchor)       */
+  int q_cap;        /* query-region capacity: query tokens + decode steps   */
+  float scale;      /* softmax scale; <= 0 selects 1/sqrt(D)                */
+} star_params;
+
+/* Opaque KV cache: n context segments + 1 query-region segment, the segment
+ * table and the phase-2 scratch (partials and merge tickets). */
+typedef struct star_cache star_cache;
+
+/* Allocates the cache for `p` on the current CUDA device (cudaMalloc).
+ * Layout in HBM: context segment i holds K (then V) as [B][Hkv][len_i][D]
+ * bf16, len_i = min(b, L - i*b), segments back to back; the query region is
+ * [B][Hkv][q_cap][D] for K and for V.  *out is NULL on failure. */
+STAR_API int star_cache_create(const star_params* p, star_cache** out);
+
+/* Frees everything the cache owns (synchronises the device first).  NULL is
+ * accepted. */
+STAR_API int star_cache_destroy(star_cache* c);
+
+/* Number of segments: n context segments followed by the query region. */
+STAR_API int star_cache_num_segments(const star_cache* c);
+
+/* Segment table entry `seg` (0..n-1 context, n = query region): device
+ * pointers to its K and V ([B][Hkv][cap][D] bf16), the first context token
+ * it holds (`start`; L for the query region), the rows in use (`len`) and the
+ * rows reserved (`cap`).  Any output pointer may be NULL. */
+STAR_API int star_cache_segment(const star_cache* c, int seg, void** k, void** v,
+                       long long* start, long long* len, long long* cap);
+
+/* Empties the query region (length 0) so a new query can reuse the context
+ * cache.  Nothing is launched. */
+STAR_API int star_cache_reset_query(star_cache* c);
+
+/* Phase 1 -- context encoding ([P2] Phase 1 Steps 1-5; [P3] Phase 1).
+ * Q [B][Hq][L][D], K, V [B][Hkv][L][D] bf16 in; O [B][Hq][L][D] bf16 and
+ * LSE [B][Hq][L] float32 out.  Token t of block i sees tokens j <= t of its
+ * own block and, when i >= 1, the whole anchor [0, b_a).  Writes the cache:
+ * segment i receives K/V rows of block i only (anchor KV discarded, every
+ * context token cached exactly once).  Empties the query region. */
+STAR_API int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V,
+                    void* O, float* LSE, void* stream);
+
+/* Phase 2 -- query prefill ([P2] Phase 2 Steps 3, 5, 7).  Appends K, V
+ * [B][Hkv][lq][D] bf16 to the query region, then every query row r of
+ * Q [B][Hq][lq][D] attends to all context segments and to query-region rows
+ * 0..len0+r (len0 = rows present before the call), computing per-partition
+ * (A_h, s_h) partials and merging them on-chip.  O [B][Hq][lq][D] bf16, LSE
+ * [B][Hq][lq] float32.  STAR_ENOSPC if len0 + lq > q_cap. */
+STAR_API int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K,
+                       const void* V, void* O, float* LSE, void* stream);
+
+/* Phase 2 -- one generation step ([P2] Phase 2 Step 7).  Appends k, v
+ * [B][Hkv][1][D] to the query region, then q [B][Hq][1][D] attends to every
+ * context token and every query-region row (itself included): split-KV
+ * partials merged on-chip.  o [B][Hq][1][D] bf16, lse [B][Hq] float32.
+ * STAR_ENOSPC if the query region is full. */
+STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
+                     void* o, float* lse, void* stream);
+
+/* Phase 2 merge of P partials ([P2] Phase 2 Step 5; [P3] s_global, A_global):
+ * A [P][R][D], s [P][R] float32 (s_h as natural-log LSE, -inf = empty part)
+ * -> out_A [R][D] = sum_h exp(s_h - s) A_h, out_s [R] = s = log sum_h
+ * exp(s_h).  Rows whose parts are all empty give 0 and -inf.  P >= 1,
+ * R >= 0, 1 <= D <= 1024.  out_* must not alias the inputs. */
+STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const float* s,
+                   float* out_A, float* out_s, void* stream);
+
+/* Description of the last error in this thread ("" if none). */
+STAR_API const char* star_last_error(void);
+
+/* Library version string. */
+STAR_API const char* star_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STAR_ATTENTION_H */

@@ -50,6 +50,16 @@ import numpy as np
 NEG_INF = -np.inf
 
 
+def _f64(x) -> np.ndarray:
+    """Exact float64 copy on the host of a NumPy array or a torch tensor
+    (bf16 and fp32 values are representable exactly in float64)."""
+    if isinstance(x, np.ndarray):
+        return x.astype(np.float64, copy=False)
+    if hasattr(x, "detach"):
+        return x.detach().double().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
 # ---------------------------------------------------------------------------
 # Phase 1, Step 1: partition of the context into blocks.
 # ---------------------------------------------------------------------------
@@ -109,9 +119,9 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     softmax-weighted mean of the visible values.  A row with no visible key
     gets ``O = 0`` and ``LSE = -inf``.
     """
-    q = np.asarray(q, np.float64)
-    k = np.asarray(k, np.float64)
-    v = np.asarray(v, np.float64)
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
     x = scale * (q @ k.T)
     x = np.where(mask, x, NEG_INF)
     m = x.max(axis=1, initial=NEG_INF)
@@ -128,17 +138,17 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 # ---------------------------------------------------------------------------
 # Phase 1: context encoding.
 # ---------------------------------------------------------------------------
-def ctx_encode(Q: np.ndarray, K: np.ndarray, V: np.ndarray, b: int, b_a: int,
-               scale: float, rows=None):
-    """Phase-1 outputs for Q [B, Hq, L, D], K/V [B, Hkv, L, D] (float64).
+def ctx_encode(Q, K, V, b: int, b_a: int, scale: float, rows=None):
+    """Phase-1 outputs for Q [B, Hq, L, D], K/V [B, Hkv, L, D].
 
     For every context token ``t`` and q head ``h`` (kv head ``h // G``), the
     output is softmax attention over the tokens the Star mask lets ``t`` see
-    ([P2] Phase 1 Step 4).  ``rows`` restricts the computation to the given
-    token indices (the others are left as NaN); the result for a row does not
-    depend on which other rows are computed.
+    ([P2] Phase 1 Step 4).  ``rows`` (default: all) selects the token indices
+    to compute; the result for a row does not depend on which other rows are
+    computed.  Inputs may be NumPy arrays or torch tensors (only the rows and
+    keys used are copied to float64).
 
-    Returns ``(O [B, Hq, L, D], LSE [B, Hq, L])``.
+    Returns ``(O [B, Hq, R, D], LSE [B, Hq, R])`` float64 for the R rows.
     """
     Bn, Hq, L, D = Q.shape
     Hkv = K.shape[1]
@@ -146,8 +156,8 @@ def ctx_encode(Q: np.ndarray, K: np.ndarray, V: np.ndarray, b: int, b_a: int,
         raise ValueError("Hq must be a multiple of Hkv")
     G = Hq // Hkv
     rows = np.arange(L) if rows is None else np.asarray(rows, np.int64)
-    O = np.full((Bn, Hq, L, D), np.nan)
-    LSE = np.full((Bn, Hq, L), np.nan)
+    O = np.zeros((Bn, Hq, len(rows), D))
+    LSE = np.zeros((Bn, Hq, len(rows)))
     if len(rows) == 0:
         return O, LSE
     mask = star_mask_rows(L, b, b_a, rows)
@@ -155,12 +165,13 @@ def ctx_encode(Q: np.ndarray, K: np.ndarray, V: np.ndarray, b: int, b_a: int,
     cols = np.nonzero(mask.any(axis=0))[0]
     sub = mask[:, cols]
     for bi in range(Bn):
-        for h in range(Hq):
-            g = h // G
-            o, lse = masked_attention(Q[bi, h, rows], K[bi, g, cols],
-                                      V[bi, g, cols], sub, scale)
-            O[bi, h, rows] = o
-            LSE[bi, h, rows] = lse
+        for g in range(Hkv):
+            k = _f64(K[bi, g][cols])
+            v = _f64(V[bi, g][cols])
+            for h in range(g * G, (g + 1) * G):
+                o, lse = masked_attention(_f64(Q[bi, h][rows]), k, v, sub, scale)
+                O[bi, h] = o
+                LSE[bi, h] = lse
     return O, LSE
 
 
@@ -204,8 +215,8 @@ def lse_merge(A: np.ndarray, s: np.ndarray):
     ``A = sum_h exp(s_h - s) A_h``.  The maximum is subtracted before
     exponentiating; partitions with ``s_h = -inf`` contribute nothing.
     """
-    A = np.asarray(A, np.float64)
-    s = np.asarray(s, np.float64)
+    A = _f64(A)
+    s = _f64(s)
     m = s.max(axis=0)
     empty = ~np.isfinite(m)
     m_safe = np.where(empty, 0.0, m)
@@ -220,8 +231,8 @@ def lse_merge(A: np.ndarray, s: np.ndarray):
 
 def _context_keys(segments, bi, g):
     """Concatenation of every context segment's cache for (batch, kv head)."""
-    ks = [seg[2][bi, g] for seg in segments]
-    vs = [seg[3][bi, g] for seg in segments]
+    ks = [_f64(seg[2][bi, g]) for seg in segments]
+    vs = [_f64(seg[3][bi, g]) for seg in segments]
     return np.concatenate(ks, axis=0), np.concatenate(vs, axis=0)
 
 
@@ -247,13 +258,13 @@ def query_attend(q_rows: np.ndarray, segments, qk_region: np.ndarray,
     for bi in range(Bn):
         for g in range(Hkv):
             kc, vc = _context_keys(segments, bi, g)
-            k_all = np.concatenate([kc, qk_region[bi, g]], axis=0)
-            v_all = np.concatenate([vc, qv_region[bi, g]], axis=0)
+            k_all = np.concatenate([kc, _f64(qk_region[bi, g])], axis=0)
+            v_all = np.concatenate([vc, _f64(qv_region[bi, g])], axis=0)
             Lc = kc.shape[0]
             mask = np.ones((R, Lc + Nq), dtype=bool)
             mask[:, Lc:] = np.arange(Nq)[None, :] < np.asarray(visible_q)[:, None]
             for h in range(g * G, (g + 1) * G):
-                o, lse = masked_attention(q_rows[bi, h], k_all, v_all, mask, scale)
+                o, lse = masked_attention(_f64(q_rows[bi, h]), k_all, v_all, mask, scale)
                 O[bi, h] = o
                 LSE[bi, h] = lse
     return O, LSE
@@ -269,10 +280,10 @@ def query_prefill(Qq, Kq, Vq, segments, qk_region, qv_region, q_len0: int,
     qv_region)`` with the regions updated (copies).
     """
     lq = Qq.shape[2]
-    qk = qk_region.copy()
-    qv = qv_region.copy()
-    qk[:, :, q_len0:q_len0 + lq] = Kq
-    qv[:, :, q_len0:q_len0 + lq] = Vq
+    qk = _f64(qk_region).copy()
+    qv = _f64(qv_region).copy()
+    qk[:, :, q_len0:q_len0 + lq] = _f64(Kq)
+    qv[:, :, q_len0:q_len0 + lq] = _f64(Vq)
     vis = q_len0 + np.arange(lq) + 1
     O, LSE = query_attend(Qq, segments, qk, qv, vis, scale)
     return O, LSE, qk, qv
@@ -286,10 +297,10 @@ def decode_step(q, k, v, segments, qk_region, qv_region, q_len: int,
     only (at row ``q_len``), then the token attends to every context token
     and query-region rows ``0..q_len`` (itself included).
     """
-    qk = qk_region.copy()
-    qv = qv_region.copy()
-    qk[:, :, q_len] = k[:, :, 0]
-    qv[:, :, q_len] = v[:, :, 0]
+    qk = _f64(qk_region).copy()
+    qv = _f64(qv_region).copy()
+    qk[:, :, q_len] = _f64(k)[:, :, 0]
+    qv[:, :, q_len] = _f64(v)[:, :, 0]
     O, LSE = query_attend(q, segments, qk, qv, np.array([q_len + 1]), scale)
     return O, LSE, qk, qv
 

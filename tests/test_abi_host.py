@@ -1,0 +1,78 @@
+"""Host-side checks of the C ABI: the library builds, loads and exports every
+symbol include/star_attention.h declares.  No compute call (no GPU here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_phase_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "star_attention.h")).read()
+    return sorted(set(re.findall(r"STAR_API\s+[\w\s\*]+?\b(star_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def test_header_declares_the_four_entry_points():
+    syms = header_symbols()
+    for s in ("star_ctx_encode", "star_query_prefill", "star_decode_step", "star_lse_merge"):
+        assert s in syms
+    assert sorted(_abi.EXPORTS) == syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for s in header_symbols():
+        assert hasattr(lib, s), s
+        assert ctypes.cast(getattr(lib, s), ctypes.c_void_p).value
+
+
+def test_version_and_error_strings(lib):
+    assert b"sm_100a" in lib.star_version()
+    assert isinstance(lib.star_last_error(), bytes)
+
+
+def test_argument_errors_are_caught_on_the_host(lib):
+    """Shape errors never reach the device: these return before any CUDA call."""
+    out = ctypes.c_void_p()
+    bad = [
+        _abi.StarParams(1, 4, 3, 64, 1024, 256, 256, 8, 0.0),    # Hq % Hkv
+        _abi.StarParams(1, 4, 2, 64, 1024, 256, 300, 8, 0.0),    # b_a > b
+        _abi.StarParams(1, 4, 2, 64, 0, 256, 256, 8, 0.0),       # L = 0
+        _abi.StarParams(1, 4, 2, 64, 1024, 0, 0, 8, 0.0),        # b = 0
+        _abi.StarParams(1, 4, 2, 64, 1024, 256, -1, 8, 0.0),     # b_a < 0
+        _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 0, 0.0),    # q_cap = 0
+    ]
+    for p in bad:
+        assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EINVAL
+        assert out.value is None
+        assert lib.star_last_error()
+    p = _abi.StarParams(1, 4, 2, 96, 1024, 256, 256, 8, 0.0)     # D = 96
+    assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
+    assert lib.star_cache_create(None, ctypes.byref(out)) == _abi.STAR_EINVAL
+    assert lib.star_lse_merge(0, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_lse_merge(1, 4, 2000, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_lse_merge(1, 0, 8, None, None, None, None, None) == _abi.STAR_OK
+    assert lib.star_ctx_encode(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_decode_step(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_query_prefill(None, 4, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_cache_destroy(None) == _abi.STAR_OK
+    assert lib.star_cache_num_segments(None) == 0
+
+
+def test_binding_refuses_to_run_without_cuda():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    from block_sparse_long_phase_b200 import StarCache
+    with pytest.raises(RuntimeError):
+        StarCache(1, 4, 2, 64, 1024, 256, 256, 8)

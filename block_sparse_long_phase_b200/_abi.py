@@ -19,7 +19,7 @@ STAR_ENOMEM = -5
 
 # Every symbol the header declares.
 EXPORTS = (
-    "star_cache_create", "star_cache_destroy", "star_cache_num_segments",
+    "star_cache_create", "star_cache_destroy", "star_cache_device_error", "star_cache_num_segments",
     "star_cache_segment", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_decode_step", "star_lse_merge",
     "star_last_error", "star_version",
@@ -56,6 +56,7 @@ def load(path: str = LIB_PATH):
     lib.star_cache_create.argtypes = [ctypes.POINTER(StarParams), ctypes.POINTER(vp)]
     lib.star_cache_destroy.argtypes = [vp]
     lib.star_cache_num_segments.argtypes = [vp]
+    lib.star_cache_device_error.argtypes = [vp, ctypes.POINTER(i)]
     lib.star_cache_segment.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                        ctypes.POINTER(ll), ctypes.POINTER(ll), ctypes.POINTER(ll)]
     lib.star_cache_reset_query.argtypes = [vp]

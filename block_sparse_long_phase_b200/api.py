@@ -104,6 +104,12 @@ class StarCache:
             out.append(t)
         return out[0], out[1], seg
 
+    def device_error(self) -> int:
+        """Reads and clears the device error word (non-zero: a bounded wait gave up)."""
+        f = ctypes.c_int()
+        _abi.check(self.lib.star_cache_device_error(self.handle, ctypes.byref(f)))
+        return f.value
+
     @property
     def q_len(self) -> int:
         return self.segment(self.num_segments - 1).len

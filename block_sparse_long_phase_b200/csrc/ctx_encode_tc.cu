@@ -1,0 +1,404 @@
+// Phase-1 context encoding on the 5th-generation tensor core (tcgen05 + TMEM
+// + TMA), warp-specialised.
+//
+// "Star Attention: Efficient LLM Inference over Long Sequences" (analysis
+// page), section 3.4, "Phase 1: Context Encoding with Anchor Blocks": block i
+// >= 1 is prefixed with the anchor and encoded with causal attention over
+// [anchor | block i] (Steps 2 and 4); block 0 is encoded on its own; only the
+// block's own K/V is kept in the cache (Step 5).  The augmented block is never
+// materialised: a CTA streams the anchor's K/V tiles [0, b_a) with no mask and
+// then its own block's tiles up to the diagonal with a causal mask.
+//
+// CTA work item: one 128-row query tile of one block for TWO q heads of the
+// same kv group (GQA), so each K/V tile fetched by TMA feeds two S = Q K^T
+// and two O += P V MMAs; both heads share the mask.
+//
+// Roles (12 warps):
+//   warp 0      TMA producer: Q0/Q1 once, then K_j, V_j into a 4-slot ring
+//   warp 1      MMA issuer (one thread) and TMEM owner
+//   warps 2-3   copy the tile's own K/V rows into the block's cache segment
+//   warps 4-7   softmax for head 0: S0 row per thread, P0 back into TMEM
+//   warps 8-11  softmax for head 1
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
+// P_i (bf16) overwrites the first 64 columns of S_i.  tcgen05.mma ops issued by
+// the one MMA thread run in order, so S_i(j+1) is written only after
+// O_i += P_i(j) V_j has read P_i(j), and a commit that fires for S_i(j+1) also
+// guarantees O_i is stable, which is when its softmax warps may rescale it.
+//
+// Online softmax in base 2 with log2(e) folded into the scale; the running
+// maximum used for the exponentials is only raised when a row's maximum
+// grows by more than 2^8, so O rarely needs a TMEM read-modify-write.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "sm100_primitives.cuh"
+#include "star_common.cuh"
+#include "star_internal.h"
+#include "tmap.h"
+
+namespace star {
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;          // query rows per tile
+constexpr int BN = 128;          // keys per K/V tile
+constexpr int NBUF = 4;          // K/V ring slots
+constexpr int NTHREADS = 384;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct CtxTcArgs {
+  CUtensorMap tq;   // Q  as [B*Hq*L][D]
+  CUtensorMap tk;   // K  as [B*Hkv*L][D]
+  CUtensorMap tv;   // V  as [B*Hkv*L][D]
+  CacheView c;
+  float scale_log2;
+  const bf16* K;
+  const bf16* V;
+  bf16* O;
+  float* LSE;
+  const int4* work;   // (b*Hkv + g, head pair, block, q tile)
+  int* err;
+};
+
+SM100_DEV float ex2(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+struct Smem {
+  static constexpr int TILE = BM * D * 2;           // one Q or K/V tile, bytes
+  static constexpr int HALF = BM * 128;             // one 64-column (128 B) half
+  static constexpr int Q0 = 0;
+  static constexpr int Q1 = TILE;
+  static constexpr int RING = 2 * TILE;
+  static constexpr int BYTES = RING + NBUF * TILE;  // + barriers in static smem
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_constant__ CtxTcArgs a) {
+  using S = Smem<D>;
+  constexpr int NH = D / 64;                          // 128-byte halves per row
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t bar_q_full;
+  __shared__ __align__(8) uint64_t bar_kv_full[NBUF];
+  __shared__ __align__(8) uint64_t bar_kv_empty[NBUF];
+  __shared__ __align__(8) uint64_t bar_s_full[2];
+  __shared__ __align__(8) uint64_t bar_p_full[2];
+  __shared__ __align__(8) uint64_t bar_o_full;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  const CacheView& c = a.c;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- work item ------------------------------------------------------------
+  const int4 w = a.work[blockIdx.x];
+  const int bg = w.x;
+  const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+  const int h0 = g * c.G + 2 * w.y;
+  const int nq = (h0 + 1 < (g + 1) * c.G) ? 2 : 1;
+  const int blk = w.z;
+  const long long bstart = (long long)blk * c.b;
+  const long long bend = bstart + c.b < c.L ? bstart + c.b : c.L;
+  const long long t0 = bstart + (long long)w.w * BM;
+  const int n_rows = (int)((bend - t0) < BM ? (bend - t0) : BM);
+  const int n_anchor = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
+  const int n_kv = n_anchor + w.w + 1;
+  const long long kv_row0 = (long long)bg * c.L;     // row of (b, g, token 0) in K/V maps
+
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar_q_full), 1);
+    for (int i = 0; i < NBUF; ++i) {
+      mbar_init(smem_u32(&bar_kv_full[i]), 1);
+      mbar_init(smem_u32(&bar_kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar_s_full[i]), 1);
+      mbar_init(smem_u32(&bar_p_full[i]), 128);
+    }
+    mbar_init(smem_u32(&bar_o_full), 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tmem_base_s), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  auto fail = [&]() {
+    abort_s = 1;
+    atomicExch(a.err, 1);
+  };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer -----------------------------
+    if (elect_one()) {
+      prefetch_tmap(&a.tq);
+      prefetch_tmap(&a.tk);
+      prefetch_tmap(&a.tv);
+      const uint32_t qb = smem_u32(&bar_q_full);
+      mbar_arrive_expect_tx(qb, nq * S::TILE);
+      for (int q = 0; q < nq; ++q) {
+        const int qrow = (int)(((long long)bb * c.Hq + h0 + q) * c.L + t0);
+        for (int hf = 0; hf < NH; ++hf)
+          tma_load_2d(smem_u32(smem + (q ? S::Q1 : S::Q0) + hf * S::HALF), &a.tq, hf * 64, qrow, qb);
+      }
+      int last_use[NBUF];
+#pragma unroll
+      for (int k = 0; k < NBUF; ++k) last_use[k] = -1;
+      for (int i = 0; i < 2 * n_kv; ++i) {
+        const int j = i >> 1, slot = i % NBUF, use = i / NBUF;
+        if (use > 0 && !mbar_wait(smem_u32(&bar_kv_empty[slot]), (use - 1) & 1)) { fail(); break; }
+        if (*(volatile int*)&abort_s) break;
+        const long long tok = j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
+        const int row = (int)(kv_row0 + tok);
+        const uint32_t fb = smem_u32(&bar_kv_full[slot]);
+        mbar_arrive_expect_tx(fb, S::TILE);
+        const CUtensorMap* m = (i & 1) ? &a.tv : &a.tk;
+        for (int hf = 0; hf < NH; ++hf)
+          tma_load_2d(smem_u32(smem + S::RING + slot * S::TILE + hf * S::HALF), m, hf * 64, row, fb);
+        last_use[slot] = use;
+      }
+      if (*(volatile int*)&abort_s) {
+        // let every copy this CTA started land before its shared memory is released
+        mbar_wait(qb, 0);
+        for (int k = 0; k < NBUF; ++k)
+          if (last_use[k] >= 0) mbar_wait(smem_u32(&bar_kv_full[k]), last_use[k] & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer -------------------------------
+    if (elect_one()) {
+      const uint32_t id_qk = idesc_bf16_f32(BM, BN, false);
+      const uint32_t id_pv = idesc_bf16_f32(BM, D, true);
+      const uint32_t sO[2] = {tmem + 256, tmem + 256 + D};
+      const uint32_t sS[2] = {tmem, tmem + 128};
+      bool ok = mbar_wait(smem_u32(&bar_q_full), 0);
+      if (!ok) fail();
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int ik = 2 * j, iv = 2 * j + 1;
+        const int sk = ik % NBUF, sv = iv % NBUF;
+        if (!mbar_wait(smem_u32(&bar_kv_full[sk]), (ik / NBUF) & 1)) { fail(); break; }
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(smem + S::RING + sk * S::TILE);
+        for (int q = 0; q < nq; ++q) {
+          const uint32_t qbase = smem_u32(smem + (q ? S::Q1 : S::Q0));
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * S::HALF + (kk & 3) * 32;
+            mma_ss(sS[q], smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                   id_qk, kk > 0);
+          }
+          mma_commit(smem_u32(&bar_s_full[q]));
+        }
+        mma_commit(smem_u32(&bar_kv_empty[sk]));
+        if (!mbar_wait(smem_u32(&bar_kv_full[sv]), (iv / NBUF) & 1)) { fail(); break; }
+        const uint32_t vbase = smem_u32(smem + S::RING + sv * S::TILE);
+        for (int q = 0; q < nq; ++q) {
+          if (!mbar_wait(smem_u32(&bar_p_full[q]), j & 1)) { fail(); ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(sO[q], sS[q] + kk * 8, smem_desc_sw128(vbase + kk * 2048, S::HALF, 1024), id_pv,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&bar_kv_empty[sv]));
+        if (*(volatile int*)&abort_s) break;
+      }
+      mma_commit(smem_u32(&bar_o_full));
+    }
+  } else if (warp < 4) {
+    // ---------------- cache segment write (anchor KV discarded) ---------------
+    if (h0 == g * c.G) {
+      const long long len = seg_len(c, blk);
+      const long long sbase = (long long)blk * c.B * c.Hkv * (long long)c.b * D +
+                              ((long long)bg * len + (t0 - bstart)) * D;
+      const long long gbase = (kv_row0 + t0) * D;
+      constexpr int CPR = D / 8;
+      for (int i = tid - 64; i < n_rows * CPR; i += 64) {
+        const int r = i / CPR, ch = i - (i / CPR) * CPR;
+        const uint4 kv = *reinterpret_cast<const uint4*>(a.K + gbase + (long long)r * D + ch * 8);
+        const uint4 vv = *reinterpret_cast<const uint4*>(a.V + gbase + (long long)r * D + ch * 8);
+        *reinterpret_cast<uint4*>(c.ctxK + sbase + (long long)r * D + ch * 8) = kv;
+        *reinterpret_cast<uint4*>(c.ctxV + sbase + (long long)r * D + ch * 8) = vv;
+      }
+    }
+  } else {
+    // ------------------------------ softmax ----------------------------------
+    const int q = (warp - 4) >> 2;                    // head 0 or 1 of the pair
+    if (q < nq) {
+      const int r = ((warp & 3) << 5) | lane;         // tile row owned by this thread
+      const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+      const uint32_t tS = tmem + lane_off + q * 128;
+      const uint32_t tO = tmem + lane_off + 256 + q * D;
+      const long long pos = t0 + r;                   // token index of the row
+      float m_used = -INFINITY, l = 0.f;
+      const float sl2 = a.scale_log2;
+      for (int j = 0; j < n_kv; ++j) {
+        if (!mbar_wait(smem_u32(&bar_s_full[q]), j & 1)) { fail(); break; }
+        tc_fence_after();
+        uint32_t s[BN];
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
+        tmem_wait_ld();
+        // mask: anchor tail (keys >= b_a) and the causal diagonal
+        const bool anchor = j < n_anchor;
+        const long long k0 = anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
+        const long long lim = anchor ? (long long)c.b_a : pos + 1;   // keys < lim are visible
+        if (k0 + BN > lim) {
+          const int nvis = (int)(lim - k0 < 0 ? 0 : lim - k0);   // visible columns: [0, nvis)
+#pragma unroll
+          for (int i = 0; i < BN; ++i)
+            if (i >= nvis) s[i] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+        const float m_tile = mx * sl2;
+        const bool need = m_tile > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2(m_used - m_tile);               // 0 when m_used is -inf
+          m_used = m_tile;
+        }
+        if (__any_sync(0xffffffffu, need) && j > 0) {
+          // O_i is stable here (see header); rescale this warp's rows.
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+        }
+        l *= alpha;
+        const float base = m_used == -INFINITY ? 0.f : m_used;
+        float rs = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float e0 = ex2(fmaf(__uint_as_float(s[cc * 32 + 2 * i]), sl2, -base));
+            const float e1 = ex2(fmaf(__uint_as_float(s[cc * 32 + 2 * i + 1]), sl2, -base));
+            rs += e0 + e1;
+            p[i] = pack_bf16(e0, e1);
+          }
+          tmem_st16(tS + cc * 16, p);
+        }
+        l += rs;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bar_p_full[q]));
+      }
+      // ---- epilogue: O / l in bf16, LSE = (m + log2 l) ln 2 -------------------
+      const bool ok = mbar_wait(smem_u32(&bar_o_full), 0);
+      if (!ok) fail();
+      tc_fence_after();
+      const int h = h0 + q;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      bf16* orow = a.O + (((long long)bb * c.Hq + h) * c.L + pos) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld();
+        if (r < n_rows) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            reinterpret_cast<uint4*>(orow + cc * 32)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      if (r < n_rows)
+        a.LSE[((long long)bb * c.Hq + h) * c.L + pos] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// Work list for the tensor-core phase-1 kernel: (b*Hkv + g, head pair, block,
+// q tile) for every 128-row tile, longest (most K/V tiles) first.
+size_t ctx_tc_work_count(const CacheView& c) {
+  const int pairs = (c.G + 1) / 2;
+  size_t n = 0;
+  for (int blk = 0; blk < c.n_seg; ++blk) n += (size_t)((seg_len(c, blk) + BM - 1) / BM);
+  return n * c.B * c.Hkv * pairs;
+}
+
+void ctx_tc_fill_work(const CacheView& c, int4* out) {
+  const int pairs = (c.G + 1) / 2;
+  struct Item { long long cost; int4 v; };
+  std::vector<Item> items;
+  for (int blk = 0; blk < c.n_seg; ++blk) {
+    const long long tiles = (seg_len(c, blk) + BM - 1) / BM;
+    const long long anchor_tiles = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
+    for (int qt = 0; qt < tiles; ++qt)
+      for (int bg = 0; bg < c.B * c.Hkv; ++bg)
+        for (int hp = 0; hp < pairs; ++hp)
+          items.push_back({anchor_tiles + qt + 1, make_int4(bg, hp, blk, qt)});
+  }
+  std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
+  for (size_t i = 0; i < items.size(); ++i) out[i] = items[i].v;
+}
+
+cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
+                                 const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
+                                 int* err, cudaStream_t st) {
+  if (n_work == 0) return cudaSuccess;
+  CtxTcArgs a;
+  memset(&a, 0, sizeof(a));
+  const unsigned long long qrows = (unsigned long long)c.B * c.Hq * c.L;
+  const unsigned long long kvrows = (unsigned long long)c.B * c.Hkv * c.L;
+  if (!make_tmap_bf16_2d(&a.tq, Q, qrows, c.D, BM, 64) || !make_tmap_bf16_2d(&a.tk, K, kvrows, c.D, BN, 64) ||
+      !make_tmap_bf16_2d(&a.tv, V, kvrows, c.D, BN, 64))
+    return cudaErrorInvalidValue;
+  a.c = c;
+  a.scale_log2 = scale * kLog2e;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.LSE = LSE;
+  a.work = work;
+  a.err = err;
+  cudaError_t e;
+  if (c.D == 128) {
+    const int smem = Smem<128>::BYTES + 1024;
+    e = cudaFuncSetAttribute(ctx_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ctx_tc_kernel<128><<<n_work, NTHREADS, smem, st>>>(a);
+  } else {
+    const int smem = Smem<64>::BYTES + 1024;
+    e = cudaFuncSetAttribute(ctx_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ctx_tc_kernel<64><<<n_work, NTHREADS, smem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace star

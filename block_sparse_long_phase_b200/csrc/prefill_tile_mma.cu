@@ -1,24 +1,18 @@
-// Flash-style attention tile kernel on warp-level bf16 MMA (mma.sync m16n8k16).
+// Phase-2 query-prefill partials: flash-style attention tile kernel on
+// warp-level bf16 MMA (mma.sync m16n8k16).
 //
-// One CTA computes a 64-row Q tile against a sequence of 64-key K/V tiles with
-// an online softmax (exp2 with log2(e) folded into the scale), fp32
-// accumulation, and double-buffered cp.async staging in XOR-swizzled shared
-// memory.  It serves two operations:
-//
-//  * MODE_CTX -- phase-1 context encoding ("Star Attention: Efficient LLM
-//    Inference over Long Sequences", analysis page, section 3.4, "Phase 1:
-//    Context Encoding with Anchor Blocks", Steps 2, 4 and 5): the Q tile of
-//    block i >= 1 streams the anchor keys [0, b_a) unmasked, then its own
-//    block's keys up to the diagonal under a causal mask; block 0 streams only
-//    its own keys.  The "augmented block" is never materialised: the anchor is
-//    just the first key range.  The CTA of the first q head of a kv group also
-//    writes its tile's K/V rows into the block's cache segment (Step 5: only
-//    the block's own KV is kept).
-//  * MODE_PART -- phase-2 query prefill partials (same page, "Phase 2", Step
-//    3): packed query rows of one kv group (the G q heads x lq rows of one kv
-//    head are contiguous) against one key chunk, either a slice of a context
-//    segment (fully visible) or the query region (causal), giving the local
-//    (A_h, s_h) of that chunk in fp32 for the merge kernel.
+// "Star Attention: Efficient LLM Inference over Long Sequences" (analysis
+// page), section 3.4, "Phase 2: Query Encoding and Token Generation with
+// Distributed Softmax", Step 3: every context block computes the local
+// attention A_h of the query rows over its own cache, with the log of its
+// exponent sum s_h; the query region is one more partition, attended causally.
+// A CTA takes 64 packed query rows of one kv group (the G q heads x lq rows of
+// one kv head are contiguous in Q) against one key chunk -- a slice of a
+// context segment (fully visible) or the query region (causal) -- streaming
+// 64-key K/V tiles through double-buffered cp.async stages in XOR-swizzled
+// shared memory with an online softmax (exp2, log2(e) folded into the scale)
+// and fp32 accumulation, and writes (A_h, s_h) of that chunk in fp32.  A
+// second kernel merges the chunks' partials per row (Step 5).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -31,25 +25,21 @@ namespace {
 constexpr int BM = 64;
 constexpr int BN = 64;
 constexpr int NTHREADS = 128;
-enum { MODE_CTX = 0, MODE_PART = 1 };
 
 struct TileArgs {
   CacheView c;
   float scale_log2;
-  const bf16* Q;  // CTX: [B][Hq][L][D]; PART: query rows [B][Hq][lq][D]
-  const bf16* K;  // CTX: context K [B][Hkv][L][D]; PART: new query K [B][Hkv][lq][D]
+  const bf16* Q;  // query rows [B][Hq][lq][D]
+  const bf16* K;  // this call's query K [B][Hkv][lq][D]
   const bf16* V;
-  bf16* O;        // CTX output
-  float* LSE;     // CTX output
-  const int4* work;
   int lq, len0;
   float* partA;
   float* partS;
   PrefillPlan plan;
 };
 
-template <int D, int MODE>
-__global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_constant__ TileArgs a) {
+template <int D>
+__global__ void __launch_bounds__(NTHREADS) prefill_tile_kernel(const __grid_constant__ TileArgs a) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int TILE_BYTES = BM * D * 2;     // BM == BN
   constexpr int NT_O = D / 8;                // output n-tiles
@@ -61,76 +51,43 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
   const CacheView& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work item ---------------------------------------------------------
-  int bb, g, hq = 0;
-  long long row0;          // CTX: token index of tile row 0; PART: packed row index
-  int n_rows;
-  const bf16* qptr;
-  long long nk0, nk1;      // keys in range 0 / range 1
-  long long bstart = 0;    // CTX: first token of the block
-  int chunk_id = 0, blk = 0;
-  if (MODE == MODE_CTX) {
-    const int4 w = a.work[blockIdx.x];
-    bb = w.x / c.Hq;
-    hq = w.x % c.Hq;
-    g = hq / c.G;
-    blk = w.y;
-    bstart = (long long)blk * c.b;
-    long long bend = bstart + c.b < c.L ? bstart + c.b : c.L;
-    row0 = bstart + (long long)w.z * BM;
-    n_rows = (int)((bend - row0) < BM ? (bend - row0) : BM);
-    qptr = a.Q + (((long long)bb * c.Hq + hq) * c.L + row0) * D;
-    nk0 = blk > 0 ? c.b_a : 0;
-    nk1 = row0 + n_rows - bstart;
-  } else {
-    const int per_bg = a.plan.row_tiles * a.plan.n_chunks;
-    const int bg = blockIdx.x / per_bg;
-    const int rem = blockIdx.x - bg * per_bg;
-    chunk_id = rem / a.plan.row_tiles;
-    const int rt = rem - chunk_id * a.plan.row_tiles;
-    bb = bg / c.Hkv;
-    g = bg - bb * c.Hkv;
-    const int rows_total = c.G * a.lq;
-    row0 = (long long)rt * BM;
-    n_rows = (int)(rows_total - row0 < BM ? rows_total - row0 : BM);
-    qptr = a.Q + (((long long)bb * c.Hq + (long long)g * c.G) * a.lq + row0) * D;
-    nk0 = a.plan.chunk[chunk_id].len;
-    nk1 = 0;
-  }
-  const int t0 = (int)((nk0 + BN - 1) / BN);
-  const int t1 = (int)((nk1 + BN - 1) / BN);
-  const int n_tiles = t0 + t1;
+  // ---- work item: (batch*kv head, key chunk, 64-row tile) -------------------
+  const int per_bg = a.plan.row_tiles * a.plan.n_chunks;
+  const int bg = blockIdx.x / per_bg;
+  const int rem = blockIdx.x - bg * per_bg;
+  const int chunk_id = rem / a.plan.row_tiles;
+  const int rt = rem - chunk_id * a.plan.row_tiles;
+  const int bb = bg / c.Hkv;
+  const int g = bg - bb * c.Hkv;
+  const int rows_total = c.G * a.lq;
+  const long long row0 = (long long)rt * BM;
+  const int n_rows = (int)(rows_total - row0 < BM ? rows_total - row0 : BM);
+  const bf16* qptr = a.Q + (((long long)bb * c.Hq + (long long)g * c.G) * a.lq + row0) * D;
+  const long long nk = a.plan.chunk[chunk_id].len;   // keys in this chunk
+  const int n_tiles = (int)((nk + BN - 1) / BN);
 
-  // Row pointer of key j of range r (K when v == false, V otherwise).
-  auto key_row = [&](int r, long long j, bool v) -> const bf16* {
-    if (MODE == MODE_CTX) {
-      const bf16* base = v ? a.V : a.K;
-      long long tok = (r == 0) ? j : bstart + j;
-      return base + (((long long)bb * c.Hkv + g) * c.L + tok) * D;
-    } else {
-      const PrefillChunk ch = a.plan.chunk[chunk_id];
-      if (ch.seg >= 0) {
-        const bf16* base = v ? c.ctxV : c.ctxK;
-        return base + ctx_row_offset(c, bb, g, (long long)ch.seg * c.b + ch.start + j);
-      }
-      if (j < a.len0) return (v ? c.qV : c.qK) + q_row_offset(c, bb, g, j);
-      const bf16* base = v ? a.V : a.K;
-      return base + (((long long)bb * c.Hkv + g) * a.lq + (j - a.len0)) * D;
+  // Row pointer of key j of the chunk (K when v == false, V otherwise).
+  auto key_row = [&](long long j, bool v) -> const bf16* {
+    const PrefillChunk ch = a.plan.chunk[chunk_id];
+    if (ch.seg >= 0) {
+      const bf16* base = v ? c.ctxV : c.ctxK;
+      return base + ctx_row_offset(c, bb, g, (long long)ch.seg * c.b + ch.start + j);
     }
+    if (j < a.len0) return (v ? c.qV : c.qK) + q_row_offset(c, bb, g, j);
+    const bf16* base = v ? a.V : a.K;
+    return base + (((long long)bb * c.Hkv + g) * a.lq + (j - a.len0)) * D;
   };
 
   auto load_tile = [&](int stage, int t) {
-    const int r = t < t0 ? 0 : 1;
-    const long long j0 = (long long)(r == 0 ? t : t - t0) * BN;
-    const long long nk = r == 0 ? nk0 : nk1;
+    const long long j0 = (long long)t * BN;
     const uint32_t dk = smem_u32(sK + stage * TILE_BYTES);
     const uint32_t dv = smem_u32(sV + stage * TILE_BYTES);
     for (int i = tid; i < BN * CPR; i += NTHREADS) {
       const int row = i / CPR, ch = i - (i / CPR) * CPR;
       const long long j = j0 + row;
       const bool ok = j < nk;
-      const bf16* kp = ok ? key_row(r, j, false) : qptr;
-      const bf16* vp = ok ? key_row(r, j, true) : qptr;
+      const bf16* kp = ok ? key_row(j, false) : qptr;
+      const bf16* vp = ok ? key_row(j, true) : qptr;
       cp_async16(dk + swz(row, ch, CPR), kp + ch * 8, ok ? 16 : 0);
       cp_async16(dv + swz(row, ch, CPR), vp + ch * 8, ok ? 16 : 0);
     }
@@ -149,16 +106,10 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
   // Per-thread rows inside the tile: r_a = warp*16 + lane/4, r_b = r_a + 8.
   const int ra = warp * 16 + (lane >> 2);
   const int rb = ra + 8;
-  // Causal position of each row (CTX: token index; PART: query-region index).
-  long long pos_a, pos_b;
-  if (MODE == MODE_CTX) {
-    pos_a = row0 + ra;
-    pos_b = row0 + rb;
-  } else {
-    pos_a = a.len0 + (row0 + ra) % a.lq;
-    pos_b = a.len0 + (row0 + rb) % a.lq;
-  }
-  const bool causal_part = (MODE == MODE_PART) && a.plan.chunk[chunk_id].seg < 0;
+  // Causal position of each row in the query region.
+  const long long pos_a = a.len0 + (row0 + ra) % a.lq;
+  const long long pos_b = a.len0 + (row0 + rb) % a.lq;
+  const bool causal = a.plan.chunk[chunk_id].seg < 0;
 
   uint32_t qa[D / 16][4];
   float o[NT_O][4];
@@ -201,10 +152,7 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
     }
 
     // Scale into log2 units and mask.
-    const int r = t < t0 ? 0 : 1;
-    const long long j0 = (long long)(r == 0 ? t : t - t0) * BN;
-    const long long nk = r == 0 ? nk0 : nk1;
-    const bool causal = (MODE == MODE_CTX) ? (r == 1) : causal_part;
+    const long long j0 = (long long)t * BN;
     const bool need_mask = (j0 + BN > nk) || causal;
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
@@ -212,8 +160,7 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
       for (int e = 0; e < 4; ++e) s[n][e] *= a.scale_log2;
     }
     if (need_mask) {
-      // key position used by the causal test
-      const long long kpos0 = (MODE == MODE_CTX) ? bstart + j0 : j0;
+      const long long kpos0 = j0;
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
 #pragma unroll
@@ -298,43 +245,8 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
   const float lse_b = l_b > 0.f ? (m_b + log2f(l_b)) * kLn2 : -INFINITY;
   const int cq = 2 * (lane & 3);
 
-  if (MODE == MODE_CTX) {
-    bf16* obase = a.O + (((long long)bb * c.Hq + hq) * c.L + row0) * D;
-    float* lbase = a.LSE + ((long long)bb * c.Hq + hq) * c.L + row0;
-    if (ra < n_rows) {
-#pragma unroll
-      for (int n = 0; n < NT_O; ++n)
-        *reinterpret_cast<uint32_t*>(obase + (long long)ra * D + 8 * n + cq) =
-            pack_bf16(o[n][0] * inv_a, o[n][1] * inv_a);
-      if ((lane & 3) == 0) lbase[ra] = lse_a;
-    }
-    if (rb < n_rows) {
-#pragma unroll
-      for (int n = 0; n < NT_O; ++n)
-        *reinterpret_cast<uint32_t*>(obase + (long long)rb * D + 8 * n + cq) =
-            pack_bf16(o[n][2] * inv_b, o[n][3] * inv_b);
-      if ((lane & 3) == 0) lbase[rb] = lse_b;
-    }
-    // Cache write (anchor discarded): the last staged tile holds exactly this
-    // tile's own K/V rows; the first q head of the kv group stores them.
-    if (hq % c.G == 0) {
-      const int stage = (n_tiles - 1) & 1;
-      const long long seg_row0 = row0 - bstart;
-      const long long len = seg_len(c, blk);
-      const long long base = (long long)blk * c.B * c.Hkv * (long long)c.b * D +
-                             (((long long)bb * c.Hkv + g) * len + seg_row0) * D;
-      for (int i = tid; i < n_rows * CPR; i += NTHREADS) {
-        const int row = i / CPR, ch = i - (i / CPR) * CPR;
-        const uint4 kv = *reinterpret_cast<const uint4*>(sK + stage * TILE_BYTES + swz(row, ch, CPR));
-        const uint4 vv = *reinterpret_cast<const uint4*>(sV + stage * TILE_BYTES + swz(row, ch, CPR));
-        *reinterpret_cast<uint4*>(c.ctxK + base + (long long)row * D + ch * 8) = kv;
-        *reinterpret_cast<uint4*>(c.ctxV + base + (long long)row * D + ch * 8) = vv;
-      }
-    }
-  } else {
-    const int rows_total = c.G * a.lq;
-    const long long bg = (long long)bb * c.Hkv + g;
-    const long long pbase = (bg * a.plan.n_chunks + chunk_id) * rows_total;
+  {
+    const long long pbase = ((long long)bg * a.plan.n_chunks + chunk_id) * rows_total;
     if (ra < n_rows) {
       float* pa_ = a.partA + (pbase + row0 + ra) * D;
 #pragma unroll
@@ -352,8 +264,8 @@ __global__ void __launch_bounds__(NTHREADS) attn_tile_kernel(const __grid_consta
     // Append this call's query K/V to the query region (one writer per
     // (batch, kv head); readers in this launch take those rows from the input).
     if (a.plan.chunk[chunk_id].seg < 0 && row0 == 0) {
-      const bf16* ks = a.K + bg * a.lq * D;
-      const bf16* vs = a.V + bg * a.lq * D;
+      const bf16* ks = a.K + (long long)bg * a.lq * D;
+      const bf16* vs = a.V + (long long)bg * a.lq * D;
       bf16* kd = c.qK + q_row_offset(c, bb, g, a.len0);
       bf16* vd = c.qV + q_row_offset(c, bb, g, a.len0);
       for (int i = tid; i < a.lq * CPR; i += NTHREADS) {
@@ -404,34 +316,17 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq,
   if (lane == 0) LSE[((long long)bb * c.Hq + h) * lq + rr] = lse;
 }
 
-template <int D, int MODE>
+template <int D>
 cudaError_t launch_tile(const TileArgs& a, int grid, cudaStream_t st) {
   const int smem = 5 * BM * D * 2;
-  cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<D, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(prefill_tile_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_tile_kernel<D, MODE><<<grid, NTHREADS, smem, st>>>(a);
+  prefill_tile_kernel<D><<<grid, NTHREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
-
-cudaError_t launch_ctx_encode_mma(const CacheView& c, float scale, const bf16* Q, const bf16* K,
-                                  const bf16* V, bf16* O, float* LSE, const int4* work,
-                                  int n_work, cudaStream_t st) {
-  if (n_work == 0) return cudaSuccess;
-  TileArgs a{};
-  a.c = c;
-  a.scale_log2 = scale * kLog2e;
-  a.Q = Q;
-  a.K = K;
-  a.V = V;
-  a.O = O;
-  a.LSE = LSE;
-  a.work = work;
-  if (c.D == 128) return launch_tile<128, MODE_CTX>(a, n_work, st);
-  return launch_tile<64, MODE_CTX>(a, n_work, st);
-}
 
 cudaError_t launch_query_prefill_mma(const CacheView& c, float scale, int lq, int len0,
                                      const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
@@ -449,8 +344,7 @@ cudaError_t launch_query_prefill_mma(const CacheView& c, float scale, int lq, in
   a.partS = s.partS;
   a.plan = plan;
   const int grid = c.B * c.Hkv * plan.row_tiles * plan.n_chunks;
-  cudaError_t e = (c.D == 128) ? launch_tile<128, MODE_PART>(a, grid, st)
-                               : launch_tile<64, MODE_PART>(a, grid, st);
+  cudaError_t e = (c.D == 128) ? launch_tile<128>(a, grid, st) : launch_tile<64>(a, grid, st);
   if (e != cudaSuccess) return e;
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
   const int mgrid = (int)((rows + 3) / 4);

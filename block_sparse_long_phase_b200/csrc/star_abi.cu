@@ -93,30 +93,6 @@ star::DecodePlan plan_decode(const star_cache* c, long long len0) {
   return pl;
 }
 
-// Phase-1 work list: (b*Hq + h, block, q tile), sorted by the number of K/V
-// tiles each item streams, longest first, so the tail of the grid is short.
-std::vector<int4> plan_ctx(const star_params& p) {
-  std::vector<int4> w;
-  const long long n = (p.L + p.block - 1) / p.block;
-  struct Item { long long cost; int4 v; };
-  std::vector<Item> items;
-  for (int blk = 0; blk < n; ++blk) {
-    const long long bs = (long long)blk * p.block;
-    const long long len = std::min<long long>(p.block, p.L - bs);
-    const long long tiles = (len + kTileRows - 1) / kTileRows;
-    const long long anchor_tiles = blk > 0 ? (p.anchor + kTileRows - 1) / kTileRows : 0;
-    for (int qt = 0; qt < tiles; ++qt)
-      for (int b = 0; b < p.B; ++b)
-        for (int h = 0; h < p.Hq; ++h)
-          items.push_back({anchor_tiles + qt + 1, make_int4(b * p.Hq + h, blk, qt, 0)});
-  }
-  std::stable_sort(items.begin(), items.end(),
-                   [](const Item& a, const Item& b) { return a.cost > b.cost; });
-  w.reserve(items.size());
-  for (auto& it : items) w.push_back(it.v);
-  return w;
-}
-
 int validate_params(const star_params* p) {
   if (!p) return fail(STAR_EINVAL, "params is NULL");
   if (p->B < 1 || p->Hq < 1 || p->Hkv < 1) return fail(STAR_EINVAL, "B, Hq, Hkv must be >= 1");
@@ -185,7 +161,8 @@ int star_cache_create(const star_params* p, star_cache** out) {
     partA = std::max(partA, rows * v.D);
     partS = std::max(partS, rows);
   }
-  std::vector<int4> work = plan_ctx(c->p);
+  std::vector<int4> work(star::ctx_tc_work_count(v));
+  star::ctx_tc_fill_work(v, work.data());
   c->n_ctx_work = (int)work.size();
 
   const long long kv_ctx = (long long)p->B * p->Hkv * p->L * p->D;        // elements
@@ -197,6 +174,7 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const size_t o_qk = take(kv_q * 2), o_qv = take(kv_q * 2);
   const size_t o_pa = take(partA * 4), o_ps = take(partS * 4);
   const size_t o_t = take(n_tickets * 4);
+  const size_t o_e = take(sizeof(int));
   const size_t o_w = take(work.size() * sizeof(int4));
   e = cudaMalloc(&c->block, off);
   if (e != cudaSuccess) {
@@ -211,11 +189,13 @@ int star_cache_create(const star_params* p, star_cache** out) {
   c->scratch.partA = reinterpret_cast<float*>(base + o_pa);
   c->scratch.partS = reinterpret_cast<float*>(base + o_ps);
   c->scratch.tickets = reinterpret_cast<unsigned*>(base + o_t);
+  c->scratch.err = reinterpret_cast<int*>(base + o_e);
   c->scratch.partA_elems = partA;
   c->scratch.partS_elems = partS;
   c->scratch.n_tickets = (int)n_tickets;
   c->ctx_work = reinterpret_cast<int4*>(base + o_w);
   e = cudaMemset(c->scratch.tickets, 0, n_tickets * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->scratch.err, 0, sizeof(int));
   if (e == cudaSuccess)
     e = cudaMemcpy(c->ctx_work, work.data(), work.size() * sizeof(int4), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
@@ -236,6 +216,16 @@ int star_cache_destroy(star_cache* c) {
   delete c;
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   if (f != cudaSuccess) return cuda_fail(f, "cudaFree");
+  return STAR_OK;
+}
+
+int star_cache_device_error(star_cache* c, int* flag) {
+  if (!c || !flag) return fail(STAR_EINVAL, "NULL argument");
+  int h = 0;
+  cudaError_t e = cudaMemcpy(&h, c->scratch.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && h) e = cudaMemset(c->scratch.err, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  *flag = h;
   return STAR_OK;
 }
 
@@ -275,10 +265,11 @@ int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, 
   if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
     return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
-  cudaError_t e = star::launch_ctx_encode_mma(
+  cudaError_t e = star::launch_ctx_encode_tc(
       c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
       static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work,
-      static_cast<cudaStream_t>(stream));
+      c->scratch.err, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
   c->q_len = 0;
   return STAR_OK;

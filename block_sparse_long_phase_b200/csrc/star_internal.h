@@ -51,15 +51,18 @@ struct Scratch {
   float* partA;        // partial outputs A_h
   float* partS;        // partial log-sum-exp s_h
   unsigned* tickets;   // per (batch, kv head) arrival counters, kept at 0 between calls
+  int* err;            // device error word: set by a kernel whose bounded wait gave up
   long long partA_elems;
   long long partS_elems;
   int n_tickets;
 };
 
 // ---- launchers (defined in the .cu files) --------------------------------
-cudaError_t launch_ctx_encode_mma(const CacheView& c, float scale, const bf16* Q, const bf16* K,
-                                  const bf16* V, bf16* O, float* LSE, const int4* work,
-                                  int n_work, cudaStream_t st);
+size_t ctx_tc_work_count(const CacheView& c);
+void ctx_tc_fill_work(const CacheView& c, int4* out);
+cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
+                                 const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
+                                 int* err, cudaStream_t st);
 
 struct PrefillChunk {
   int seg;     // context segment, or -1 for the query region

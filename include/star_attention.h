@@ -83,6 +83,12 @@ STAR_API int star_cache_create(const star_params* p, star_cache** out);
  * accepted. */
 STAR_API int star_cache_destroy(star_cache* c);
 
+/* Reads and clears the cache's device error word (synchronous: waits for
+ * the work already queued on the device).  *flag is non-zero if a kernel
+ * gave up a bounded wait on one of its own pipeline barriers since the last
+ * call -- outputs of that call are then invalid.  Kernels never trap. */
+STAR_API int star_cache_device_error(star_cache* c, int* flag);
+
 /* Number of segments: n context segments followed by the query region. */
 STAR_API int star_cache_num_segments(const star_cache* c);
 

@@ -47,6 +47,7 @@ def run_path(w, x, T=None):
     Oq, LSEq = cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
     dec = [cache.star_decode_step(x["qd"][t], x["kd"][t], x["vd"][t]) for t in range(T)]
     torch.cuda.synchronize()
+    assert cache.device_error() == 0, "a kernel gave up a bounded pipeline wait"
     return cache, O, LSE, Oq, LSEq, dec
 
 

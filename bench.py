@@ -13,7 +13,7 @@ Reported (one JSON line from rank 0):
                 inputs copied in and results copied out inside the timed region
   cpu_baseline -- the fp64 oracle on a bounded sample, extrapolated
 
-L2 is flushed (a 256 MB write) before every timed kernel region; the flush is
+L2 is flushed (a 512 MB write) before every timed kernel region; the flush is
 outside the CUDA-event brackets.  Multi-GPU runs are independent replicas
 (the single-GPU path has no exchange step): value = all ranks' tokens / the
 slowest rank's time.
@@ -68,7 +68,7 @@ def decode_bytes(w, t):
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -78,14 +78,25 @@ class Clocks:
         self.path = os.path.join("/tmp", f"star_clocks_{os.getpid()}.csv")
 
     def start(self):
+        """Start sampling (call before warm-up: nvidia-smi takes a moment to start)."""
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark(self, begin: bool):
+        """Wall-clock bounds of the timed region; samples outside it are ignored."""
+        import datetime
+        now = datetime.datetime.now()
+        if begin:
+            self.t0 = now
+        else:
+            self.t1 = now
 
     def stop(self):
         if self.proc is None:
@@ -93,18 +104,27 @@ class Clocks:
         self.proc.terminate()
         self.proc.wait()
         self.f.close()
+        import datetime
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+        inside = [r for r in rows if self.t0 and self.t1 and
+                  self.t0 - datetime.timedelta(milliseconds=150) <= r[0] <= self.t1]
+        if not inside and rows and self.t1:
+            inside = [min(rows, key=lambda r: abs((r[0] - self.t1).total_seconds()))]
+        for ts, clk, cmax, rs in inside:
+            sm.append(clk)
+            mx = cmax
+            for n, v in zip(names, rs):
                 if v.lower() == "active":
                     reasons.add(n)
         os.unlink(self.path)
@@ -173,6 +193,39 @@ def _blas_threads():
     return os.cpu_count()
 
 
+def measure_long_decode(dev, flush, warmup, steps, world):
+    """Decode steps at 128K context (the 8B-128K workload), L2 flushed before each."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+    w = wl.get("8b-128k-needle")
+    x = wl.make_inputs(w, dev)
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+    cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
+    cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
+    del x["Qc"]
+    stream = torch.cuda.current_stream(dev)
+    o = torch.empty((w.B, w.Hq, 1, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    n = min(w.T, warmup + steps)
+    ms = []
+    for t in range(n):
+        flush.fill_(5.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cache.star_decode_step(x["qd"][t], x["kd"][t], x["vd"][t], o, lse)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize(dev)
+    times = [a.elapsed_time(b) for a, b in ms[warmup:]]
+    t = torch.tensor([sum(times) / len(times)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    cache.close()
+    del x
+    torch.cuda.empty_cache()
+    return w, t.item() * 1e3
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -228,12 +281,14 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="star", choices=["star", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-long-decode", action="store_true",
+                    help="skip the decode measurement at 128K context")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -252,7 +307,9 @@ def main():
     LSEq = torch.empty((w.B, w.Hq, w.lq), dtype=torch.float32, device=dev)
     od = torch.empty((w.T, w.B, w.Hq, 1, w.D), dtype=torch.bfloat16, device=dev)
     lsed = torch.empty((w.T, w.B, w.Hq), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    # 512 MB: larger than L2, and long enough (~80 us) for the host to queue the
+    # timed launch behind it, so the start event is not recorded on an idle GPU
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def ev():
@@ -279,20 +336,22 @@ def main():
             dec.append((a, b))
         times.append(((e0, e1), (e2, e3), dec))
 
+    clocks = Clocks(local)
+    clocks.start()
     for _ in range(args.warmup):
         step([])
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    clocks = Clocks(local)
-    clocks.start()
     torch.cuda.synchronize(dev)
+    clocks.mark(True)
     t_wall = time.perf_counter()
     times = []
     for _ in range(args.steps):
         step(times)
     torch.cuda.synchronize(dev)
     wall = time.perf_counter() - t_wall
+    clocks.mark(False)
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
@@ -337,6 +396,10 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "what": "H2D of Q,K,V from pinned host + star_ctx_encode + D2H of O,LSE"}
 
+    long_dec = None
+    if not args.no_long_decode:
+        long_dec = measure_long_decode(dev, flush, args.warmup, args.steps, world)
+
     pk = peaks()
     flops, _ = phase1_flops(w)
     enc_avg_s = enc_total / args.steps / 1e3
@@ -353,7 +416,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
                    "block": w.b, "anchor": w.b_a, "lq": w.lq, "decode_steps": w.T,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed (256 MB write) before every timed kernel region"},
+                   "l2": "flushed (512 MB write) before every timed kernel region"},
         "decode": {"value": world * w.B * w.T / dec_avg_s, "unit": "decode tok/s",
                    "us_per_step": dec_avg_s / w.T * 1e6,
                    "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"],
@@ -370,6 +433,17 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
+    if long_dec:
+        wl2, t_us = long_dec
+        lb = sum(decode_bytes(wl2, wl2.lq + t) for t in range(1)) / 1.0
+        gbs = decode_bytes(wl2, 0) / (t_us * 1e-6) / 1e9
+        line["decode_long"] = {
+            "workload": wl2.name, "value": world * wl2.B / (t_us * 1e-6), "unit": "decode tok/s",
+            "us_per_step": t_us,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "bytes_per_step": decode_bytes(wl2, 0)}}
+        del lb
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d, sample, threads = cpu_oracle_sample(w, x)
         line["cpu_baseline"] = {"value": v, "unit": "ctx tok/s", "cores": threads, "kind": "oracle",

@@ -185,36 +185,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
       const uint32_t id_pv = idesc_bf16_f32(BM, D, true);
       const uint32_t sO[2] = {tmem + 256, tmem + 256 + D};
       const uint32_t sS[2] = {tmem, tmem + 128};
-      bool ok = mbar_wait(smem_u32(&bar_q_full), 0);
-      if (!ok) fail();
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int ik = 2 * j, iv = 2 * j + 1;
-        const int sk = ik % NBUF, sv = iv % NBUF;
-        if (!mbar_wait(smem_u32(&bar_kv_full[sk]), (ik / NBUF) & 1)) { fail(); break; }
-        tc_fence_after();
-        const uint32_t kbase = smem_u32(smem + S::RING + sk * S::TILE);
-        for (int q = 0; q < nq; ++q) {
-          const uint32_t qbase = smem_u32(smem + (q ? S::Q1 : S::Q0));
+      // Issue order per K/V tile j (two heads):
+      //   PV0(j), S0(j+1), PV1(j), S1(j+1)
+      // so the tensor core computes head 0's next scores while head 1's
+      // softmax still runs, and the other way round.
+      auto issue_s = [&](int q, uint32_t kbase) {
+        const uint32_t qbase = smem_u32(smem + (q ? S::Q1 : S::Q0));
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * S::HALF + (kk & 3) * 32;
-            mma_ss(sS[q], smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                   id_qk, kk > 0);
-          }
-          mma_commit(smem_u32(&bar_s_full[q]));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * S::HALF + (kk & 3) * 32;
+          mma_ss(sS[q], smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                 id_qk, kk > 0);
         }
-        mma_commit(smem_u32(&bar_kv_empty[sk]));
-        if (!mbar_wait(smem_u32(&bar_kv_full[sv]), (iv / NBUF) & 1)) { fail(); break; }
-        const uint32_t vbase = smem_u32(smem + S::RING + sv * S::TILE);
+        mma_commit(smem_u32(&bar_s_full[q]));
+      };
+      auto issue_pv = [&](int q, uint32_t vbase, int j) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(sO[q], sS[q] + kk * 8, smem_desc_sw128(vbase + kk * 2048, S::HALF, 1024), id_pv,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      auto kv_slot = [&](int i) { return smem_u32(smem + S::RING + (i % NBUF) * S::TILE); };
+      bool ok = mbar_wait(smem_u32(&bar_q_full), 0) && mbar_wait(smem_u32(&bar_kv_full[0]), 0);
+      if (!ok) fail();
+      if (ok) {
+        tc_fence_after();
+        for (int q = 0; q < nq; ++q) issue_s(q, kv_slot(0));
+        mma_commit(smem_u32(&bar_kv_empty[0]));
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int iv = 2 * j + 1, ik = 2 * j + 2;       // ring indices of V_j and K_{j+1}
+        const bool more = j + 1 < n_kv;
+        if (!mbar_wait(smem_u32(&bar_kv_full[iv % NBUF]), (iv / NBUF) & 1)) { fail(); break; }
+        if (more && !mbar_wait(smem_u32(&bar_kv_full[ik % NBUF]), (ik / NBUF) & 1)) { fail(); break; }
         for (int q = 0; q < nq; ++q) {
           if (!mbar_wait(smem_u32(&bar_p_full[q]), j & 1)) { fail(); ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ts(sO[q], sS[q] + kk * 8, smem_desc_sw128(vbase + kk * 2048, S::HALF, 1024), id_pv,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+          issue_pv(q, kv_slot(iv), j);
+          if (more) issue_s(q, kv_slot(ik));
         }
-        mma_commit(smem_u32(&bar_kv_empty[sv]));
+        if (!ok) break;
+        mma_commit(smem_u32(&bar_kv_empty[iv % NBUF]));
+        if (more) mma_commit(smem_u32(&bar_kv_empty[ik % NBUF]));
         if (*(volatile int*)&abort_s) break;
       }
       mma_commit(smem_u32(&bar_o_full));

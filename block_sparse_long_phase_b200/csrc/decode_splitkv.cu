@@ -1,309 +1,495 @@
-// Phase-2 generation step: split-KV HBM-streaming attention with a fused
+// Phase-2 generation step: split-KV, HBM-streaming attention with a fused
 // log-sum-exp merge.
 //
 // "Star Attention: Efficient LLM Inference over Long Sequences" (analysis
 // page), section 3.4, "Phase 2: Query Encoding and Token Generation with
 // Distributed Softmax": every context block ("host") computes the local
-// attention A_h and its exponent sum s_h for the new token (Step 3), the
-// partials are combined with the log-sum-exp rule (Step 5), and only the query
-// region's cache grows (Step 7).  On one GPU each CTA plays a "host" for one
-// contiguous chunk of the (batch, kv head)'s key sequence
-// [context segments | query region | new token]; chunks are sized so that the
-// grid is two CTAs per SM.  The last CTA of each (batch, kv head) to finish --
-// chosen by an atomic ticket, no CTA ever waits for another -- merges that
-// head's partials and writes the output.
+// attention A_h of the new token and the log of its exponent sum s_h (Step 3);
+// the partials are combined with the log-sum-exp rule (Step 5); only the
+// query region's cache grows (Step 7).
 //
-// Inside a CTA: the G query heads that share the kv head are the M rows of a
-// 16x8x16 bf16 MMA (rows G..15 are zero), K/V stream through a 3-stage
-// cp.async ring of 64-key stages in XOR-swizzled shared memory, and each of
-// the 4 warps owns 16 keys of every stage with its own online softmax; the
-// warps' states are combined in shared memory at the end.
+// One GPU plays all the hosts.  The cached keys of every (batch, kv head) --
+// its context segments, then its query region -- are laid end to end and cut
+// into one balanced span per CTA (one CTA per SM), so each CTA streams the
+// same number of bytes whatever the segment sizes.  Inside a CTA:
+//   warp 0     TMA producer: 128-key K and V stages (128-byte swizzled boxes)
+//              of the span, never crossing a segment, through a 3-slot ring;
+//   warps 1-8  consumers: each owns 16 keys of every stage; the G query heads
+//              of the kv group are the M rows of a 16x8x16 bf16 MMA (rows G..15
+//              zero), online softmax in base 2, fp32 accumulation.
+// When a span ends a (batch, kv head) piece, the consumer warps combine their
+// states in shared memory into one partial (A, s) of that piece; the CTA that
+// holds the piece's last cached row also folds in the new token (attended
+// from its input k, v, which it appends to the query region).  The last CTA
+// of a (batch, kv head) to finish -- an atomic ticket, no CTA ever waits for
+// another -- merges that head's partials and writes o and lse.
 #include <cuda_bf16.h>
 #include <math.h>
+#include <string.h>
 
+#include "sm100_primitives.cuh"
 #include "star_common.cuh"
 #include "star_internal.h"
+#include "tmap.h"
 
 namespace star {
 namespace {
 
-constexpr int KS = 64;        // keys per stage
+using namespace sm100;
+
+constexpr int KS = 128;                 // keys per stage
 constexpr int NSTAGE = 3;
-constexpr int NTHREADS = 128;
+constexpr int NCW = 8;                  // consumer warps
+constexpr int NTHREADS = 32 * (NCW + 1);
+constexpr int kMaxG = 16;
+
+struct StageMeta {
+  int n;         // valid keys in the stage
+  int last;      // 1: the stage ends a (batch, kv head) piece of this span
+  int bg;        // batch * Hkv + kv head
+  int pad;
+};
 
 struct DecodeArgs {
+  CUtensorMap tk_ctx, tv_ctx;   // context cache as [B*Hkv*L][D]
+  CUtensorMap tk_q, tv_q;       // query region as [B*Hkv*q_cap][D]
   CacheView c;
   float scale_log2;
-  int len0;                   // query-region rows before this step
-  int cph;                    // chunks per (batch, kv head)
-  int chunk_rows;
-  const bf16* q;              // [B][Hq][D]
-  const bf16* k;              // [B][Hkv][D]
+  int len0;                     // query-region rows before this step
+  int ncta;
+  int maxp;                     // partial slots per (batch, kv head)
+  long long rpb;                // cached rows per (batch, kv head): L + len0
+  const bf16* q;                // [B][Hq][D]
+  const bf16* k;                // [B][Hkv][D]
   const bf16* v;
-  bf16* o;                    // [B][Hq][D]
-  float* lse;                 // [B][Hq]
-  float* partA;               // [B*Hkv][cph][G][D]
-  float* partS;               // [B*Hkv][cph][G]
-  unsigned* tickets;          // [B*Hkv]
+  bf16* o;                      // [B][Hq][D]
+  float* lse;                   // [B][Hq]
+  float* partA;                 // [B*Hkv][maxp][G][D]
+  float* partS;                 // [B*Hkv][maxp][G]
+  unsigned* tickets;            // [B*Hkv]
+  int* err;
+};
+
+__device__ __forceinline__ long long span_start(long long i, long long R, int n) {
+  return i * R / n;
+}
+// CTA whose span holds global cached row x (largest i with span_start(i) <= x).
+__device__ __forceinline__ int cta_of(long long x, long long R, int n) {
+  return (int)(((x + 1) * n - 1) / R);
+}
+
+SM100_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
+
+template <int D>
+struct DSmem {
+  static constexpr int HALF = KS * 128;               // one 64-column half of a stage tile
+  static constexpr int TILE = KS * D * 2;              // K (or V) of one stage
+  static constexpr int STAGE = 2 * TILE;
+  // 4 rows of O per warp per round; also holds the merge weights (<= 16 x 160)
+  static constexpr int COMB = NCW * 4 * 128 * 4;
+  static constexpr int BYTES = NSTAGE * STAGE + COMB;
 };
 
 template <int D>
-__global__ void __launch_bounds__(NTHREADS) decode_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int CPR = D / 8;
-  constexpr int STAGE_BYTES = KS * D * 2;
+__global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
+  using S = DSmem<D>;
+  constexpr int NH = D / 64;
   constexpr int NT_O = D / 8;
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* sQ = smem;                               // 16 x D bf16
-  uint8_t* sK = smem + 16 * D * 2;                  // NSTAGE stages
-  uint8_t* sV = sK + NSTAGE * STAGE_BYTES;
-  __shared__ int s_last;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  float* comb = reinterpret_cast<float*>(smem + NSTAGE * S::STAGE);   // [NCW][4][D]
+  __shared__ __align__(8) uint64_t bar_full[NSTAGE];
+  __shared__ __align__(8) uint64_t bar_empty[NSTAGE];
+  __shared__ StageMeta meta[NSTAGE];
+  __shared__ float wm[NCW][16], wl[NCW][16];
+  __shared__ float s_new[kMaxG];
+  __shared__ float s_lse[kMaxG];
+  __shared__ int s_last, abort_s;
 
   const CacheView& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bg = blockIdx.x / a.cph;
-  const int chunk = blockIdx.x - bg * a.cph;
-  const int bb = bg / c.Hkv, g = bg - bb * c.Hkv;
   const int G = c.G;
-  const int Lc = (int)c.L;
-  const int n_keys_total = Lc + a.len0 + 1;
-  const int j_begin = chunk * a.chunk_rows;
-  int j_end = j_begin + a.chunk_rows;
-  if (j_end > n_keys_total) j_end = n_keys_total;
-  const int nk = j_end > j_begin ? j_end - j_begin : 0;
-  const int n_st = (nk + KS - 1) / KS;
+  const long long R = (long long)c.B * c.Hkv * a.rpb;
+  const long long x0 = span_start(blockIdx.x, R, a.ncta);
+  const long long x1 = span_start(blockIdx.x + 1, R, a.ncta);
 
-  const bf16* knew = a.k + (long long)bg * D;
-  const bf16* vnew = a.v + (long long)bg * D;
-
-  // Append the new token to the query region (readers in this launch take it
-  // from the input, so the write order does not matter).
-  if (chunk == a.cph - 1 && tid < CPR) {
-    const long long off = q_row_offset(c, bb, g, a.len0);
-    reinterpret_cast<uint4*>(c.qK + off)[tid] = reinterpret_cast<const uint4*>(knew)[tid];
-    reinterpret_cast<uint4*>(c.qV + off)[tid] = reinterpret_cast<const uint4*>(vnew)[tid];
-  }
-
-  auto row_ptr = [&](int j, bool v) -> const bf16* {
-    if (j < Lc) {
-      const int seg = j / c.b;
-      const int off = j - seg * c.b;
-      const long long len = seg_len(c, seg);
-      const long long base = (long long)seg * c.B * c.Hkv * (long long)c.b * D +
-                             (((long long)bb * c.Hkv + g) * len + off) * D;
-      return (v ? c.ctxV : c.ctxK) + base;
+  if (tid == 0) {
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(smem_u32(&bar_full[i]), 1);
+      mbar_init(smem_u32(&bar_empty[i]), NCW);
     }
-    if (j < Lc + a.len0) return (v ? c.qV : c.qK) + q_row_offset(c, bb, g, j - Lc);
-    return v ? vnew : knew;
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto fail = [&]() {
+    *(volatile int*)&abort_s = 1;
+    atomicExch(a.err, 1);
   };
-  auto load_stage = [&](int slot, int st) {
-    const int j0 = j_begin + st * KS;
-    const uint32_t dk = smem_u32(sK + slot * STAGE_BYTES);
-    const uint32_t dv = smem_u32(sV + slot * STAGE_BYTES);
-    for (int i = tid; i < KS * CPR; i += NTHREADS) {
-      const int row = i / CPR, ch = i - (i / CPR) * CPR;
-      const int j = j0 + row;
-      const bool ok = j < j_end;
-      const bf16* kp = ok ? row_ptr(j, false) : knew;
-      const bf16* vp = ok ? row_ptr(j, true) : vnew;
-      cp_async16(dk + swz(row, ch, CPR), kp + ch * 8, ok ? 16 : 0);
-      cp_async16(dv + swz(row, ch, CPR), vp + ch * 8, ok ? 16 : 0);
+  auto aborted = [&]() { return *(volatile int*)&abort_s != 0; };
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (elect_one()) {
+      prefetch_tmap(&a.tk_ctx);
+      prefetch_tmap(&a.tv_ctx);
+      prefetch_tmap(&a.tk_q);
+      prefetch_tmap(&a.tv_q);
+      int last_use[NSTAGE];
+      for (int k = 0; k < NSTAGE; ++k) last_use[k] = -1;
+      long long x = x0;
+      for (int st = 0; x < x1; ++st) {
+        const int bg = (int)(x / a.rpb);
+        const long long off = x - (long long)bg * a.rpb;           // key index within (b, g)
+        const long long piece_end = ((long long)bg + 1) * a.rpb < x1 ? ((long long)bg + 1) * a.rpb : x1;
+        long long region_end;
+        int row;
+        bool ctx;
+        if (off < c.L) {
+          const int seg = (int)(off / c.b);
+          const long long len = seg_len(c, seg);
+          region_end = (long long)seg * c.b + len;
+          row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * len + (off - (long long)seg * c.b));
+          ctx = true;
+        } else {
+          region_end = a.rpb;
+          row = (int)((long long)bg * c.q_cap + (off - c.L));
+          ctx = false;
+        }
+        long long n = KS;
+        if (region_end - off < n) n = region_end - off;
+        if (piece_end - x < n) n = piece_end - x;
+        const int slot = st % NSTAGE, use = st / NSTAGE;
+        if (use > 0 && !mbar_wait(smem_u32(&bar_empty[slot]), (use - 1) & 1)) { fail(); break; }
+        if (aborted()) break;
+        meta[slot].n = (int)n;
+        meta[slot].last = (x + n == piece_end) ? 1 : 0;
+        meta[slot].bg = bg;
+        const uint32_t fb = smem_u32(&bar_full[slot]);
+        mbar_arrive_expect_tx(fb, S::STAGE);
+        const uint32_t dst = smem_u32(smem + slot * S::STAGE);
+        for (int hf = 0; hf < NH; ++hf) {
+          tma_load_2d(dst + hf * S::HALF, ctx ? &a.tk_ctx : &a.tk_q, hf * 64, row, fb);
+          tma_load_2d(dst + S::TILE + hf * S::HALF, ctx ? &a.tv_ctx : &a.tv_q, hf * 64, row, fb);
+        }
+        last_use[slot] = use;
+        x += n;
+      }
+      if (aborted())
+        for (int k = 0; k < NSTAGE; ++k)
+          if (last_use[k] >= 0) mbar_wait(smem_u32(&bar_full[k]), last_use[k] & 1);
     }
-  };
-
-  // Q rows 0..G-1 of this kv group, zero beyond.
-  for (int i = tid; i < 16 * CPR; i += NTHREADS) {
-    const int row = i / CPR, ch = i - (i / CPR) * CPR;
-    const bool ok = row < G;
-    const bf16* src = a.q + ((long long)bb * c.Hq + g * G + (ok ? row : 0)) * D + ch * 8;
-    cp_async16(smem_u32(sQ) + swz(row, ch, CPR), src, ok ? 16 : 0);
-  }
-#pragma unroll
-  for (int s = 0; s < NSTAGE - 1; ++s) {
-    if (s < n_st) load_stage(s, s);
-    cp_async_commit();
+    return;   // the producer takes part in no named barrier
   }
 
+  // --------------------------------- consumers --------------------------------
+  const int cw = warp - 1;                       // consumer warp 0..7
+  const int ctid = tid - 32;                     // 0..255
   uint32_t qa[D / 16][4];
   float o[NT_O][4];
-#pragma unroll
-  for (int n = 0; n < NT_O; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-
-  for (int st = 0; st < n_st; ++st) {
-    const int slot = st % NSTAGE;
-    if (st + NSTAGE - 1 < n_st) load_stage((st + NSTAGE - 1) % NSTAGE, st + NSTAGE - 1);
-    cp_async_commit();
-    cp_async_wait<NSTAGE - 1>();
-    __syncthreads();
-    if (st == 0) {
-#pragma unroll
-      for (int kd = 0; kd < D / 16; ++kd) {
-        const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ch = 2 * kd + (lane >> 4);
-        ldmatrix_x4(smem_u32(sQ) + swz(row, ch, CPR), qa[kd][0], qa[kd][1], qa[kd][2], qa[kd][3]);
-      }
-    }
-    const uint32_t kbase = smem_u32(sK + slot * STAGE_BYTES);
-    const uint32_t vbase = smem_u32(sV + slot * STAGE_BYTES);
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  int cur_bg = -1;
+  auto load_q = [&](int bg) {
+    const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+    const int r0 = lane >> 2, r1 = r0 + 8;
+    const bf16* qb = a.q + ((long long)bb * c.Hq + (long long)g * G) * D;
 #pragma unroll
     for (int kd = 0; kd < D / 16; ++kd) {
-      const int row = 16 * warp + (lane & 7) + ((lane >> 4) << 3);
-      const int ch = 2 * kd + ((lane >> 3) & 1);
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(kbase + swz(row, ch, CPR), b0, b1, b2, b3);
-      mma_bf16_16816(s[0], qa[kd], b0, b1);
-      mma_bf16_16816(s[1], qa[kd], b2, b3);
+      const int col = 16 * kd + 2 * (lane & 3);
+      qa[kd][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col) : 0u;
+      qa[kd][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col) : 0u;
+      qa[kd][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col + 8) : 0u;
+      qa[kd][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col + 8) : 0u;
     }
-    const int jw = j_begin + st * KS + 16 * warp;   // first key of this warp
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
+    for (int n = 0; n < NT_O; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    m_a = m_b = -INFINITY;
+    l_a = l_b = 0.f;
+  };
+
+  long long x = x0;
+  for (int st = 0; x < x1; ++st) {
+    const int slot = st % NSTAGE, use = st / NSTAGE;
+    bool ok = !aborted() && mbar_wait(smem_u32(&bar_full[slot]), use & 1);
+    if (!ok) fail();
+    const StageMeta m = meta[slot];
+    const int n = ok ? m.n : (int)(x1 - x < KS ? x1 - x : KS);
+    const int bg = ok ? m.bg : (int)(x / a.rpb);
+    const bool last = ok ? (m.last != 0) : true;
+    if (bg != cur_bg) {
+      load_q(bg);
+      cur_bg = bg;
+    }
+    if (ok) {
+      const uint32_t kb = smem_u32(smem + slot * S::STAGE);
+      const uint32_t vb = kb + S::TILE;
+      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = jw + 8 * n + 2 * (lane & 3) + (e & 1);
-        s[n][e] = j < j_end ? s[n][e] * a.scale_log2 : -INFINITY;
+      for (int kd = 0; kd < D / 16; ++kd) {
+        const int row = 16 * cw + (lane & 7) + ((lane >> 4) << 3);
+        const int ch = 2 * kd + ((lane >> 3) & 1);
+        const uint32_t addr = kb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(addr, b0, b1, b2, b3);
+        mma_bf16_16816(s[0], qa[kd], b0, b1);
+        mma_bf16_16816(s[1], qa[kd], b2, b3);
+      }
+      const int kw = 16 * cw;   // first key of this warp in the stage
+#pragma unroll
+      for (int nn = 0; nn < 2; ++nn)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = kw + 8 * nn + 2 * (lane & 3) + (e & 1);
+          s[nn][e] = j < n ? s[nn][e] * a.scale_log2 : -INFINITY;
+        }
+      float mx_a = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      float mx_b = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+      // The exponent base only moves up when a row's maximum grows by more
+      // than 2^8, so the accumulator is rarely rescaled.
+      const bool up_a = mx_a > m_a + 8.f, up_b = mx_b > m_b + 8.f;
+      if (__any_sync(0xffffffffu, up_a || up_b)) {
+        const float al_a = up_a ? exp2f(m_a - mx_a) : 1.f;
+        const float al_b = up_b ? exp2f(m_b - mx_b) : 1.f;
+        if (up_a) m_a = mx_a;
+        if (up_b) m_b = mx_b;
+        l_a *= al_a;
+        l_b *= al_b;
+#pragma unroll
+        for (int nn = 0; nn < NT_O; ++nn) {
+          o[nn][0] *= al_a;
+          o[nn][1] *= al_a;
+          o[nn][2] *= al_b;
+          o[nn][3] *= al_b;
+        }
+      }
+      const float base_a = m_a == -INFINITY ? 0.f : m_a;
+      const float base_b = m_b == -INFINITY ? 0.f : m_b;
+#pragma unroll
+      for (int nn = 0; nn < 2; ++nn) {
+        s[nn][0] = exp2f(s[nn][0] - base_a);
+        s[nn][1] = exp2f(s[nn][1] - base_a);
+        s[nn][2] = exp2f(s[nn][2] - base_b);
+        s[nn][3] = exp2f(s[nn][3] - base_b);
+      }
+      l_a += s[0][0] + s[0][1] + s[1][0] + s[1][1];
+      l_b += s[0][2] + s[0][3] + s[1][2] + s[1][3];
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[0][0], s[0][1]);
+      pa[1] = pack_bf16(s[0][2], s[0][3]);
+      pa[2] = pack_bf16(s[1][0], s[1][1]);
+      pa[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+      for (int j = 0; j < D / 16; ++j) {
+        const int row = 16 * cw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int ch = 2 * j + (lane >> 4);
+        const uint32_t addr = vb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(addr, b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * j], pa, b0, b1);
+        mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_empty[slot]));
+    }
+    x += n;
+    if (!last) continue;
+
+    // ---- piece epilogue: one partial (A, s) for (bg, this CTA) ---------------
+    const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+    const long long first_row = (long long)bg * a.rpb;
+    const int first = cta_of(first_row, R, a.ncta);
+    const int lastc = cta_of(first_row + a.rpb - 1, R, a.ncta);
+    const bool owns_new = (int)blockIdx.x == lastc;          // holds the piece's last cached row
+    const int pslot = (int)blockIdx.x - first;
+    const int count = lastc - first + 1;
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    if (owns_new) {
+      // score of the new token for every head of the group (warp r: head r)
+      const bf16* kn = a.k + (long long)bg * D;
+      for (int r = cw; r < G; r += NCW) {
+        const bf16* qr = a.q + (((long long)bb * c.Hq + (long long)g * G + r) * D);
+        float acc = 0.f;
+        for (int d = lane; d < D; d += 32) acc += __bfloat162float(qr[d]) * __bfloat162float(kn[d]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) s_new[r] = acc * a.scale_log2;
       }
     }
-    float mx_a = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-    float mx_b = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-    const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
-    const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
-    const float al_a = exp2f(m_a - base_a), al_b = exp2f(m_b - base_b);
-    m_a = mn_a;
-    m_b = mn_b;
+    for (int rh = 0; rh < G; rh += 4) {            // rows rh .. rh+3 per round
+      const int ra = lane >> 2, rb = ra + 8;       // fragment rows of this thread
+      if ((lane & 3) == 0) {
+        wm[cw][ra] = m_a;
+        wm[cw][rb] = m_b;
+        wl[cw][ra] = l_a;
+        wl[cw][rb] = l_b;
+      }
+      const int cq = 2 * (lane & 3);
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
-      s[n][0] = exp2f(s[n][0] - base_a);
-      s[n][1] = exp2f(s[n][1] - base_a);
-      s[n][2] = exp2f(s[n][2] - base_b);
-      s[n][3] = exp2f(s[n][3] - base_b);
-    }
-    l_a = l_a * al_a + s[0][0] + s[0][1] + s[1][0] + s[1][1];
-    l_b = l_b * al_b + s[0][2] + s[0][3] + s[1][2] + s[1][3];
-    uint32_t pa[4];
-    pa[0] = pack_bf16(s[0][0], s[0][1]);
-    pa[1] = pack_bf16(s[0][2], s[0][3]);
-    pa[2] = pack_bf16(s[1][0], s[1][1]);
-    pa[3] = pack_bf16(s[1][2], s[1][3]);
+      for (int nn = 0; nn < NT_O; ++nn) {
+        if (ra >= rh && ra < rh + 4) {
+          comb[(cw * 4 + ra - rh) * D + 8 * nn + cq] = o[nn][0];
+          comb[(cw * 4 + ra - rh) * D + 8 * nn + cq + 1] = o[nn][1];
+        }
+        if (rb >= rh && rb < rh + 4) {
+          comb[(cw * 4 + rb - rh) * D + 8 * nn + cq] = o[nn][2];
+          comb[(cw * 4 + rb - rh) * D + 8 * nn + cq + 1] = o[nn][3];
+        }
+      }
+      named_sync(1, 32 * NCW);
+      const int rows = G - rh < 4 ? G - rh : 4;
+      for (int idx = ctid; idx < rows * D; idx += 32 * NCW) {
+        const int r = idx / D, d = idx - (idx / D) * D, rr = rh + r;
+        float M = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < D / 16; ++j) {
-      o[2 * j][0] *= al_a;
-      o[2 * j][1] *= al_a;
-      o[2 * j][2] *= al_b;
-      o[2 * j][3] *= al_b;
-      o[2 * j + 1][0] *= al_a;
-      o[2 * j + 1][1] *= al_a;
-      o[2 * j + 1][2] *= al_b;
-      o[2 * j + 1][3] *= al_b;
-      const int row = 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int ch = 2 * j + (lane >> 4);
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4_trans(vbase + swz(row, ch, CPR), b0, b1, b2, b3);
-      mma_bf16_16816(o[2 * j], pa, b0, b1);
-      mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-
-  // ---- combine the 4 warps (shared memory reuses the K ring) ---------------
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-  float* wm = reinterpret_cast<float*>(sK);          // [4][16]
-  float* wl = wm + 4 * 16;                            // [4][16]
-  float* wo = wl + 4 * 16;                            // [4][16][D]
-  const int ra = lane >> 2, rb = ra + 8, cq = 2 * (lane & 3);
-  if ((lane & 3) == 0) {
-    wm[warp * 16 + ra] = m_a;
-    wm[warp * 16 + rb] = m_b;
-    wl[warp * 16 + ra] = l_a;
-    wl[warp * 16 + rb] = l_b;
-  }
+        for (int w = 0; w < NCW; ++w) M = fmaxf(M, wm[w][rr]);
+        if (owns_new) M = fmaxf(M, s_new[rr]);
+        const float base = M == -INFINITY ? 0.f : M;
+        float Ls = 0.f, acc = 0.f;
 #pragma unroll
-  for (int n = 0; n < NT_O; ++n) {
-    wo[(warp * 16 + ra) * D + 8 * n + cq] = o[n][0];
-    wo[(warp * 16 + ra) * D + 8 * n + cq + 1] = o[n][1];
-    wo[(warp * 16 + rb) * D + 8 * n + cq] = o[n][2];
-    wo[(warp * 16 + rb) * D + 8 * n + cq + 1] = o[n][3];
-  }
-  __syncthreads();
-  const long long pbase = ((long long)bg * a.cph + chunk) * G;
-  for (int idx = tid; idx < G * D; idx += NTHREADS) {
-    const int r = idx / D, d = idx - (idx / D) * D;
-    float M = -INFINITY;
+        for (int w = 0; w < NCW; ++w) {
+          const float f = exp2f(wm[w][rr] - base);
+          Ls += f * wl[w][rr];
+          acc += f * comb[(w * 4 + r) * D + d];
+        }
+        if (owns_new) {
+          const float f = exp2f(s_new[rr] - base);
+          Ls += f;
+          acc += f * __bfloat162float(a.v[(long long)bg * D + d]);
+        }
+        const long long pr = ((long long)bg * a.maxp + pslot) * G + rr;
+        a.partA[pr * D + d] = Ls > 0.f ? acc / Ls : 0.f;
+        if (d == 0) a.partS[pr] = Ls > 0.f ? (base + log2f(Ls)) * kLn2 : -INFINITY;
+      }
+      named_sync(1, 32 * NCW);
+    }
+    if (owns_new && ctid < D / 8) {
+      // append the new token to the query region (row len0); no reader in this launch
+      const long long qo = q_row_offset(c, bb, g, a.len0);
+      reinterpret_cast<uint4*>(c.qK + qo)[ctid] = reinterpret_cast<const uint4*>(a.k + (long long)bg * D)[ctid];
+      reinterpret_cast<uint4*>(c.qV + qo)[ctid] = reinterpret_cast<const uint4*>(a.v + (long long)bg * D)[ctid];
+    }
+    // ticket: the last CTA of this (batch, kv head) merges its partials.  The
+    // barrier orders every consumer's partial stores before thread 0's
+    // gpu-scope release fence (cumulative), which precedes the ticket.
+    named_sync(1, 32 * NCW);
+    if (ctid == 0) {
+      __threadfence();
+      s_last = (atomicAdd(&a.tickets[bg], 1u) == (unsigned)(count - 1));
+    }
+    named_sync(1, 32 * NCW);
+    if (s_last) {
+      __threadfence();
+      // merge weights: load every s_h once (in parallel), then per-row max/sum
+      float* sv = comb;                           // [G][count] log-sum-exps, then weights
+      for (int i = ctid; i < G * count; i += 32 * NCW) {
+        const int r = i / count, p = i - (i / count) * count;
+        sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + p) * G + r);
+      }
+      named_sync(1, 32 * NCW);
+      if (ctid < G) {
+        const int r = ctid;
+        float M = -INFINITY;
+        for (int p = 0; p < count; ++p) M = fmaxf(M, sv[r * count + p]);
+        const float base = M == -INFINITY ? 0.f : M;
+        float tot = 0.f;
+        for (int p = 0; p < count; ++p) tot += __expf(sv[r * count + p] - base);
+        const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
+        s_lse[r] = l;
+        for (int p = 0; p < count; ++p) {
+          const float sp = sv[r * count + p];
+          sv[r * count + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
+        }
+      }
+      named_sync(1, 32 * NCW);
+      // weighted sum over the partials: float4 columns, eight loads in flight
+      for (int idx = ctid; idx < G * (D / 4); idx += 32 * NCW) {
+        const int r = idx / (D / 4), d4 = idx - (idx / (D / 4)) * (D / 4);
+        const float4* pa = reinterpret_cast<const float4*>(a.partA + ((long long)bg * a.maxp * G + r) * D) + d4;
+        const long long pstride = (long long)G * D / 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p0 = 0; p0 < count; p0 += 8) {
+          float4 v16[8];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w * 16 + r]);
-    const float base = M == -INFINITY ? 0.f : M;
-    float Lsum = 0.f, acc = 0.f;
+          for (int u = 0; u < 8; ++u)
+            v16[u] = p0 + u < count ? __ldcg(pa + (p0 + u) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = exp2f(wm[w * 16 + r] - base);
-      Lsum += f * wl[w * 16 + r];
-      acc += f * wo[(w * 16 + r) * D + d];
+          for (int u = 0; u < 8; ++u) {
+            const float wgt = p0 + u < count ? sv[r * count + p0 + u] : 0.f;
+            acc.x += wgt * v16[u].x;
+            acc.y += wgt * v16[u].y;
+            acc.z += wgt * v16[u].z;
+            acc.w += wgt * v16[u].w;
+          }
+        }
+        const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
+        uint2 pk;
+        pk.x = pack_bf16(acc.x, acc.y);
+        pk.y = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+        if (d4 == 0) a.lse[orow] = s_lse[r];
+      }
+      if (ctid == 0) a.tickets[bg] = 0u;   // ready for the next step
+      named_sync(1, 32 * NCW);
     }
-    a.partA[(pbase + r) * D + d] = Lsum > 0.f ? acc / Lsum : 0.f;
-    if (d == 0) a.partS[pbase + r] = Lsum > 0.f ? (base + log2f(Lsum)) * kLn2 : -INFINITY;
+    cur_bg = -1;                            // the next piece reloads q and resets the state
   }
-
-  // ---- last CTA of this (batch, kv head) merges ----------------------------
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.tickets[bg], 1u) == (unsigned)(a.cph - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float* wts = reinterpret_cast<float*>(sV);          // [G][cph] merge weights
-  float* lse_s = wts + G * a.cph;                     // [G]
-  if (tid < G) {
-    const int r = tid;
-    float M = -INFINITY;
-    for (int p = 0; p < a.cph; ++p)
-      M = fmaxf(M, __ldcg(a.partS + ((long long)bg * a.cph + p) * G + r));
-    const float base = M == -INFINITY ? 0.f : M;
-    float tot = 0.f;
-    for (int p = 0; p < a.cph; ++p)
-      tot += __expf(__ldcg(a.partS + ((long long)bg * a.cph + p) * G + r) - base);
-    const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
-    lse_s[r] = l;
-    for (int p = 0; p < a.cph; ++p) {
-      const float sp = __ldcg(a.partS + ((long long)bg * a.cph + p) * G + r);
-      wts[r * a.cph + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
-    }
-  }
-  __syncthreads();
-  for (int idx = tid; idx < G * D; idx += NTHREADS) {
-    const int r = idx / D, d = idx - (idx / D) * D;
-    float acc = 0.f;
-    for (int p = 0; p < a.cph; ++p) {
-      const float w = wts[r * a.cph + p];
-      if (w != 0.f) acc += w * __ldcg(a.partA + (((long long)bg * a.cph + p) * G + r) * D + d);
-    }
-    const long long orow = (long long)bb * c.Hq + g * G + r;
-    a.o[orow * D + d] = __float2bfloat16_rn(acc);
-    if (d == 0) a.lse[orow] = lse_s[r];
-  }
-  if (tid == 0) a.tickets[bg] = 0u;   // ready for the next step
 }
 
 }  // namespace
 
-cudaError_t launch_decode_step(const CacheView& c, float scale, int len0, const bf16* q,
-                               const bf16* k, const bf16* v, bf16* o, float* lse,
+int decode_max_partials(const CacheView& c, int ncta) {
+  // a (batch, kv head) of R/(B*Hkv) rows is touched by at most this many spans
+  const int bgs = c.B * c.Hkv;
+  return (ncta + bgs - 1) / bgs + 2;
+}
+
+int decode_num_ctas(const CacheView& c, long long len0, int num_sms) {
+  const long long R = (long long)c.B * c.Hkv * (c.L + len0);
+  long long n = R / 512;                    // at least 512 cached rows per span
+  if (n < 1) n = 1;
+  if (n > num_sms) n = num_sms;
+  return (int)n;
+}
+
+bool decode_make_maps(const CacheView& c, DecodeMaps* m) {
+  const unsigned long long ctx_rows = (unsigned long long)c.B * c.Hkv * c.L;
+  const unsigned long long q_rows = (unsigned long long)c.B * c.Hkv * c.q_cap;
+  return make_tmap_bf16_2d(&m->k_ctx, c.ctxK, ctx_rows, c.D, KS, 64) &&
+         make_tmap_bf16_2d(&m->v_ctx, c.ctxV, ctx_rows, c.D, KS, 64) &&
+         make_tmap_bf16_2d(&m->k_q, c.qK, q_rows, c.D, KS, 64) &&
+         make_tmap_bf16_2d(&m->v_q, c.qV, q_rows, c.D, KS, 64);
+}
+
+cudaError_t decode_prepare(int D) {
+  if (D == 128)
+    return cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                DSmem<128>::BYTES + 1024);
+  return cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              DSmem<64>::BYTES + 1024);
+}
+
+cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
+                               const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,
                                const DecodePlan& plan, const Scratch& s, cudaStream_t st) {
-  DecodeArgs a{};
+  DecodeArgs a;
+  a.tk_ctx = maps.k_ctx;
+  a.tv_ctx = maps.v_ctx;
+  a.tk_q = maps.k_q;
+  a.tv_q = maps.v_q;
   a.c = c;
   a.scale_log2 = scale * kLog2e;
   a.len0 = len0;
-  a.cph = plan.chunks_per_head;
-  a.chunk_rows = (int)plan.chunk_rows;
+  a.ncta = plan.ncta;
+  a.maxp = plan.maxp;
+  a.rpb = c.L + len0;
   a.q = q;
   a.k = k;
   a.v = v;
@@ -312,19 +498,11 @@ cudaError_t launch_decode_step(const CacheView& c, float scale, int len0, const 
   a.partA = s.partA;
   a.partS = s.partS;
   a.tickets = s.tickets;
-  const int grid = c.B * c.Hkv * plan.chunks_per_head;
-  cudaError_t e;
-  if (c.D == 128) {
-    const int smem = 16 * 128 * 2 + 2 * NSTAGE * KS * 128 * 2;
-    e = cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_kernel<128><<<grid, NTHREADS, smem, st>>>(a);
-  } else {
-    const int smem = 16 * 64 * 2 + 2 * NSTAGE * KS * 64 * 2;
-    e = cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_kernel<64><<<grid, NTHREADS, smem, st>>>(a);
-  }
+  a.err = s.err;
+  if (c.D == 128)
+    decode_kernel<128><<<plan.ncta, NTHREADS, DSmem<128>::BYTES + 1024, st>>>(a);
+  else
+    decode_kernel<64><<<plan.ncta, NTHREADS, DSmem<64>::BYTES + 1024, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -24,6 +24,7 @@ struct star_cache {
   void* block;              // the one cudaMalloc holding everything below
   int4* ctx_work;           // phase-1 work list, longest first
   int n_ctx_work;
+  star::DecodeMaps dmaps;   // TMA maps of the cache (built once)
 };
 
 namespace {
@@ -81,15 +82,9 @@ star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
 }
 
 star::DecodePlan plan_decode(const star_cache* c, long long len0) {
-  const star::CacheView& v = c->view;
-  const long long total = v.L + len0 + 1;
-  const long long bg = (long long)v.B * v.Hkv;
-  long long cph = std::max(1LL, (2LL * c->num_sms) / bg);
-  long long rows = round_up((total + cph - 1) / cph, 64);
-  cph = (total + rows - 1) / rows;
   star::DecodePlan pl;
-  pl.chunks_per_head = (int)cph;
-  pl.chunk_rows = rows;
+  pl.ncta = star::decode_num_ctas(c->view, len0, c->num_sms);
+  pl.maxp = star::decode_max_partials(c->view, c->num_sms);
   return pl;
 }
 
@@ -149,15 +144,8 @@ int star_cache_create(const star_params* p, star_cache** out) {
     partA = std::max(partA, rows * v.D);
     partS = std::max(partS, rows);
   }
-  for (long long len0 = 0; len0 < p->q_cap; len0 += std::max(1, p->q_cap / 64)) {
-    star::DecodePlan pl = plan_decode(c, len0);
-    const long long rows = (long long)v.B * v.Hkv * pl.chunks_per_head * v.G;
-    partA = std::max(partA, rows * v.D);
-    partS = std::max(partS, rows);
-  }
   {
-    star::DecodePlan pl = plan_decode(c, p->q_cap - 1);
-    const long long rows = (long long)v.B * v.Hkv * pl.chunks_per_head * v.G;
+    const long long rows = (long long)v.B * v.Hkv * star::decode_max_partials(v, c->num_sms) * v.G;
     partA = std::max(partA, rows * v.D);
     partS = std::max(partS, rows);
   }
@@ -194,7 +182,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
   c->scratch.partS_elems = partS;
   c->scratch.n_tickets = (int)n_tickets;
   c->ctx_work = reinterpret_cast<int4*>(base + o_w);
-  e = cudaMemset(c->scratch.tickets, 0, n_tickets * 4);
+  // Zero everything once: decode streams whole 128-row boxes and masks the
+  // rows past the end, which must hold finite values.
+  e = cudaMemset(c->block, 0, off);
+  if (e == cudaSuccess) e = cudaMemset(c->scratch.tickets, 0, n_tickets * 4);
   if (e == cudaSuccess) e = cudaMemset(c->scratch.err, 0, sizeof(int));
   if (e == cudaSuccess)
     e = cudaMemcpy(c->ctx_work, work.data(), work.size() * sizeof(int4), cudaMemcpyHostToDevice);
@@ -202,6 +193,17 @@ int star_cache_create(const star_params* p, star_cache** out) {
     cudaFree(c->block);
     delete c;
     return cuda_fail(e, "cache initialisation");
+  }
+  if (!star::decode_make_maps(v, &c->dmaps)) {
+    cudaFree(c->block);
+    delete c;
+    return fail(STAR_EINVAL, "TMA tensor maps of the cache rejected");
+  }
+  e = star::decode_prepare(v.D);
+  if (e != cudaSuccess) {
+    cudaFree(c->block);
+    delete c;
+    return cuda_fail(e, "decode kernel attributes");
   }
   c->q_len = 0;
   *out = c;
@@ -304,7 +306,7 @@ int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
     return fail(STAR_ENOSPC, "query region full: %lld rows, q_cap %d", c->q_len, c->view.q_cap);
   star::DecodePlan pl = plan_decode(c, c->q_len);
   cudaError_t e = star::launch_decode_step(
-      c->view, c->p.scale, (int)c->q_len, static_cast<const bf16*>(q),
+      c->view, c->dmaps, c->p.scale, (int)c->q_len, static_cast<const bf16*>(q),
       static_cast<const bf16*>(k), static_cast<const bf16*>(v), static_cast<bf16*>(o), lse, pl,
       c->scratch, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_decode_step launch");

@@ -1,6 +1,7 @@
 // Host/device view of a star_cache shared by the libstar kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -83,12 +84,20 @@ cudaError_t launch_query_prefill_mma(const CacheView& c, float scale, int lq, in
                                      cudaStream_t st);
 
 struct DecodePlan {
-  int chunks_per_head;   // split-KV chunks per (batch, kv head)
-  long long chunk_rows;  // keys per chunk (multiple of 64)
+  int ncta;   // CTAs (one balanced span of cached rows each)
+  int maxp;   // partial slots per (batch, kv head)
 };
+int decode_max_partials(const CacheView& c, int ncta);
+int decode_num_ctas(const CacheView& c, long long len0, int num_sms);
 
-cudaError_t launch_decode_step(const CacheView& c, float scale, int len0, const bf16* q,
-                               const bf16* k, const bf16* v, bf16* o, float* lse,
+// TMA maps of the cache, built once per cache.
+struct DecodeMaps {
+  CUtensorMap k_ctx, v_ctx, k_q, v_q;
+};
+bool decode_make_maps(const CacheView& c, DecodeMaps* m);
+cudaError_t decode_prepare(int D);   // one-time kernel attributes
+cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
+                               const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,
                                const DecodePlan& plan, const Scratch& s, cudaStream_t st);
 
 cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,

@@ -278,6 +278,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       }
       l_a += s[0][0] + s[0][1] + s[1][0] + s[1][1];
       l_b += s[0][2] + s[0][3] + s[1][2] + s[1][3];
+      if (16 * cw + 16 > n) {
+        // Rows past the stage's valid count carry p = 0, but 0 * NaN is NaN:
+        // clear this warp's V rows there (bytes past the end of a buffer need
+        // not be finite).  Each warp reads only its own 16 V rows.
+        for (int i = lane; i < 16 * (D / 8); i += 32) {
+          const int row = 16 * cw + i / (D / 8), ch = i % (D / 8);
+          if (row >= n) {
+            uint8_t* dst = smem + slot * S::STAGE + S::TILE + (ch >> 3) * S::HALF + row * 128 +
+                           (((ch & 7) ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        __syncwarp();
+      }
       uint32_t pa[4];
       pa[0] = pack_bf16(s[0][0], s[0][1]);
       pa[1] = pack_bf16(s[0][2], s[0][3]);
@@ -293,6 +307,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         mma_bf16_16816(o[2 * j], pa, b0, b1);
         mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
       }
+      // generic-proxy writes above must be ordered before the next TMA write
+      if (16 * cw + 16 > n) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_empty[slot]));
     }

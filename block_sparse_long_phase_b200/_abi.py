@@ -22,7 +22,7 @@ EXPORTS = (
     "star_cache_create", "star_cache_destroy", "star_cache_device_error", "star_cache_num_segments",
     "star_cache_segment", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_decode_step", "star_lse_merge",
-    "star_last_error", "star_version",
+    "star_decode_step_noalloc", "star_last_error", "star_version",
 )
 
 
@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH):
     lib.star_query_prefill.argtypes = [vp, i, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_lse_merge.argtypes = [i, ll, i, vp, vp, vp, vp, vp]
+    lib.star_decode_step_noalloc.argtypes = [ctypes.POINTER(StarParams), ll, vp, vp, vp, vp,
+                                             vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = i
     lib.star_last_error.restype = ctypes.c_char_p

@@ -182,6 +182,40 @@ def star_lse_merge(A: torch.Tensor, s: torch.Tensor, out_A=None, out_s=None):
     return out_A, out_s
 
 
+def star_decode_step_noalloc(params, q_len, ctx_k, ctx_v, q_k, q_v, q, k, v, o=None, lse=None):
+    """Decode step that allocates no device memory in libstar.
+
+    For callers that cannot call the CUDA allocator while serving (a runtime
+    that hands out all device memory from its own pool): the KV cache is the
+    caller's tensors -- ``ctx_k``/``ctx_v`` in the segmented layout of
+    ``star_cache_create`` (flat bf16, B*Hkv*L*D elements), ``q_k``/``q_v`` as
+    [B, Hkv, q_cap, D] -- and the split-KV scratch is a static device array of
+    the library.  ``params`` is a ``_abi.StarParams``; row ``q_len`` of the
+    query region receives ``k``/``v``.  Calls that overlap on the GPU race on
+    the shared scratch.
+    """
+    lib = _abi.load()
+    B, Hq, Hkv, D = params.B, params.Hq, params.Hkv, params.D
+    n_ctx = B * Hkv * params.L * D
+    _need(ctx_k, (n_ctx,), torch.bfloat16, "ctx_k")
+    _need(ctx_v, (n_ctx,), torch.bfloat16, "ctx_v")
+    _need(q_k, (B, Hkv, params.q_cap, D), torch.bfloat16, "q_k")
+    _need(q_v, (B, Hkv, params.q_cap, D), torch.bfloat16, "q_v")
+    _need(q, (B, Hq, 1, D), torch.bfloat16, "q")
+    _need(k, (B, Hkv, 1, D), torch.bfloat16, "k")
+    _need(v, (B, Hkv, 1, D), torch.bfloat16, "v")
+    if o is None:
+        o = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(o, (B, Hq, 1, D), torch.bfloat16, "o")
+    _need(lse, (B, Hq), torch.float32, "lse")
+    _abi.check(lib.star_decode_step_noalloc(ctypes.byref(params), q_len, _ptr(ctx_k), _ptr(ctx_v),
+                                            _ptr(q_k), _ptr(q_v), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(o), _ptr(lse), _stream(q.device)))
+    return o, lse
+
+
 def _tensor_from_ptr(ptr: int, n_elems: int, device) -> torch.Tensor:
     """A bf16 view of ``n_elems`` elements of device memory owned by libstar."""
 

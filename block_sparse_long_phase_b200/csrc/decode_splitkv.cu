@@ -27,6 +27,9 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
+#include "../../include/star_attention.h"
 #include "sm100_primitives.cuh"
 #include "star_common.cuh"
 #include "star_internal.h"
@@ -523,3 +526,116 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
 }
 
 }  // namespace star
+
+// ===========================================================================
+// Allocation-free decode step.
+//
+// Some callers cannot allocate device memory when they run a step: a runtime
+// that owns every byte of the GPU through its own pool, or a caller that must
+// not touch the CUDA allocator on its serving path.  For them the decode step
+// below takes the KV cache as caller-owned buffers and keeps its own split-KV
+// scratch (partials, merge tickets, error word) in one file-scope device
+// array, reserved when the library is loaded on a GPU and held until exit.
+// ===========================================================================
+namespace star {
+int check_params(const star_params* p);
+namespace {
+
+constexpr long long kNoAllocPartA = 1LL << 20;    // floats of partial outputs (4 MiB)
+constexpr long long kNoAllocPartS = 1LL << 14;    // floats of partial log-sum-exps (64 KiB)
+constexpr long long kNoAllocTickets = 1024;       // merge tickets (one per batch x kv head)
+constexpr long long kNoAllocFloats = kNoAllocPartA + kNoAllocPartS + kNoAllocTickets + 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_addr[kMaxDevices];
+int g_noalloc_sms[kMaxDevices];
+
+// Device address of the static scratch on `dev` (the current device), looked
+// up once per device: in host code the array's name is only a host-side
+// stand-in, never a device address.
+cudaError_t noalloc_setup(int dev, float** addr, int* sms) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = decode_prepare(64);
+    if (e == cudaSuccess) e = decode_prepare(128);
+    if (e != cudaSuccess) return e;
+    g_noalloc_sms[dev] = n;
+    g_noalloc_addr[dev] = static_cast<float*>(p);
+  }
+  *addr = g_noalloc_addr[dev];
+  *sms = g_noalloc_sms[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace star
+
+extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long q_len,
+                                                 const void* ctx_k, const void* ctx_v, void* q_k,
+                                                 void* q_v, const void* q, const void* k,
+                                                 const void* v, void* o, float* lse, void* stream) {
+  using namespace star;
+  int rc = check_params(p);
+  if (rc) return rc;
+  if (!ctx_k || !ctx_v || !q_k || !q_v || !q || !k || !v || !o || !lse)
+    return set_error(STAR_EINVAL, "NULL tensor pointer");
+  const void* ptrs[] = {ctx_k, ctx_v, q_k, q_v, q, k, v, o, lse};
+  for (const void* x : ptrs)
+    if (reinterpret_cast<uintptr_t>(x) & 15u) return set_error(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (q_len < 0) return set_error(STAR_EINVAL, "q_len must be >= 0");
+  if (q_len + 1 > p->q_cap) return set_error(STAR_ENOSPC, "query region full");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return set_error(STAR_ECUDA, "cudaGetDevice failed");
+  float* base = nullptr;
+  int sms = 0;
+  e = noalloc_setup(dev, &base, &sms);
+  if (e != cudaSuccess) return set_error(STAR_ECUDA, cudaGetErrorString(e));
+
+  CacheView c;
+  c.B = p->B; c.Hq = p->Hq; c.Hkv = p->Hkv; c.D = p->D; c.G = p->Hq / p->Hkv;
+  c.L = p->L; c.b = p->block; c.b_a = p->anchor;
+  c.n_seg = (int)((p->L + p->block - 1) / p->block);
+  c.q_cap = p->q_cap;
+  c.ctxK = static_cast<bf16*>(const_cast<void*>(ctx_k));
+  c.ctxV = static_cast<bf16*>(const_cast<void*>(ctx_v));
+  c.qK = static_cast<bf16*>(q_k);
+  c.qV = static_cast<bf16*>(q_v);
+
+  DecodePlan pl;
+  pl.ncta = decode_num_ctas(c, q_len, sms);
+  pl.maxp = decode_max_partials(c, sms);
+  const long long rows = (long long)c.B * c.Hkv * pl.maxp * c.G;
+  if (rows * c.D > kNoAllocPartA || rows > kNoAllocPartS || (long long)c.B * c.Hkv > kNoAllocTickets)
+    return set_error(STAR_EINVAL, "problem too large for the static decode scratch "
+                                  "(B*Hkv*G*D*(ceil(SMs/(B*Hkv))+2) must be <= 1048576 floats, "
+                                  "B*Hkv <= 1024)");
+  DecodeMaps maps;
+  if (!decode_make_maps(c, &maps)) return set_error(STAR_EINVAL, "TMA tensor maps rejected");
+  Scratch sc;
+  sc.partA = base;
+  sc.partS = base + kNoAllocPartA;
+  sc.tickets = reinterpret_cast<unsigned*>(base + kNoAllocPartA + kNoAllocPartS);
+  sc.err = reinterpret_cast<int*>(base + kNoAllocPartA + kNoAllocPartS + kNoAllocTickets);
+  sc.partA_elems = kNoAllocPartA;
+  sc.partS_elems = kNoAllocPartS;
+  sc.n_tickets = (int)kNoAllocTickets;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the tickets (and the error word next to them) must start at zero
+  e = cudaMemsetAsync(sc.tickets, 0, (kNoAllocTickets + 1) * sizeof(float), st);
+  if (e == cudaSuccess)
+    e = launch_decode_step(c, maps, p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->D), (int)q_len,
+                           static_cast<const bf16*>(q), static_cast<const bf16*>(k),
+                           static_cast<const bf16*>(v), static_cast<bf16*>(o), lse, pl, sc, st);
+  if (e != cudaSuccess) return set_error(STAR_ECUDA, cudaGetErrorString(e));
+  return STAR_OK;
+}

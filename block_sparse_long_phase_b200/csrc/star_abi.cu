@@ -106,6 +106,14 @@ int validate_params(const star_params* p) {
 
 }  // namespace
 
+namespace star {
+int set_error(int code, const char* msg) {
+  snprintf(g_err, sizeof(g_err), "%s", msg);
+  return code;
+}
+int check_params(const star_params* p) { return validate_params(p); }
+}  // namespace star
+
 extern "C" {
 
 const char* star_last_error(void) { return g_err; }

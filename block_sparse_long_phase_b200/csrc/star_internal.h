@@ -10,6 +10,9 @@ namespace star {
 
 typedef __nv_bfloat16 bf16;
 
+// Error reporting shared by the C entry points (star_last_error()).
+int set_error(int code, const char* msg);
+
 // Geometry of the per-block KV cache.  Context segment i holds rows
 // [i*b, i*b + len_i) of every (batch, kv head), laid out [B][Hkv][len_i][D];
 // segments are back to back, so segment i starts i*B*Hkv*b*D elements in.

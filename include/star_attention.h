@@ -137,6 +137,31 @@ STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const
 STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const float* s,
                    float* out_A, float* out_s, void* stream);
 
+/* Decode step that allocates nothing (the pages have no counterpart: this is
+ * an integration entry point).  For callers that cannot call cudaMalloc on
+ * their serving path -- a runtime that hands out all device memory from its
+ * own pool, or one that forbids the CUDA allocator while it serves -- the KV
+ * cache is the caller's memory and the split-KV scratch (partials, merge
+ * tickets, error word) lives in one static device array of the library,
+ * 4.3 MiB, present on every GPU that loads the library until the process
+ * exits.  Same arithmetic and kernel as star_decode_step.
+ *   p          layer parameters, as for star_cache_create (scale <= 0: 1/sqrt(D))
+ *   q_len      query-region rows in use before this step; this call writes
+ *              row q_len of q_k / q_v with k / v
+ *   ctx_k/v    context cache, the layout star_cache_create uses: segment i
+ *              as [B][Hkv][len_i][D] bf16, segments back to back
+ *   q_k/v      query region [B][Hkv][q_cap][D] bf16
+ *   q, k, v, o, lse   as for star_decode_step
+ * Limits: B*Hkv*G*D*(ceil(SMs/(B*Hkv)) + 2) <= 1048576 and B*Hkv <= 1024,
+ * else STAR_EINVAL.  The first call on a device looks up the array's device
+ * address (make it before any stream capture).  Every call shares the one
+ * array, so calls that overlap on the GPU (other streams, other threads) race;
+ * each call clears the merge tickets it needs. */
+STAR_API int star_decode_step_noalloc(const star_params* p, long long q_len,
+                                      const void* ctx_k, const void* ctx_v, void* q_k, void* q_v,
+                                      const void* q, const void* k, const void* v,
+                                      void* o, float* lse, void* stream);
+
 /* Description of the last error in this thread ("" if none). */
 STAR_API const char* star_last_error(void);
 

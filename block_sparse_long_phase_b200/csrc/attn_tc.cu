@@ -1,24 +1,29 @@
-// Phase-1 context encoding on the 5th-generation tensor core (tcgen05 + TMEM
-// + TMA), warp-specialised.
+// Tensor-core attention tile kernel for sm_100a (tcgen05 + TMEM + TMA),
+// warp-specialised.  Two operations share it:
 //
-// "Star Attention: Efficient LLM Inference over Long Sequences" (analysis
-// page), section 3.4, "Phase 1: Context Encoding with Anchor Blocks": block i
-// >= 1 is prefixed with the anchor and encoded with causal attention over
-// [anchor | block i] (Steps 2 and 4); block 0 is encoded on its own; only the
-// block's own K/V is kept in the cache (Step 5).  The augmented block is never
-// materialised: a CTA streams the anchor's K/V tiles [0, b_a) with no mask and
-// then its own block's tiles up to the diagonal with a causal mask.
-//
-// CTA work item: one 128-row query tile of one block for TWO q heads of the
-// same kv group (GQA), so each K/V tile fetched by TMA feeds two S = Q K^T
-// and two O += P V MMAs; both heads share the mask.
+// * Phase-1 context encoding -- "Star Attention: Efficient LLM Inference over
+//   Long Sequences" (analysis page), section 3.4, "Phase 1: Context Encoding
+//   with Anchor Blocks": block i >= 1 is prefixed with the anchor and encoded
+//   with causal attention over [anchor | block i] (Steps 2 and 4); block 0 is
+//   encoded on its own; only the block's own K/V is kept in the cache (Step
+//   5).  The augmented block is never materialised: a CTA streams the anchor's
+//   K/V tiles [0, b_a) with no mask and then its own block's tiles up to the
+//   diagonal with a causal mask.  CTA work item: one 128-row query tile of one
+//   block for TWO q heads of the same kv group (GQA), so each K/V tile fetched
+//   by TMA feeds two S = Q K^T and two O += P V MMAs; both heads share the mask.
+// * Phase-2 query prefill -- same page, "Phase 2: Query Encoding and Token
+//   Generation with Distributed Softmax", Step 3: the query rows attend to one
+//   key chunk (a slice of a context segment, fully visible, or the query
+//   region, causal) and leave that chunk's local (A_h, s_h) in fp32 for the
+//   merge (Step 5).  The G q heads x lq query rows of one kv head are
+//   contiguous, so a CTA takes two 128-row tiles of those packed rows.
 //
 // Roles (12 warps):
 //   warp 0      TMA producer: Q0/Q1 once, then K_j, V_j into a 4-slot ring
 //   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 2-3   copy the tile's own K/V rows into the block's cache segment
-//   warps 4-7   softmax for head 0: S0 row per thread, P0 back into TMEM
-//   warps 8-11  softmax for head 1
+//   warps 2-3   phase 1: copy the tile's own K/V rows into the block's segment
+//   warps 4-7   softmax for tile 0: one S row per thread, P back into TMEM
+//   warps 8-11  softmax for tile 1
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
 // P_i (bf16) overwrites the first 64 columns of S_i.  tcgen05.mma ops issued by
 // the one MMA thread run in order, so S_i(j+1) is written only after
@@ -52,17 +57,24 @@ constexpr int NTHREADS = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct CtxTcArgs {
-  CUtensorMap tq;   // Q  as [B*Hq*L][D]
-  CUtensorMap tk;   // K  as [B*Hkv*L][D]
-  CUtensorMap tv;   // V  as [B*Hkv*L][D]
+  CUtensorMap tq;   // phase 1: Q as [B*Hq*L][D]; prefill: query rows as [B*Hq*lq][D]
+  CUtensorMap tk;   // phase 1: K as [B*Hkv*L][D]; prefill: context cache as [B*Hkv*L][D]
+  CUtensorMap tv;
+  CUtensorMap tkq;  // prefill: query region as [B*Hkv*q_cap][D]
+  CUtensorMap tvq;
   CacheView c;
   float scale_log2;
   const bf16* K;
   const bf16* V;
   bf16* O;
   float* LSE;
-  const int4* work;   // (b*Hkv + g, head pair, block, q tile)
+  const int4* work;   // phase 1: (b*Hkv + g, head pair, block, q tile)
   int* err;
+  // prefill
+  int lq, len0, row_pairs;
+  float* partA;
+  float* partS;
+  PrefillPlan plan;
 };
 
 SM100_DEV float ex2(float x) {
@@ -81,8 +93,8 @@ struct Smem {
   static constexpr int BYTES = RING + NBUF * TILE;  // + barriers in static smem
 };
 
-template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_constant__ CtxTcArgs a) {
+template <int D, bool PF>
+__global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_constant__ CtxTcArgs a) {
   using S = Smem<D>;
   constexpr int NH = D / 64;                          // 128-byte halves per row
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -101,19 +113,43 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- work item ------------------------------------------------------------
-  const int4 w = a.work[blockIdx.x];
-  const int bg = w.x;
-  const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
-  const int h0 = g * c.G + 2 * w.y;
-  const int nq = (h0 + 1 < (g + 1) * c.G) ? 2 : 1;
-  const int blk = w.z;
-  const long long bstart = (long long)blk * c.b;
-  const long long bend = bstart + c.b < c.L ? bstart + c.b : c.L;
-  const long long t0 = bstart + (long long)w.w * BM;
-  const int n_rows = (int)((bend - t0) < BM ? (bend - t0) : BM);
-  const int n_anchor = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
-  const int n_kv = n_anchor + w.w + 1;
-  const long long kv_row0 = (long long)bg * c.L;     // row of (b, g, token 0) in K/V maps
+  int bg, bb, g, h0 = 0, nq, blk = 0, n_rows0, n_rows1, n_anchor = 0, n_kv, chunk = 0;
+  long long bstart = 0, t0 = 0, kv_row0, qrow0;
+  if (!PF) {
+    const int4 w = a.work[blockIdx.x];
+    bg = w.x;
+    bb = bg / c.Hkv;
+    g = bg - bb * c.Hkv;
+    h0 = g * c.G + 2 * w.y;
+    nq = (h0 + 1 < (g + 1) * c.G) ? 2 : 1;
+    blk = w.z;
+    bstart = (long long)blk * c.b;
+    const long long bend = bstart + c.b < c.L ? bstart + c.b : c.L;
+    t0 = bstart + (long long)w.w * BM;
+    n_rows0 = n_rows1 = (int)((bend - t0) < BM ? (bend - t0) : BM);
+    n_anchor = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
+    n_kv = n_anchor + w.w + 1;
+    kv_row0 = (long long)bg * c.L;                          // (b, g, token 0) in the K/V maps
+    qrow0 = ((long long)bb * c.Hq + h0) * c.L + t0;         // Q0's first row; Q1 is one head later
+  } else {
+    const int bgs = c.B * c.Hkv;
+    const int pair = blockIdx.x % a.row_pairs;
+    bg = (blockIdx.x / a.row_pairs) % bgs;
+    chunk = blockIdx.x / (a.row_pairs * bgs);
+    bb = bg / c.Hkv;
+    g = bg - bb * c.Hkv;
+    const int rows_total = c.G * a.lq;
+    const int r0 = pair * 2 * BM;
+    nq = r0 + BM < rows_total ? 2 : 1;
+    n_rows0 = rows_total - r0 < BM ? rows_total - r0 : BM;
+    n_rows1 = rows_total - r0 - BM < BM ? rows_total - r0 - BM : BM;
+    t0 = r0;                                                // packed row of Q0's first row
+    n_kv = (a.plan.chunk[chunk].len + BN - 1) / BN;
+    const PrefillChunk ch = a.plan.chunk[chunk];
+    kv_row0 = ch.seg >= 0 ? (long long)ch.seg * c.B * c.Hkv * c.b + (long long)bg * seg_len(c, ch.seg) + ch.start
+                          : (long long)bg * c.q_cap;
+    qrow0 = ((long long)bb * c.Hq + (long long)g * c.G) * a.lq + r0;   // Q1 is 128 rows later
+  }
 
   if (tid == 0) {
     mbar_init(smem_u32(&bar_q_full), 1);
@@ -145,13 +181,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
   if (warp == 0) {
     // ------------------------------ TMA producer -----------------------------
     if (elect_one()) {
+      const bool qregion = PF && a.plan.chunk[chunk].seg < 0;
+      const CUtensorMap* mk = qregion ? &a.tkq : &a.tk;
+      const CUtensorMap* mv = qregion ? &a.tvq : &a.tv;
       prefetch_tmap(&a.tq);
-      prefetch_tmap(&a.tk);
-      prefetch_tmap(&a.tv);
+      prefetch_tmap(mk);
+      prefetch_tmap(mv);
       const uint32_t qb = smem_u32(&bar_q_full);
       mbar_arrive_expect_tx(qb, nq * S::TILE);
       for (int q = 0; q < nq; ++q) {
-        const int qrow = (int)(((long long)bb * c.Hq + h0 + q) * c.L + t0);
+        const int qrow = (int)(qrow0 + (PF ? (long long)q * BM : (long long)q * c.L));
         for (int hf = 0; hf < NH; ++hf)
           tma_load_2d(smem_u32(smem + (q ? S::Q1 : S::Q0) + hf * S::HALF), &a.tq, hf * 64, qrow, qb);
       }
@@ -162,11 +201,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
         const int j = i >> 1, slot = i % NBUF, use = i / NBUF;
         if (use > 0 && !mbar_wait(smem_u32(&bar_kv_empty[slot]), (use - 1) & 1)) { fail(); break; }
         if (*(volatile int*)&abort_s) break;
-        const long long tok = j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
+        const long long tok = PF ? (long long)j * BN
+                                 : (j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN);
         const int row = (int)(kv_row0 + tok);
         const uint32_t fb = smem_u32(&bar_kv_full[slot]);
         mbar_arrive_expect_tx(fb, S::TILE);
-        const CUtensorMap* m = (i & 1) ? &a.tv : &a.tk;
+        const CUtensorMap* m = (i & 1) ? mv : mk;
         for (int hf = 0; hf < NH; ++hf)
           tma_load_2d(smem_u32(smem + S::RING + slot * S::TILE + hf * S::HALF), m, hf * 64, row, fb);
         last_use[slot] = use;
@@ -233,7 +273,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
     }
   } else if (warp < 4) {
     // ---------------- cache segment write (anchor KV discarded) ---------------
-    if (h0 == g * c.G) {
+    if (!PF && h0 == g * c.G) {
+      const int n_rows = n_rows0;
       const long long len = seg_len(c, blk);
       const long long sbase = (long long)blk * c.B * c.Hkv * (long long)c.b * D +
                               ((long long)bg * len + (t0 - bstart)) * D;
@@ -255,7 +296,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
       const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
       const uint32_t tS = tmem + lane_off + q * 128;
       const uint32_t tO = tmem + lane_off + 256 + q * D;
-      const long long pos = t0 + r;                   // token index of the row
+      const long long pos = t0 + (PF ? q * BM : 0) + r;  // token (phase 1) / packed row (prefill)
+      const int n_rows = q ? (n_rows1 > 0 ? n_rows1 : 0) : n_rows0;
+      // prefill: keys visible to this row in the chunk are [0, lim_pf)
+      long long lim_pf = 0;
+      if (PF) {
+        const PrefillChunk ch = a.plan.chunk[chunk];
+        lim_pf = ch.seg >= 0 ? ch.len : a.len0 + (pos % a.lq) + 1;
+      }
       float m_used = -INFINITY, l = 0.f;
       const float sl2 = a.scale_log2;
       for (int j = 0; j < n_kv; ++j) {
@@ -265,10 +313,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
         tmem_wait_ld();
-        // mask: anchor tail (keys >= b_a) and the causal diagonal
-        const bool anchor = j < n_anchor;
-        const long long k0 = anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
-        const long long lim = anchor ? (long long)c.b_a : pos + 1;   // keys < lim are visible
+        // mask: phase 1 -- anchor tail (keys >= b_a) and the causal diagonal;
+        // prefill -- chunk tail, or the causal query region
+        const bool anchor = !PF && j < n_anchor;
+        const long long k0 = (PF || anchor) ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
+        const long long lim = PF ? lim_pf : (anchor ? (long long)c.b_a : pos + 1);   // keys < lim visible
         if (k0 + BN > lim) {
           const int nvis = (int)(lim - k0 < 0 ? 0 : lim - k0);   // visible columns: [0, nvis)
 #pragma unroll
@@ -317,30 +366,51 @@ __global__ void __launch_bounds__(NTHREADS, 1) ctx_tc_kernel(const __grid_consta
         tc_fence_before();
         mbar_arrive(smem_u32(&bar_p_full[q]));
       }
-      // ---- epilogue: O / l in bf16, LSE = (m + log2 l) ln 2 -------------------
+      // ---- epilogue -------------------------------------------------------------
+      // phase 1: O / l in bf16 and LSE = (m + log2 l) ln 2;  prefill: the chunk's
+      // fp32 partial (A_h, s_h) of every packed row.
       const bool ok = mbar_wait(smem_u32(&bar_o_full), 0);
       if (!ok) fail();
       tc_fence_after();
-      const int h = h0 + q;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* orow = a.O + (((long long)bb * c.Hq + h) * c.L + pos) * D;
+      const float lse = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      if (!PF) {
+        const int h = h0 + q;
+        bf16* orow = a.O + (((long long)bb * c.Hq + h) * c.L + pos) * D;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_wait_ld();
-        if (r < n_rows) {
-          uint32_t pk[16];
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+          if (r < n_rows) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            reinterpret_cast<uint4*>(orow + cc * 32)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v)
+              reinterpret_cast<uint4*>(orow + cc * 32)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
+        if (r < n_rows) a.LSE[((long long)bb * c.Hq + h) * c.L + pos] = lse;
+      } else {
+        const long long prow = ((long long)bg * a.plan.n_chunks + chunk) * (c.G * a.lq) + pos;
+        float* arow = a.partA + prow * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+          if (r < n_rows) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              reinterpret_cast<float4*>(arow + cc * 32)[v] =
+                  make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                              __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
+          }
+        }
+        if (r < n_rows) a.partS[prow] = lse;
       }
-      if (r < n_rows)
-        a.LSE[((long long)bb * c.Hq + h) * c.L + pos] = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
     }
   }
 
@@ -379,6 +449,22 @@ void ctx_tc_fill_work(const CacheView& c, int4* out) {
   for (size_t i = 0; i < items.size(); ++i) out[i] = items[i].v;
 }
 
+cudaError_t attn_tc_prepare(int D) {
+  cudaError_t e;
+  if (D == 128) {
+    const int smem = Smem<128>::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  } else {
+    const int smem = Smem<64>::BYTES + 1024;
+    e = cudaFuncSetAttribute(attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  }
+  return e;
+}
+
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
                                  int* err, cudaStream_t st) {
@@ -398,18 +484,113 @@ cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q,
   a.LSE = LSE;
   a.work = work;
   a.err = err;
-  cudaError_t e;
-  if (c.D == 128) {
-    const int smem = Smem<128>::BYTES + 1024;
-    e = cudaFuncSetAttribute(ctx_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    ctx_tc_kernel<128><<<n_work, NTHREADS, smem, st>>>(a);
-  } else {
-    const int smem = Smem<64>::BYTES + 1024;
-    e = cudaFuncSetAttribute(ctx_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    ctx_tc_kernel<64><<<n_work, NTHREADS, smem, st>>>(a);
+  if (c.D == 128)
+    attn_tc_kernel<128, false><<<n_work, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
+  else
+    attn_tc_kernel<64, false><<<n_work, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+  return cudaGetLastError();
+}
+
+// ---- query prefill ------------------------------------------------------------
+namespace {
+
+// Append this call's query K/V rows to the query region (rows len0..len0+lq-1).
+__global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, int len0,
+                                                           const uint4* __restrict__ K,
+                                                           const uint4* __restrict__ V) {
+  const int cpr = c.D / 8;                                    // 16-byte chunks per row
+  const long long n = (long long)c.B * c.Hkv * lq * cpr;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / cpr;
+    const int ch = (int)(i - row * cpr);
+    const int bg = (int)(row / lq), t = (int)(row - (long long)bg * lq);
+    const long long dst = (((long long)bg * c.q_cap) + len0 + t) * cpr + ch;
+    reinterpret_cast<uint4*>(c.qK)[dst] = K[i];
+    reinterpret_cast<uint4*>(c.qV)[dst] = V[i];
   }
+}
+
+// Merge the chunks' partials of every packed query row and scatter to O / LSE.
+template <int D>
+__global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq, int n_chunks,
+                                                            const float* __restrict__ partA,
+                                                            const float* __restrict__ partS,
+                                                            bf16* __restrict__ O,
+                                                            float* __restrict__ LSE) {
+  const int rows_total = c.G * lq;
+  const long long gw = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= (long long)c.B * c.Hkv * rows_total) return;
+  const long long bg = gw / rows_total;
+  const int m = (int)(gw - bg * rows_total);
+  const int bb = (int)(bg / c.Hkv), g = (int)(bg - (long long)bb * c.Hkv);
+  float mx = -INFINITY;
+  for (int p = 0; p < n_chunks; ++p) mx = fmaxf(mx, partS[(bg * n_chunks + p) * rows_total + m]);
+  const float base = mx == -INFINITY ? 0.f : mx;
+  float tot = 0.f;
+  for (int p = 0; p < n_chunks; ++p) tot += __expf(partS[(bg * n_chunks + p) * rows_total + m] - base);
+  const float lse = mx == -INFINITY ? -INFINITY : base + __logf(tot);
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  for (int p = 0; p < n_chunks; ++p) {
+    const long long r = (bg * n_chunks + p) * rows_total + m;
+    const float s = partS[r];
+    if (s == -INFINITY) continue;
+    const float w = __expf(s - lse);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] += w * partA[r * D + lane + 32 * i];
+  }
+  const int h = g * c.G + m / lq;
+  const int rr = m % lq;
+  bf16* orow = O + (((long long)bb * c.Hq + h) * lq + rr) * D;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
+  if (lane == 0) LSE[((long long)bb * c.Hq + h) * lq + rr] = lse;
+}
+
+}  // namespace
+
+int prefill_row_pairs(const CacheView& c, int lq) { return (c.G * lq + 2 * BM - 1) / (2 * BM); }
+
+cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, float scale, int lq,
+                                    int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
+                                    float* LSE, const PrefillPlan& plan, const Scratch& s,
+                                    cudaStream_t st) {
+  CtxTcArgs a;
+  memset(&a, 0, sizeof(a));
+  const unsigned long long qrows = (unsigned long long)c.B * c.Hq * lq;
+  if (!make_tmap_bf16_2d(&a.tq, Q, qrows, c.D, BM, 64)) return cudaErrorInvalidValue;
+  a.tk = maps.k_ctx;
+  a.tv = maps.v_ctx;
+  a.tkq = maps.k_q;
+  a.tvq = maps.v_q;
+  a.c = c;
+  a.scale_log2 = scale * kLog2e;
+  a.err = s.err;
+  a.lq = lq;
+  a.len0 = len0;
+  a.row_pairs = prefill_row_pairs(c, lq);
+  a.partA = s.partA;
+  a.partS = s.partS;
+  a.plan = plan;
+  const long long n16 = (long long)c.B * c.Hkv * lq * (c.D / 8);
+  const int agrid = (int)((n16 + 255) / 256 < 1024 ? (n16 + 255) / 256 : 1024);
+  query_append_kernel<<<agrid, 256, 0, st>>>(c, lq, len0, reinterpret_cast<const uint4*>(Kq),
+                                             reinterpret_cast<const uint4*>(Vq));
+  const int grid = c.B * c.Hkv * a.row_pairs * plan.n_chunks;
+  if (c.D == 128)
+    attn_tc_kernel<128, true><<<grid, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
+  else
+    attn_tc_kernel<64, true><<<grid, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+  const long long rows = (long long)c.B * c.Hkv * c.G * lq;
+  const int mgrid = (int)((rows + 3) / 4);
+  if (c.D == 128)
+    prefill_merge_kernel<128><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE);
+  else
+    prefill_merge_kernel<64><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE);
   return cudaGetLastError();
 }
 

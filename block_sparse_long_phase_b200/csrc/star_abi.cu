@@ -50,14 +50,16 @@ long long round_up(long long x, long long m) { return (x + m - 1) / m * m; }
 constexpr int kTileRows = 64;
 
 // ---- phase-2 plans --------------------------------------------------------
+// Prefill chunks: each context segment is cut into equal pieces (multiples of
+// 128 keys) so that (batch x kv head) x (256-row pairs) x chunks is about one
+// CTA per SM; the query region is one more chunk.
 star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
   const star::CacheView& v = c->view;
   star::PrefillPlan pl{};
-  pl.row_tiles = (int)((v.G * (long long)lq + kTileRows - 1) / kTileRows);
-  const long long bg = (long long)v.B * v.Hkv;
-  const long long target = 2LL * c->num_sms * 2;  // ~2 waves of 2 CTAs per SM
-  long long want = std::max(1LL, (target + bg * pl.row_tiles - 1) / (bg * pl.row_tiles));
-  long long chunk_len = std::max<long long>(256, round_up((v.L + want - 1) / want, kTileRows));
+  const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
+  const long long want = std::max(1LL, (long long)c->num_sms / bgp);
+  const long long per_seg = std::max(1LL, (want - 1) / v.n_seg);
+  long long chunk_len = round_up((v.b + per_seg - 1) / per_seg, 128);
   for (;;) {
     int n = 0;
     for (int s = 0; s < v.n_seg; ++s) n += (int)((star::seg_len(v, s) + chunk_len - 1) / chunk_len);
@@ -208,6 +210,7 @@ int star_cache_create(const star_params* p, star_cache** out) {
     return fail(STAR_EINVAL, "TMA tensor maps of the cache rejected");
   }
   e = star::decode_prepare(v.D);
+  if (e == cudaSuccess) e = star::attn_tc_prepare(v.D);
   if (e != cudaSuccess) {
     cudaFree(c->block);
     delete c;
@@ -295,8 +298,8 @@ int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K, cons
   if (c->q_len + lq > c->view.q_cap)
     return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, c->view.q_cap);
   star::PrefillPlan pl = plan_prefill(c, lq, c->q_len);
-  cudaError_t e = star::launch_query_prefill_mma(
-      c->view, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
+  cudaError_t e = star::launch_query_prefill_tc(
+      c->view, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
       static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
       c->scratch, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_query_prefill launch");

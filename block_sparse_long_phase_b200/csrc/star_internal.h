@@ -77,14 +77,8 @@ constexpr int kMaxPrefillChunks = 96;
 
 struct PrefillPlan {
   int n_chunks;
-  int row_tiles;   // ceil(G*lq / 64)
   PrefillChunk chunk[kMaxPrefillChunks];
 };
-
-cudaError_t launch_query_prefill_mma(const CacheView& c, float scale, int lq, int len0,
-                                     const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
-                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
-                                     cudaStream_t st);
 
 struct DecodePlan {
   int ncta;   // CTAs (one balanced span of cached rows each)
@@ -102,6 +96,13 @@ cudaError_t decode_prepare(int D);   // one-time kernel attributes
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
                                const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,
                                const DecodePlan& plan, const Scratch& s, cudaStream_t st);
+
+cudaError_t attn_tc_prepare(int D);   // one-time kernel attributes
+int prefill_row_pairs(const CacheView& c, int lq);   // 256-row pairs of packed query rows
+cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, float scale, int lq,
+                                    int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
+                                    float* LSE, const PrefillPlan& plan, const Scratch& s,
+                                    cudaStream_t st);
 
 cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,
                              float* outA, float* outS, cudaStream_t st);

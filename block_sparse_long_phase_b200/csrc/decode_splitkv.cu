@@ -81,6 +81,14 @@ __device__ __forceinline__ int cta_of(long long x, long long R, int n) {
   return (int)(((x + 1) * n - 1) / R);
 }
 
+// Release the partials this CTA wrote (ordered before by the consumer barrier,
+// cumulatively) and acquire every other CTA's, in one atomic.
+SM100_DEV unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 SM100_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
 
 template <int D>
@@ -205,11 +213,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       qa[kd][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col + 8) : 0u;
       qa[kd][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col + 8) : 0u;
     }
+  };
+  auto reset_state = [&]() {
 #pragma unroll
     for (int n = 0; n < NT_O; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+#pragma unroll
+    for (int kd = 0; kd < D / 16; ++kd) qa[kd][0] = qa[kd][1] = qa[kd][2] = qa[kd][3] = 0u;
     m_a = m_b = -INFINITY;
     l_a = l_b = 0.f;
   };
+  reset_state();
 
   long long x = x0;
   for (int st = 0; x < x1; ++st) {
@@ -389,6 +402,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       }
       named_sync(1, 32 * NCW);
     }
+    reset_state();                             // the piece's state now lives in the partial
+    cur_bg = -1;
     if (owns_new && ctid < D / 8) {
       // append the new token to the query region (row len0); no reader in this launch
       const long long qo = q_row_offset(c, bb, g, a.len0);
@@ -399,66 +414,88 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     // barrier orders every consumer's partial stores before thread 0's
     // gpu-scope release fence (cumulative), which precedes the ticket.
     named_sync(1, 32 * NCW);
-    if (ctid == 0) {
-      __threadfence();
-      s_last = (atomicAdd(&a.tickets[bg], 1u) == (unsigned)(count - 1));
-    }
+    if (ctid == 0) s_last = (atom_add_acq_rel_gpu(&a.tickets[bg], 1u) == (unsigned)(count - 1));
     named_sync(1, 32 * NCW);
     if (s_last) {
-      __threadfence();
-      // merge weights: load every s_h once (in parallel), then per-row max/sum
-      float* sv = comb;                           // [G][count] log-sum-exps, then weights
-      for (int i = ctid; i < G * count; i += 32 * NCW) {
-        const int r = i / count, p = i - (i / count) * count;
-        sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + p) * G + r);
-      }
-      named_sync(1, 32 * NCW);
-      if (ctid < G) {
-        const int r = ctid;
-        float M = -INFINITY;
-        for (int p = 0; p < count; ++p) M = fmaxf(M, sv[r * count + p]);
-        const float base = M == -INFINITY ? 0.f : M;
-        float tot = 0.f;
-        for (int p = 0; p < count; ++p) tot += __expf(sv[r * count + p] - base);
-        const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
-        s_lse[r] = l;
-        for (int p = 0; p < count; ++p) {
-          const float sp = sv[r * count + p];
-          sv[r * count + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
-        }
-      }
-      named_sync(1, 32 * NCW);
-      // weighted sum over the partials: float4 columns, eight loads in flight
-      for (int idx = ctid; idx < G * (D / 4); idx += 32 * NCW) {
-        const int r = idx / (D / 4), d4 = idx - (idx / (D / 4)) * (D / 4);
+      // Merge this head's `count` partials.  A thread owns one float4 column of
+      // one row and every npg-th partial; its partial loads are issued before
+      // the s_h loads and the weights, so the merge costs about one L2 round
+      // trip when count <= KMAX * npg.
+      constexpr int NT = 32 * NCW;
+      constexpr int KMAX = 11;
+      const int nout = G * (D / 4);
+      float* sv = comb;                              // [G][count] s_h, then weights
+      float4* red = reinterpret_cast<float4*>(comb + kMaxG * 160);   // [npg][nb]
+      bool have_w = false;
+      for (int ob = 0; ob < nout; ob += NT) {
+        const int nb = nout - ob < NT ? nout - ob : NT;
+        const int npg = NT / nb;
+        const bool active = ctid < nb * npg;
+        const int oi = ob + ctid % nb, pg = ctid / nb;
+        const int r = oi / (D / 4), d4 = oi - (oi / (D / 4)) * (D / 4);
         const float4* pa = reinterpret_cast<const float4*>(a.partA + ((long long)bg * a.maxp * G + r) * D) + d4;
         const long long pstride = (long long)G * D / 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p0 = 0; p0 < count; p0 += 8) {
-          float4 v16[8];
+        for (int p0 = 0; p0 < count; p0 += KMAX * npg) {
+          float4 v[KMAX];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            v16[u] = p0 + u < count ? __ldcg(pa + (p0 + u) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int k = 0; k < KMAX; ++k) {
+            const int p = p0 + pg + k * npg;
+            v[k] = (active && p < count) ? __ldcg(pa + p * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          if (!have_w) {
+            for (int i = ctid; i < G * count; i += NT) {
+              const int rr = i / count, p = i - (i / count) * count;
+              sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + p) * G + rr);
+            }
+            named_sync(1, NT);
+            if (ctid < G) {                           // per-row log-sum-exp, then weights
+              float M = -INFINITY;
+              for (int p = 0; p < count; ++p) M = fmaxf(M, sv[ctid * count + p]);
+              const float base = M == -INFINITY ? 0.f : M;
+              float tot = 0.f;
+              for (int p = 0; p < count; ++p) tot += __expf(sv[ctid * count + p] - base);
+              const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
+              s_lse[ctid] = l;
+              for (int p = 0; p < count; ++p) {
+                const float sp = sv[ctid * count + p];
+                sv[ctid * count + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
+              }
+            }
+            named_sync(1, NT);
+            have_w = true;
+          }
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float wgt = p0 + u < count ? sv[r * count + p0 + u] : 0.f;
-            acc.x += wgt * v16[u].x;
-            acc.y += wgt * v16[u].y;
-            acc.z += wgt * v16[u].z;
-            acc.w += wgt * v16[u].w;
+          for (int k = 0; k < KMAX; ++k) {
+            const int p = p0 + pg + k * npg;
+            const float wgt = (active && p < count) ? sv[r * count + p] : 0.f;
+            acc.x += wgt * v[k].x;
+            acc.y += wgt * v[k].y;
+            acc.z += wgt * v[k].z;
+            acc.w += wgt * v[k].w;
           }
         }
-        const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
-        uint2 pk;
-        pk.x = pack_bf16(acc.x, acc.y);
-        pk.y = pack_bf16(acc.z, acc.w);
-        *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
-        if (d4 == 0) a.lse[orow] = s_lse[r];
+        if (active) red[pg * nb + (oi - ob)] = acc;   // sum the npg partial sums of each column
+        named_sync(1, NT);
+        if (active && pg == 0) {
+          for (int q2 = 1; q2 < npg; ++q2) {
+            const float4 u = red[q2 * nb + (oi - ob)];
+            acc.x += u.x;
+            acc.y += u.y;
+            acc.z += u.z;
+            acc.w += u.w;
+          }
+          const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
+          uint2 pk;
+          pk.x = pack_bf16(acc.x, acc.y);
+          pk.y = pack_bf16(acc.z, acc.w);
+          *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+          if (d4 == 0) a.lse[orow] = s_lse[r];
+        }
+        named_sync(1, NT);
       }
       if (ctid == 0) a.tickets[bg] = 0u;   // ready for the next step
-      named_sync(1, 32 * NCW);
     }
-    cur_bg = -1;                            // the next piece reloads q and resets the state
   }
 }
 

@@ -193,6 +193,16 @@ def _blas_threads():
     return os.cpu_count()
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise maximum over ranks of per-rank timings: the slowest rank
+    decides a replica run's time (NCCL on GPUs; any backend works)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 def measure_long_decode(dev, flush, warmup, steps, world):
     """Decode steps at 128K context (the 8B-128K workload), L2 flushed before each."""
     import torch
@@ -217,13 +227,11 @@ def measure_long_decode(dev, flush, warmup, steps, world):
         ms.append((a, b))
     torch.cuda.synchronize(dev)
     times = [a.elapsed_time(b) for a, b in ms[warmup:]]
-    t = torch.tensor([sum(times) / len(times)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    (t_ms,) = max_over_ranks([sum(times) / len(times)], dev, world)
     cache.close()
     del x
     torch.cuda.empty_cache()
-    return w, t.item() * 1e3
+    return w, t_ms * 1e3
 
 
 def dist_setup(args):
@@ -361,10 +369,7 @@ def main():
     step_ms = [e + p + sum(d) for e, p, d in zip(enc_ms, pre_ms, dec_ms)]
     enc_total = sum(enc_ms)
     dec_total = sum(sum(d) for d in dec_ms)
-    tot = torch.tensor([enc_total, dec_total, sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
-    enc_total, dec_total, step_total = tot.tolist()
+    enc_total, dec_total, step_total = max_over_ranks([enc_total, dec_total, sum(step_ms)], dev, world)
 
     # ---- end to end through the public API (pinned host buffers) ----------------
     e2e = None
@@ -387,12 +392,10 @@ def main():
             torch.cuda.synchronize(dev)
             if it >= args.warmup:
                 e2e_ms.append(a.elapsed_time(b))
-        t = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        (e2e_total,) = max_over_ranks([sum(e2e_ms)], dev, world)
         h2d = sum(v.numel() * v.element_size() for v in hx.values())
         d2h = hO.numel() * 2 + hL.numel() * 4
-        e2e = {"value": world * w.B * w.L * args.steps / (t.item() / 1e3), "unit": "ctx tok/s",
+        e2e = {"value": world * w.B * w.L * args.steps / (e2e_total / 1e3), "unit": "ctx tok/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "what": "H2D of Q,K,V from pinned host + star_ctx_encode + D2H of O,LSE"}
 
@@ -435,7 +438,6 @@ def main():
         line["e2e"] = e2e
     if long_dec:
         wl2, t_us = long_dec
-        lb = sum(decode_bytes(wl2, wl2.lq + t) for t in range(1)) / 1.0
         gbs = decode_bytes(wl2, 0) / (t_us * 1e-6) / 1e9
         line["decode_long"] = {
             "workload": wl2.name, "value": world * wl2.B / (t_us * 1e-6), "unit": "decode tok/s",
@@ -443,7 +445,6 @@ def main():
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "bytes_per_step": decode_bytes(wl2, 0)}}
-        del lb
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d, sample, threads = cpu_oracle_sample(w, x)
         line["cpu_baseline"] = {"value": v, "unit": "ctx tok/s", "cores": threads, "kind": "oracle",

@@ -82,6 +82,26 @@ SM100_DEV float ex2(float x) {
   asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
+SM100_DEV void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n"
+      " mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+SM100_DEV void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n"
+      " mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+SM100_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 template <int D>
 struct Smem {
@@ -229,28 +249,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       //   PV0(j), S0(j+1), PV1(j), S1(j+1)
       // so the tensor core computes head 0's next scores while head 1's
       // softmax still runs, and the other way round.
-      auto issue_s = [&](int q, uint32_t kbase) {
-        const uint32_t qbase = smem_u32(smem + (q ? S::Q1 : S::Q0));
+      // Descriptors are built once; an MMA then costs one add (the start
+      // address is the low field, and every offset stays inside it).
+      // Q1 follows Q0 and the ring slots follow each other at TILE bytes.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + S::Q0), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem + S::RING), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + S::RING), S::HALF, 1024);
+      constexpr uint64_t kTileStep = S::TILE >> 4;
+      auto issue_s = [&](int q, int slot) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * S::HALF + (kk & 3) * 32;
-          mma_ss(sS[q], smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                 id_qk, kk > 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * S::HALF + (kk & 3) * 32) >> 4);
+          mma_ss(sS[q], dq0 + q * kTileStep + off, dk0 + slot * kTileStep + off, id_qk, kk > 0);
         }
         mma_commit(smem_u32(&bar_s_full[q]));
       };
-      auto issue_pv = [&](int q, uint32_t vbase, int j) {
+      auto issue_pv = [&](int q, int slot, int j) {
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(sO[q], sS[q] + kk * 8, smem_desc_sw128(vbase + kk * 2048, S::HALF, 1024), id_pv,
+          mma_ts(sO[q], sS[q] + kk * 8, dv0 + slot * kTileStep + (uint64_t)((kk * 2048) >> 4), id_pv,
                  (j > 0 || kk > 0) ? 1u : 0u);
       };
-      auto kv_slot = [&](int i) { return smem_u32(smem + S::RING + (i % NBUF) * S::TILE); };
       bool ok = mbar_wait(smem_u32(&bar_q_full), 0) && mbar_wait(smem_u32(&bar_kv_full[0]), 0);
       if (!ok) fail();
       if (ok) {
         tc_fence_after();
-        for (int q = 0; q < nq; ++q) issue_s(q, kv_slot(0));
+        for (int q = 0; q < nq; ++q) issue_s(q, 0);
         mma_commit(smem_u32(&bar_kv_empty[0]));
       }
       for (int j = 0; ok && j < n_kv; ++j) {
@@ -259,10 +283,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         if (!mbar_wait(smem_u32(&bar_kv_full[iv % NBUF]), (iv / NBUF) & 1)) { fail(); break; }
         if (more && !mbar_wait(smem_u32(&bar_kv_full[ik % NBUF]), (ik / NBUF) & 1)) { fail(); break; }
         for (int q = 0; q < nq; ++q) {
-          if (!mbar_wait(smem_u32(&bar_p_full[q]), j & 1)) { fail(); ok = false; break; }
+          if (!mbar_spin(smem_u32(&bar_p_full[q]), j & 1)) { fail(); ok = false; break; }
           tc_fence_after();
-          issue_pv(q, kv_slot(iv), j);
-          if (more) issue_s(q, kv_slot(ik));
+          issue_pv(q, iv % NBUF, j);
+          if (more) issue_s(q, ik % NBUF);
         }
         if (!ok) break;
         mma_commit(smem_u32(&bar_kv_empty[iv % NBUF]));
@@ -324,9 +348,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
           for (int i = 0; i < BN; ++i)
             if (i >= nvis) s[i] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // row maximum: eight independent chains of 3-input max, then a tree
+        float mk[8];
 #pragma unroll
-        for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+        for (int k = 0; k < 8; ++k) mk[k] = fmaxf(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]));
+#pragma unroll
+        for (int i = 16; i < BN; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mk[k] = fmax3(mk[k], __uint_as_float(s[i + 2 * k]), __uint_as_float(s[i + 2 * k + 1]));
+        const float mx = fmaxf(fmax3(mk[0], mk[1], mk[2]), fmax3(fmax3(mk[3], mk[4], mk[5]), mk[6], mk[7]));
         const float m_tile = mx * sl2;
         const bool need = m_tile > m_used + kRescaleThreshold;
         float alpha = 1.f;
@@ -348,19 +379,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         }
         l *= alpha;
         const float base = m_used == -INFINITY ? 0.f : m_used;
-        float rs = 0.f;
+        // P = 2^(s*scale - base): packed-pair FMA, ex2, four packed row-sum chains
+        float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int cc = 0; cc < BN / 32; ++cc) {
           uint32_t p[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float e0 = ex2(fmaf(__uint_as_float(s[cc * 32 + 2 * i]), sl2, -base));
-            const float e1 = ex2(fmaf(__uint_as_float(s[cc * 32 + 2 * i + 1]), sl2, -base));
-            rs += e0 + e1;
+            float x0, x1;
+            ffma2(x0, x1, __uint_as_float(s[cc * 32 + 2 * i]), __uint_as_float(s[cc * 32 + 2 * i + 1]),
+                  sl2, sl2, -base, -base);
+            const float e0 = ex2(x0), e1 = ex2(x1);
+            fadd2(ra[i & 3], rb[i & 3], ra[i & 3], rb[i & 3], e0, e1);
             p[i] = pack_bf16(e0, e1);
           }
           tmem_st16(tS + cc * 16, p);
         }
+        const float rs = (ra[0] + rb[0]) + (ra[1] + rb[1]) + ((ra[2] + rb[2]) + (ra[3] + rb[3]));
         l += rs;
         tmem_wait_st();
         tc_fence_before();

@@ -42,6 +42,25 @@ SM100_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+SM100_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded spin without suspending the thread, for the latency-critical
+// waits of a single issuing thread.
+constexpr uint32_t kSpinLimit = 1u << 28;
+SM100_DEV bool mbar_spin(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_test_wait(bar, parity)) return true;
+  return false;
+}
+
 // Bounded wait: gives up after `limit` polls (each poll may suspend briefly)
 // and returns false, so a broken pipeline ends instead of hanging the GPU.
 constexpr uint32_t kWaitLimit = 1u << 22;

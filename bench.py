@@ -65,6 +65,12 @@ def decode_bytes(w, t):
     return w.B * w.Hkv * (w.L + w.lq + t + 1) * w.D * 2 * 2
 
 
+def decode_bytes_fp8(w, t):
+    """Same, FP8 context cache: one byte per context element plus a float32
+    scale per context row, for K and for V; the query region stays bf16."""
+    return w.B * w.Hkv * (w.L * (w.D + 4) * 2 + (w.lq + t + 1) * w.D * 2 * 2)
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
 
@@ -203,13 +209,14 @@ def max_over_ranks(values, device, world):
     return t.tolist()
 
 
-def measure_long_decode(dev, flush, warmup, steps, world):
-    """Decode steps at 128K context (the 8B-128K workload), L2 flushed before each."""
+def measure_long_decode(dev, flush, warmup, steps, world, kv_fp8=False):
+    """Decode steps at 128K context (the 8B-128K workload), L2 flushed before each;
+    with ``kv_fp8`` the context is streamed from the cache's FP8 copy."""
     import torch
     from block_sparse_long_phase_b200 import StarCache, workloads as wl
     w = wl.get("8b-128k-needle")
     x = wl.make_inputs(w, dev)
-    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale, kv_fp8=kv_fp8)
     cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
     cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
     del x["Qc"]
@@ -232,6 +239,50 @@ def measure_long_decode(dev, flush, warmup, steps, world):
     del x
     torch.cuda.empty_cache()
     return w, t_ms * 1e3
+
+
+PHASE1_VARIANTS = {
+    # anchor shorter than the block (the pages' anchor-size sweep), ragged last block, batch 4
+    "8b-32k-anchor2k": dict(b_a=2048),
+    "8b-30000-ragged": dict(L=30000, b=8000, b_a=8000),
+    "8b-32k-batch4": dict(B=4),
+}
+
+
+def measure_phase1_variants(dev, flush, warmup, steps, world):
+    """Phase-1 TFLOP/s on the variant shapes (same kernel, same timing rules)."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    for name, over in PHASE1_VARIANTS.items():
+        w = wl.get(WORKLOAD).with_(name=name, **over)
+        g = torch.Generator(device=dev).manual_seed(w.seed + 7)
+        Q = torch.randn((w.B, w.Hq, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+        K = torch.randn((w.B, w.Hkv, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn((w.B, w.Hkv, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+        cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, 1, w.scale)
+        O = torch.empty_like(Q)
+        LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+        evs = []
+        for it in range(warmup + steps):
+            flush.fill_(6.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            cache.star_ctx_encode(Q, K, V, O, LSE)
+            b.record(stream)
+            if it >= warmup:
+                evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+        (ms,) = max_over_ranks([ms], dev, world)
+        flops, _ = phase1_flops(w)
+        out[name] = {"B": w.B, "L": w.L, "block": w.b, "anchor": w.b_a, "ms": ms,
+                     "ctx_tok_s": world * w.B * w.L / (ms / 1e3), "tflops": flops / (ms / 1e3) / 1e12}
+        cache.close()
+        del Q, K, V, O, LSE
+        torch.cuda.empty_cache()
+    return out
 
 
 def dist_setup(args):
@@ -297,6 +348,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-long-decode", action="store_true",
                     help="skip the decode measurement at 128K context")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the phase-1 variants (anchor shorter than the block, ragged context, batch 4)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -399,9 +452,13 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "what": "H2D of Q,K,V from pinned host + star_ctx_encode + D2H of O,LSE"}
 
+    variants = None
+    if not args.no_variants:
+        variants = measure_phase1_variants(dev, flush, args.warmup, min(args.steps, 10), world)
     long_dec = None
     if not args.no_long_decode:
         long_dec = measure_long_decode(dev, flush, args.warmup, args.steps, world)
+        long_dec_fp8 = measure_long_decode(dev, flush, args.warmup, args.steps, world, kv_fp8=True)
 
     pk = peaks()
     flops, _ = phase1_flops(w)
@@ -436,6 +493,13 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
+    if variants:
+        for v in variants.values():
+            # burst peak for a launch of a few ms; a launch of 10+ ms runs under
+            # the power cap, where the sustained peak is the fair denominator
+            v["frac"] = v["tflops"] / pk["bf16_tflops"]
+            v["frac_sustained"] = v["tflops"] / pk["bf16_tflops_sustained"]
+        line["phase1_variants"] = variants
     if long_dec:
         wl2, t_us = long_dec
         gbs = decode_bytes(wl2, 0) / (t_us * 1e-6) / 1e9
@@ -445,6 +509,14 @@ def main():
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,
                          "bytes_per_step": decode_bytes(wl2, 0)}}
+        wl3, t3 = long_dec_fp8
+        gbs = decode_bytes_fp8(wl3, 0) / (t3 * 1e-6) / 1e9
+        line["decode_long_fp8"] = {
+            "workload": wl3.name, "kv_cache": "context K/V in E4M3 with a float32 scale per row",
+            "value": world * wl3.B / (t3 * 1e-6), "unit": "decode tok/s", "us_per_step": t3,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "bytes_per_step": decode_bytes_fp8(wl3, 0)}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d, sample, threads = cpu_oracle_sample(w, x)
         line["cpu_baseline"] = {"value": v, "unit": "ctx tok/s", "cores": threads, "kind": "oracle",

@@ -20,7 +20,7 @@ STAR_ENOMEM = -5
 # Every symbol the header declares.
 EXPORTS = (
     "star_cache_create", "star_cache_destroy", "star_cache_device_error", "star_cache_num_segments",
-    "star_cache_segment", "star_cache_reset_query", "star_ctx_encode",
+    "star_cache_segment", "star_cache_segment_fp8", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
 )
@@ -30,7 +30,7 @@ class StarParams(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("D", ctypes.c_int),
         ("L", ctypes.c_longlong), ("block", ctypes.c_int), ("anchor", ctypes.c_int),
-        ("q_cap", ctypes.c_int), ("scale", ctypes.c_float),
+        ("q_cap", ctypes.c_int), ("scale", ctypes.c_float), ("kv_fp8", ctypes.c_int),
     ]
 
 
@@ -59,6 +59,8 @@ def load(path: str = LIB_PATH):
     lib.star_cache_device_error.argtypes = [vp, ctypes.POINTER(i)]
     lib.star_cache_segment.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                        ctypes.POINTER(ll), ctypes.POINTER(ll), ctypes.POINTER(ll)]
+    lib.star_cache_segment_fp8.argtypes = [vp, i, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                           ctypes.POINTER(fp), ctypes.POINTER(fp)]
     lib.star_cache_reset_query.argtypes = [vp]
     lib.star_ctx_encode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_query_prefill.argtypes = [vp, i, vp, vp, vp, vp, vp, vp]

@@ -52,17 +52,19 @@ class StarCache:
     Wraps ``star_cache_create``; the cache lives on the current CUDA device.
     """
 
-    def __init__(self, B, Hq, Hkv, D, L, block, anchor, q_cap, scale=0.0):
+    def __init__(self, B, Hq, Hkv, D, L, block, anchor, q_cap, scale=0.0, kv_fp8=False):
         if not torch.cuda.is_available():
             raise RuntimeError("libstar needs a CUDA device; there is no CPU fallback")
         self.lib = _abi.load()
-        self.params = _abi.StarParams(B, Hq, Hkv, D, L, block, anchor, q_cap, float(scale))
+        self.params = _abi.StarParams(B, Hq, Hkv, D, L, block, anchor, q_cap, float(scale),
+                                      int(bool(kv_fp8)))
         self.device = torch.device("cuda", torch.cuda.current_device())
         h = ctypes.c_void_p()
         _abi.check(self.lib.star_cache_create(ctypes.byref(self.params), ctypes.byref(h)))
         self.handle = h
         self.B, self.Hq, self.Hkv, self.D, self.L = B, Hq, Hkv, D, L
         self.block, self.anchor, self.q_cap = block, anchor, q_cap
+        self.kv_fp8 = bool(kv_fp8)
 
     # -- lifetime ------------------------------------------------------------
     def close(self):
@@ -103,6 +105,21 @@ class StarCache:
             t = _tensor_from_ptr(p, n, self.device).view(self.B, self.Hkv, seg.cap, self.D)
             out.append(t)
         return out[0], out[1], seg
+
+    def segment_fp8_tensors(self, i: int):
+        """FP8 copy of context segment ``i`` (``kv_fp8`` caches): E4M3 codes of K
+        and V as uint8 [B, Hkv, len, D] and their float32 row scales [B, Hkv, len]."""
+        k8, v8 = ctypes.c_void_p(), ctypes.c_void_p()
+        ks, vs = ctypes.POINTER(ctypes.c_float)(), ctypes.POINTER(ctypes.c_float)()
+        _abi.check(self.lib.star_cache_segment_fp8(self.handle, i, ctypes.byref(k8), ctypes.byref(v8),
+                                                   ctypes.byref(ks), ctypes.byref(vs)))
+        n = self.segment(i).len
+        shape = (self.B, self.Hkv, n)
+        codes = [_view_from_ptr(p, self.B * self.Hkv * n * self.D, "|u1", self.device)
+                 .view(*shape, self.D) for p in (k8.value, v8.value)]
+        scales = [_view_from_ptr(ctypes.cast(p, ctypes.c_void_p).value, self.B * self.Hkv * n, "<f4",
+                                 self.device).view(*shape) for p in (ks, vs)]
+        return codes[0], codes[1], scales[0], scales[1]
 
     def device_error(self) -> int:
         """Reads and clears the device error word (non-zero: a bounded wait gave up)."""
@@ -216,15 +233,19 @@ def star_decode_step_noalloc(params, q_len, ctx_k, ctx_v, q_k, q_v, q, k, v, o=N
     return o, lse
 
 
-def _tensor_from_ptr(ptr: int, n_elems: int, device) -> torch.Tensor:
-    """A bf16 view of ``n_elems`` elements of device memory owned by libstar."""
+def _view_from_ptr(ptr: int, n_elems: int, typestr: str, device) -> torch.Tensor:
+    """A flat view of ``n_elems`` elements of device memory owned by libstar."""
 
     class _CudaArray:
         def __init__(self):
             self.__cuda_array_interface__ = {
-                "shape": (n_elems,), "typestr": "<u2", "data": (ptr, False), "version": 3,
+                "shape": (n_elems,), "typestr": typestr, "data": (ptr, False), "version": 3,
                 "strides": None,
             }
 
-    t = torch.as_tensor(_CudaArray(), device=device)
-    return t.view(torch.bfloat16)
+    return torch.as_tensor(_CudaArray(), device=device)
+
+
+def _tensor_from_ptr(ptr: int, n_elems: int, device) -> torch.Tensor:
+    """A bf16 view of ``n_elems`` elements of device memory owned by libstar."""
+    return _view_from_ptr(ptr, n_elems, "<u2", device).view(torch.bfloat16)

@@ -24,6 +24,7 @@
 // of a (batch, kv head) to finish -- an atomic ticket, no CTA ever waits for
 // another -- merges that head's partials and writes o and lse.
 #include <cuda_bf16.h>
+#include <stdio.h>
 #include <math.h>
 #include <string.h>
 
@@ -50,12 +51,15 @@ struct StageMeta {
   int n;         // valid keys in the stage
   int last;      // 1: the stage ends a (batch, kv head) piece of this span
   int bg;        // batch * Hkv + kv head
-  int pad;
+  int row0;      // FP8 context stage: its first row in the context cache; else -1
 };
 
 struct DecodeArgs {
   CUtensorMap tk_ctx, tv_ctx;   // context cache as [B*Hkv*L][D]
   CUtensorMap tk_q, tv_q;       // query region as [B*Hkv*q_cap][D]
+  CUtensorMap tk8, tv8;         // FP8 context cache as [B*Hkv*L][D] bytes
+  CUtensorMap tkq64, tvq64;     // query region in 64-row boxes (FP8 mode)
+  CUtensorMap tks, tvs;         // FP8 row scales: one row of B*Hkv*L float32
   CacheView c;
   float scale_log2;
   int len0;                     // query-region rows before this step
@@ -91,28 +95,68 @@ SM100_DEV unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
 
 SM100_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory"); }
 
-template <int D>
+template <int D, bool FP8 = false>
 struct DSmem {
-  static constexpr int HALF = KS * 128;               // one 64-column half of a stage tile
-  static constexpr int TILE = KS * D * 2;              // K (or V) of one stage
+  static constexpr int HALF = KS * 128;               // one 64-column half of a bf16 stage tile
+  static constexpr int HALF64 = 64 * 128;             // ... of a 64-row bf16 tile (FP8 mode)
+  // K (or V) of one stage: 128 rows of bf16, or in FP8 mode 128 rows of E4M3
+  // codes (128- or 64-byte swizzled) / 64 query-region rows of bf16
+  static constexpr int TILE = FP8 ? KS * D : KS * D * 2;
   static constexpr int STAGE = 2 * TILE;
+  static constexpr int NST = FP8 ? 6 : NSTAGE;
+  // FP8 row scales of a stage: a box of 132 floats starting at the 4-aligned
+  // row at or below the stage's first row
+  static constexpr int SCL_BOX = KS + 4;
+  static constexpr int SCL_BYTES = SCL_BOX * 4;
+  static constexpr int SCL_SLOT = 640;
+  static constexpr int SCL = FP8 ? NST * 2 * SCL_SLOT : 0;
   // 4 rows of O per warp per round; also holds the merge weights (<= 16 x 160)
   static constexpr int COMB = NCW * 4 * 128 * 4;
-  static constexpr int BYTES = NSTAGE * STAGE + COMB;
+  static constexpr int BYTES = NST * STAGE + SCL + COMB;
 };
 
+SM100_DEV uint32_t pack_f16(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+SM100_DEV uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t d;
+  const uint16_t a = (uint16_t)two_codes;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(d) : "h"(a));
+  return d;
+}
+SM100_DEV uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+// Offset of 16-byte chunk `chunk` of row `row` in a stage tile of E4M3 codes
+// (rows of D bytes) as TMA writes it: 128-byte swizzle for D = 128, 64-byte
+// swizzle for D = 64 (chunk index XOR address bits 7..9, resp. 7..8).
 template <int D>
+SM100_DEV uint32_t sw8(int row, int chunk) {
+  return (uint32_t)(row * D + ((chunk ^ (D == 128 ? (row & 7) : ((row >> 1) & 3))) << 4));
+}
+SM100_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D, bool FP8>
 __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
-  using S = DSmem<D>;
+  using S = DSmem<D, FP8>;
   constexpr int NH = D / 64;
   constexpr int NT_O = D / 8;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  float* comb = reinterpret_cast<float*>(smem + NSTAGE * S::STAGE);   // [NCW][4][D]
-  __shared__ __align__(8) uint64_t bar_full[NSTAGE];
-  __shared__ __align__(8) uint64_t bar_empty[NSTAGE];
-  __shared__ StageMeta meta[NSTAGE];
+  uint8_t* scl = smem + S::NST * S::STAGE;                     // [NST][K, V] row scales (FP8)
+  float* comb = reinterpret_cast<float*>(scl + S::SCL);         // [NCW][4][D]
+  __shared__ __align__(8) uint64_t bar_full[S::NST];
+  __shared__ __align__(8) uint64_t bar_empty[S::NST];
+  __shared__ StageMeta meta[S::NST];
   __shared__ float wm[NCW][16], wl[NCW][16];
   __shared__ float s_new[kMaxG];
   __shared__ float s_lse[kMaxG];
@@ -126,7 +170,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   const long long x1 = span_start(blockIdx.x + 1, R, a.ncta);
 
   if (tid == 0) {
-    for (int i = 0; i < NSTAGE; ++i) {
+    for (int i = 0; i < S::NST; ++i) {
       mbar_init(smem_u32(&bar_full[i]), 1);
       mbar_init(smem_u32(&bar_empty[i]), NCW);
     }
@@ -147,8 +191,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       prefetch_tmap(&a.tv_ctx);
       prefetch_tmap(&a.tk_q);
       prefetch_tmap(&a.tv_q);
-      int last_use[NSTAGE];
-      for (int k = 0; k < NSTAGE; ++k) last_use[k] = -1;
+      if (FP8) {
+        prefetch_tmap(&a.tk8);
+        prefetch_tmap(&a.tv8);
+        prefetch_tmap(&a.tkq64);
+        prefetch_tmap(&a.tvq64);
+        prefetch_tmap(&a.tks);
+        prefetch_tmap(&a.tvs);
+      }
+      int last_use[S::NST];
+      for (int k = 0; k < S::NST; ++k) last_use[k] = -1;
       long long x = x0;
       for (int st = 0; x < x1; ++st) {
         const int bg = (int)(x / a.rpb);
@@ -168,27 +220,41 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           row = (int)((long long)bg * c.q_cap + (off - c.L));
           ctx = false;
         }
-        long long n = KS;
+        long long n = (FP8 && !ctx) ? 64 : KS;
         if (region_end - off < n) n = region_end - off;
         if (piece_end - x < n) n = piece_end - x;
-        const int slot = st % NSTAGE, use = st / NSTAGE;
+        const int slot = st % S::NST, use = st / S::NST;
         if (use > 0 && !mbar_wait(smem_u32(&bar_empty[slot]), (use - 1) & 1)) { fail(); break; }
         if (aborted()) break;
         meta[slot].n = (int)n;
         meta[slot].last = (x + n == piece_end) ? 1 : 0;
         meta[slot].bg = bg;
+        meta[slot].row0 = (FP8 && ctx) ? row : -1;
         const uint32_t fb = smem_u32(&bar_full[slot]);
-        mbar_arrive_expect_tx(fb, S::STAGE);
+        mbar_arrive_expect_tx(fb, (FP8 && ctx) ? S::STAGE + 2 * S::SCL_BYTES : S::STAGE);
         const uint32_t dst = smem_u32(smem + slot * S::STAGE);
-        for (int hf = 0; hf < NH; ++hf) {
-          tma_load_2d(dst + hf * S::HALF, ctx ? &a.tk_ctx : &a.tk_q, hf * 64, row, fb);
-          tma_load_2d(dst + S::TILE + hf * S::HALF, ctx ? &a.tv_ctx : &a.tv_q, hf * 64, row, fb);
+        if (FP8 && ctx) {
+          tma_load_2d(dst, &a.tk8, 0, row, fb);
+          tma_load_2d(dst + S::TILE, &a.tv8, 0, row, fb);
+          const uint32_t sd = smem_u32(scl + slot * 2 * S::SCL_SLOT);
+          tma_load_2d(sd, &a.tks, row & ~3, 0, fb);
+          tma_load_2d(sd + S::SCL_SLOT, &a.tvs, row & ~3, 0, fb);
+        } else if (FP8) {
+          for (int hf = 0; hf < NH; ++hf) {
+            tma_load_2d(dst + hf * S::HALF64, &a.tkq64, hf * 64, row, fb);
+            tma_load_2d(dst + S::TILE + hf * S::HALF64, &a.tvq64, hf * 64, row, fb);
+          }
+        } else {
+          for (int hf = 0; hf < NH; ++hf) {
+            tma_load_2d(dst + hf * S::HALF, ctx ? &a.tk_ctx : &a.tk_q, hf * 64, row, fb);
+            tma_load_2d(dst + S::TILE + hf * S::HALF, ctx ? &a.tv_ctx : &a.tv_q, hf * 64, row, fb);
+          }
         }
         last_use[slot] = use;
         x += n;
       }
       if (aborted())
-        for (int k = 0; k < NSTAGE; ++k)
+        for (int k = 0; k < S::NST; ++k)
           if (last_use[k] >= 0) mbar_wait(smem_u32(&bar_full[k]), last_use[k] & 1);
     }
     return;   // the producer takes part in no named barrier
@@ -207,11 +273,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     const bf16* qb = a.q + ((long long)bb * c.Hq + (long long)g * G) * D;
 #pragma unroll
     for (int kd = 0; kd < D / 16; ++kd) {
-      const int col = 16 * kd + 2 * (lane & 3);
+      // FP8 mode permutes the contraction index inside each 16-column step:
+      // k-slots 2c, 2c+1 take columns 4c, 4c+1 and k-slots 2c+8, 2c+9 take
+      // 4c+2, 4c+3, the order in which one 32-bit word of a key row holds them
+      const int col = FP8 ? 16 * kd + 4 * (lane & 3) : 16 * kd + 2 * (lane & 3);
+      const int hi = FP8 ? 2 : 8;
       qa[kd][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col) : 0u;
       qa[kd][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col) : 0u;
-      qa[kd][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col + 8) : 0u;
-      qa[kd][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col + 8) : 0u;
+      qa[kd][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col + hi) : 0u;
+      qa[kd][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col + hi) : 0u;
+      if (FP8) {                                   // the FP8 path multiplies in f16
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qa[kd][e] = bf16x2_to_f16x2(qa[kd][e]);
+      }
     }
   };
   auto reset_state = [&]() {
@@ -224,9 +298,190 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   };
   reset_state();
 
+  // Scale and mask the scores of this warp's 16 keys (sk: per-key factor on
+  // the log2 scale), update the running max / sum, turn scores into p.
+  auto softmax_update = [&](float (&s)[2][4], const float (&sk)[4], int kw, int n) {
+#pragma unroll
+    for (int nn = 0; nn < 2; ++nn)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = kw + 8 * nn + 2 * (lane & 3) + (e & 1);
+        s[nn][e] = j < n ? s[nn][e] * sk[nn * 2 + (e & 1)] : -INFINITY;
+      }
+    float mx_a = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+    float mx_b = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    // The exponent base only moves up when a row's maximum grows by more
+    // than 2^8, so the accumulator is rarely rescaled.
+    const bool up_a = mx_a > m_a + 8.f, up_b = mx_b > m_b + 8.f;
+    if (__any_sync(0xffffffffu, up_a || up_b)) {
+      const float al_a = up_a ? exp2f(m_a - mx_a) : 1.f;
+      const float al_b = up_b ? exp2f(m_b - mx_b) : 1.f;
+      if (up_a) m_a = mx_a;
+      if (up_b) m_b = mx_b;
+      l_a *= al_a;
+      l_b *= al_b;
+#pragma unroll
+      for (int nn = 0; nn < NT_O; ++nn) {
+        o[nn][0] *= al_a;
+        o[nn][1] *= al_a;
+        o[nn][2] *= al_b;
+        o[nn][3] *= al_b;
+      }
+    }
+    const float base_a = m_a == -INFINITY ? 0.f : m_a;
+    const float base_b = m_b == -INFINITY ? 0.f : m_b;
+#pragma unroll
+    for (int nn = 0; nn < 2; ++nn) {
+      s[nn][0] = exp2f(s[nn][0] - base_a);
+      s[nn][1] = exp2f(s[nn][1] - base_a);
+      s[nn][2] = exp2f(s[nn][2] - base_b);
+      s[nn][3] = exp2f(s[nn][3] - base_b);
+    }
+    l_a += s[0][0] + s[0][1] + s[1][0] + s[1][1];
+    l_b += s[0][2] + s[0][3] + s[1][2] + s[1][3];
+  };
+
+  // One stage of bf16 keys: 16 keys per warp, K and V fragments straight from
+  // the 128-byte-swizzled TMA tiles.
+  auto bf16_stage = [&](uint32_t kb, uint32_t vb, int kw, int n, int slot) {
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kd = 0; kd < D / 16; ++kd) {
+      uint32_t b0, b1, b2, b3;
+      const int ch = 2 * kd + ((lane >> 3) & 1);
+      const int row = kw + (lane & 7) + ((lane >> 4) << 3);
+      ldmatrix_x4(kb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b0, b1, b2, b3);
+      mma_bf16_16816(s[0], qa[kd], b0, b1);
+      mma_bf16_16816(s[1], qa[kd], b2, b3);
+    }
+    const float sk[4] = {a.scale_log2, a.scale_log2, a.scale_log2, a.scale_log2};
+    softmax_update(s, sk, kw, n);
+    if (kw + 16 > n) {
+      // Rows past the stage's valid count carry p = 0, but 0 * NaN is NaN:
+      // clear this warp's V rows there (bytes past the end of a buffer need
+      // not be finite).  Each warp reads only its own 16 V rows.
+      for (int i = lane; i < 16 * (D / 8); i += 32) {
+        const int row = kw + i / (D / 8), ch = i % (D / 8);
+        if (row >= n) {
+          uint8_t* dst = smem + slot * S::STAGE + S::TILE + (ch >> 3) * S::HALF + row * 128 +
+                         (((ch & 7) ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      __syncwarp();
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16(s[0][0], s[0][1]);
+    pa[1] = pack_bf16(s[0][2], s[0][3]);
+    pa[2] = pack_bf16(s[1][0], s[1][1]);
+    pa[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+    for (int j = 0; j < D / 16; ++j) {
+      const int ch = 2 * j + (lane >> 4);
+      uint32_t b0, b1, b2, b3;
+      const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+      ldmatrix_x4_trans(vb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b0, b1, b2, b3);
+      mma_bf16_16816(o[2 * j], pa, b0, b1);
+      mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
+    }
+    // generic-proxy writes above must be ordered before the next TMA write
+    if (kw + 16 > n) fence_proxy_async_smem();
+  };
+
+  // One stage in FP8 mode.  Context stages hold E4M3 codes: ldmatrix on the
+  // swizzled byte tile gives each thread one 32-bit word (4 codes) per 8x16-byte
+  // matrix, converted in registers to f16 MMA operands -- for K the word is a
+  // B fragment under the permuted contraction order of qa; for V (.trans) it
+  // holds two keys x two columns, regrouped by a byte permute.  The output
+  // columns of V are permuted too: accumulator block nb, column n holds
+  // d = 16 (nb / 2) + 2 n + nb % 2.  Query-region stages hold bf16 rows, read
+  // word-wise in the same orders.  Per-row scales: K's on the score, V's on p.
+  auto fp8_stage = [&](const StageMeta& m, uint32_t kb, uint32_t vb, const uint8_t* sclp, int kw, int n) {
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const bool ctx8 = m.row0 >= 0;
+    const int t = lane >> 2, cq = lane & 3;
+    const uint8_t* kp = smem + (kb - smem_u32(smem));
+    const uint8_t* vp = kp + S::TILE;
+    if (ctx8) {
+#pragma unroll
+      for (int jp = 0; jp < D / 32; ++jp) {
+        const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4(kb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
+        mma_f16_16816(s[0], qa[2 * jp], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
+        mma_f16_16816(s[1], qa[2 * jp], e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
+        mma_f16_16816(s[0], qa[2 * jp + 1], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r2 >> 16));
+        mma_f16_16816(s[1], qa[2 * jp + 1], e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r3 >> 16));
+      }
+    } else {
+#pragma unroll
+      for (int kd = 0; kd < D / 16; ++kd)
+#pragma unroll
+        for (int nn = 0; nn < 2; ++nn) {
+          const int row = kw + 8 * nn + t;                       // < 64: kw < n <= 64
+          const int ch = 2 * (kd & 3) + (cq >> 1);
+          const uint2 w = *reinterpret_cast<const uint2*>(kp + (kd >> 2) * S::HALF64 + row * 128 +
+                                                          ((ch ^ (row & 7)) << 4) + 8 * (cq & 1));
+          mma_f16_16816(s[nn], qa[kd], bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y));
+        }
+    }
+    const float* sks = reinterpret_cast<const float*>(sclp) + (ctx8 ? (m.row0 & 3) : 0);
+    const float* svs = reinterpret_cast<const float*>(sclp + S::SCL_SLOT) + (ctx8 ? (m.row0 & 3) : 0);
+    float sk[4], sv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int key = kw + (u >> 1) * 8 + 2 * cq + (u & 1);
+      sk[u] = ctx8 ? a.scale_log2 * sks[key] : a.scale_log2;
+      sv[u] = ctx8 ? svs[key] : 1.f;
+    }
+    softmax_update(s, sk, kw, n);
+    uint32_t pa[4];
+    pa[0] = pack_f16(s[0][0] * sv[0], s[0][1] * sv[1]);
+    pa[1] = pack_f16(s[0][2] * sv[0], s[0][3] * sv[1]);
+    pa[2] = pack_f16(s[1][0] * sv[2], s[1][1] * sv[3]);
+    pa[3] = pack_f16(s[1][2] * sv[2], s[1][3] * sv[3]);
+    if (ctx8) {
+#pragma unroll
+      for (int jp = 0; jp < D / 32; ++jp) {
+        const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        uint32_t r0, r1, r2, r3;
+        ldmatrix_x4_trans(vb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
+        // r0: keys 2c, 2c+1 x columns 2t, 2t+1 of chunk 2jp; r1: keys 2c+8, 2c+9;
+        // r2, r3: the same of chunk 2jp+1.  Regroup to (key pair) per column.
+        const uint32_t p0 = __byte_perm(r0, 0u, 0x3120), p1 = __byte_perm(r1, 0u, 0x3120);
+        const uint32_t p2 = __byte_perm(r2, 0u, 0x3120), p3 = __byte_perm(r3, 0u, 0x3120);
+        mma_f16_16816(o[4 * jp], pa, e4m3x2_to_f16x2(p0), e4m3x2_to_f16x2(p1));
+        mma_f16_16816(o[4 * jp + 1], pa, e4m3x2_to_f16x2(p0 >> 16), e4m3x2_to_f16x2(p1 >> 16));
+        mma_f16_16816(o[4 * jp + 2], pa, e4m3x2_to_f16x2(p2), e4m3x2_to_f16x2(p3));
+        mma_f16_16816(o[4 * jp + 3], pa, e4m3x2_to_f16x2(p2 >> 16), e4m3x2_to_f16x2(p3 >> 16));
+      }
+    } else {
+#pragma unroll
+      for (int ch = 0; ch < D / 16; ++ch) {
+        const int cc = 2 * (ch & 3) + (t >> 2), by = 4 * (t & 3);
+        uint32_t w[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int kk = kw + 2 * cq + (q4 & 1) + 8 * (q4 >> 1);   // < 64
+          w[q4] = kk < n ? *reinterpret_cast<const uint32_t*>(vp + (ch >> 2) * S::HALF64 + kk * 128 +
+                                                              ((cc ^ (kk & 7)) << 4) + by)
+                         : 0u;
+        }
+        mma_f16_16816(o[2 * ch], pa, bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x5410)),
+                      bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x5410)));
+        mma_f16_16816(o[2 * ch + 1], pa, bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x7632)),
+                      bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x7632)));
+      }
+    }
+  };
+
   long long x = x0;
   for (int st = 0; x < x1; ++st) {
-    const int slot = st % NSTAGE, use = st / NSTAGE;
+    const int slot = st % S::NST, use = st / S::NST;
     bool ok = !aborted() && mbar_wait(smem_u32(&bar_full[slot]), use & 1);
     if (!ok) fail();
     const StageMeta m = meta[slot];
@@ -240,92 +495,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     if (ok) {
       const uint32_t kb = smem_u32(smem + slot * S::STAGE);
       const uint32_t vb = kb + S::TILE;
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int kd = 0; kd < D / 16; ++kd) {
-        const int row = 16 * cw + (lane & 7) + ((lane >> 4) << 3);
-        const int ch = 2 * kd + ((lane >> 3) & 1);
-        const uint32_t addr = kb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(addr, b0, b1, b2, b3);
-        mma_bf16_16816(s[0], qa[kd], b0, b1);
-        mma_bf16_16816(s[1], qa[kd], b2, b3);
-      }
       const int kw = 16 * cw;   // first key of this warp in the stage
-#pragma unroll
-      for (int nn = 0; nn < 2; ++nn)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = kw + 8 * nn + 2 * (lane & 3) + (e & 1);
-          s[nn][e] = j < n ? s[nn][e] * a.scale_log2 : -INFINITY;
-        }
-      float mx_a = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-      float mx_b = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-      // The exponent base only moves up when a row's maximum grows by more
-      // than 2^8, so the accumulator is rarely rescaled.
-      const bool up_a = mx_a > m_a + 8.f, up_b = mx_b > m_b + 8.f;
-      if (__any_sync(0xffffffffu, up_a || up_b)) {
-        const float al_a = up_a ? exp2f(m_a - mx_a) : 1.f;
-        const float al_b = up_b ? exp2f(m_b - mx_b) : 1.f;
-        if (up_a) m_a = mx_a;
-        if (up_b) m_b = mx_b;
-        l_a *= al_a;
-        l_b *= al_b;
-#pragma unroll
-        for (int nn = 0; nn < NT_O; ++nn) {
-          o[nn][0] *= al_a;
-          o[nn][1] *= al_a;
-          o[nn][2] *= al_b;
-          o[nn][3] *= al_b;
-        }
+      if (FP8 ? kw < n : true) {   // (FP8 mode: a warp past the valid keys adds nothing)
+        if constexpr (FP8) fp8_stage(m, kb, vb, scl + slot * 2 * S::SCL_SLOT, kw, n);
+        else bf16_stage(kb, vb, kw, n, slot);
       }
-      const float base_a = m_a == -INFINITY ? 0.f : m_a;
-      const float base_b = m_b == -INFINITY ? 0.f : m_b;
-#pragma unroll
-      for (int nn = 0; nn < 2; ++nn) {
-        s[nn][0] = exp2f(s[nn][0] - base_a);
-        s[nn][1] = exp2f(s[nn][1] - base_a);
-        s[nn][2] = exp2f(s[nn][2] - base_b);
-        s[nn][3] = exp2f(s[nn][3] - base_b);
-      }
-      l_a += s[0][0] + s[0][1] + s[1][0] + s[1][1];
-      l_b += s[0][2] + s[0][3] + s[1][2] + s[1][3];
-      if (16 * cw + 16 > n) {
-        // Rows past the stage's valid count carry p = 0, but 0 * NaN is NaN:
-        // clear this warp's V rows there (bytes past the end of a buffer need
-        // not be finite).  Each warp reads only its own 16 V rows.
-        for (int i = lane; i < 16 * (D / 8); i += 32) {
-          const int row = 16 * cw + i / (D / 8), ch = i % (D / 8);
-          if (row >= n) {
-            uint8_t* dst = smem + slot * S::STAGE + S::TILE + (ch >> 3) * S::HALF + row * 128 +
-                           (((ch & 7) ^ (row & 7)) << 4);
-            *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-        __syncwarp();
-      }
-      uint32_t pa[4];
-      pa[0] = pack_bf16(s[0][0], s[0][1]);
-      pa[1] = pack_bf16(s[0][2], s[0][3]);
-      pa[2] = pack_bf16(s[1][0], s[1][1]);
-      pa[3] = pack_bf16(s[1][2], s[1][3]);
-#pragma unroll
-      for (int j = 0; j < D / 16; ++j) {
-        const int row = 16 * cw + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ch = 2 * j + (lane >> 4);
-        const uint32_t addr = vb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(addr, b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * j], pa, b0, b1);
-        mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
-      }
-      // generic-proxy writes above must be ordered before the next TMA write
-      if (16 * cw + 16 > n) fence_proxy_async_smem();
-      __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_empty[slot]));
     }
     x += n;
@@ -363,16 +537,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         wl[cw][ra] = l_a;
         wl[cw][rb] = l_b;
       }
-      const int cq = 2 * (lane & 3);
 #pragma unroll
       for (int nn = 0; nn < NT_O; ++nn) {
+        // columns of accumulator block nn held by this thread (FP8 mode: permuted)
+        const int c0 = FP8 ? 16 * (nn >> 1) + 4 * (lane & 3) + (nn & 1) : 8 * nn + 2 * (lane & 3);
+        const int c1 = FP8 ? c0 + 2 : c0 + 1;
         if (ra >= rh && ra < rh + 4) {
-          comb[(cw * 4 + ra - rh) * D + 8 * nn + cq] = o[nn][0];
-          comb[(cw * 4 + ra - rh) * D + 8 * nn + cq + 1] = o[nn][1];
+          comb[(cw * 4 + ra - rh) * D + c0] = o[nn][0];
+          comb[(cw * 4 + ra - rh) * D + c1] = o[nn][1];
         }
         if (rb >= rh && rb < rh + 4) {
-          comb[(cw * 4 + rb - rh) * D + 8 * nn + cq] = o[nn][2];
-          comb[(cw * 4 + rb - rh) * D + 8 * nn + cq + 1] = o[nn][3];
+          comb[(cw * 4 + rb - rh) * D + c0] = o[nn][2];
+          comb[(cw * 4 + rb - rh) * D + c1] = o[nn][3];
         }
       }
       named_sync(1, 32 * NCW);
@@ -515,21 +691,38 @@ int decode_num_ctas(const CacheView& c, long long len0, int num_sms) {
   return (int)n;
 }
 
-bool decode_make_maps(const CacheView& c, DecodeMaps* m) {
+const char* decode_make_maps(const CacheView& c, DecodeMaps* m) {
   const unsigned long long ctx_rows = (unsigned long long)c.B * c.Hkv * c.L;
   const unsigned long long q_rows = (unsigned long long)c.B * c.Hkv * c.q_cap;
-  return make_tmap_bf16_2d(&m->k_ctx, c.ctxK, ctx_rows, c.D, KS, 64) &&
-         make_tmap_bf16_2d(&m->v_ctx, c.ctxV, ctx_rows, c.D, KS, 64) &&
-         make_tmap_bf16_2d(&m->k_q, c.qK, q_rows, c.D, KS, 64) &&
-         make_tmap_bf16_2d(&m->v_q, c.qV, q_rows, c.D, KS, 64);
+  if (!make_tmap_bf16_2d(&m->k_ctx, c.ctxK, ctx_rows, c.D, KS, 64) ||
+      !make_tmap_bf16_2d(&m->v_ctx, c.ctxV, ctx_rows, c.D, KS, 64))
+    return "context K/V";
+  if (!make_tmap_bf16_2d(&m->k_q, c.qK, q_rows, c.D, KS, 64) ||
+      !make_tmap_bf16_2d(&m->v_q, c.qV, q_rows, c.D, KS, 64))
+    return "query region K/V";
+  if (!c.ctxK8) return nullptr;
+  if (!make_tmap_u8_2d(&m->k8_ctx, c.ctxK8, ctx_rows, c.D, KS) ||
+      !make_tmap_u8_2d(&m->v8_ctx, c.ctxV8, ctx_rows, c.D, KS))
+    return "FP8 context K/V";
+  if (!make_tmap_f32_row(&m->ks_ctx, c.ctxKs, ctx_rows, DSmem<128, true>::SCL_BOX) ||
+      !make_tmap_f32_row(&m->vs_ctx, c.ctxVs, ctx_rows, DSmem<128, true>::SCL_BOX))
+    return "FP8 row scales";
+  if (!make_tmap_bf16_2d(&m->k_q64, c.qK, q_rows, c.D, 64, 64) ||
+      !make_tmap_bf16_2d(&m->v_q64, c.qV, q_rows, c.D, 64, 64))
+    return "64-row query region K/V";
+  return nullptr;
+}
+
+template <int D, bool FP8>
+cudaError_t decode_prepare_one() {
+  return cudaFuncSetAttribute(decode_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              DSmem<D, FP8>::BYTES + 1024);
 }
 
 cudaError_t decode_prepare(int D) {
-  if (D == 128)
-    return cudaFuncSetAttribute(decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                DSmem<128>::BYTES + 1024);
-  return cudaFuncSetAttribute(decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              DSmem<64>::BYTES + 1024);
+  cudaError_t e = D == 128 ? decode_prepare_one<128, false>() : decode_prepare_one<64, false>();
+  if (e == cudaSuccess) e = D == 128 ? decode_prepare_one<128, true>() : decode_prepare_one<64, true>();
+  return e;
 }
 
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
@@ -540,6 +733,12 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.tv_ctx = maps.v_ctx;
   a.tk_q = maps.k_q;
   a.tv_q = maps.v_q;
+  a.tk8 = maps.k8_ctx;
+  a.tv8 = maps.v8_ctx;
+  a.tkq64 = maps.k_q64;
+  a.tvq64 = maps.v_q64;
+  a.tks = maps.ks_ctx;
+  a.tvs = maps.vs_ctx;
   a.c = c;
   a.scale_log2 = scale * kLog2e;
   a.len0 = len0;
@@ -555,10 +754,15 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.partS = s.partS;
   a.tickets = s.tickets;
   a.err = s.err;
-  if (c.D == 128)
-    decode_kernel<128><<<plan.ncta, NTHREADS, DSmem<128>::BYTES + 1024, st>>>(a);
+  const bool fp8 = c.ctxK8 != nullptr;
+  if (c.D == 128 && fp8)
+    decode_kernel<128, true><<<plan.ncta, NTHREADS, DSmem<128, true>::BYTES + 1024, st>>>(a);
+  else if (c.D == 128)
+    decode_kernel<128, false><<<plan.ncta, NTHREADS, DSmem<128, false>::BYTES + 1024, st>>>(a);
+  else if (fp8)
+    decode_kernel<64, true><<<plan.ncta, NTHREADS, DSmem<64, true>::BYTES + 1024, st>>>(a);
   else
-    decode_kernel<64><<<plan.ncta, NTHREADS, DSmem<64>::BYTES + 1024, st>>>(a);
+    decode_kernel<64, false><<<plan.ncta, NTHREADS, DSmem<64, false>::BYTES + 1024, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -623,6 +827,7 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
   using namespace star;
   int rc = check_params(p);
   if (rc) return rc;
+  if (p->kv_fp8) return set_error(STAR_EINVAL, "the no-alloc decode streams bf16 only (kv_fp8 must be 0)");
   if (!ctx_k || !ctx_v || !q_k || !q_v || !q || !k || !v || !o || !lse)
     return set_error(STAR_EINVAL, "NULL tensor pointer");
   const void* ptrs[] = {ctx_k, ctx_v, q_k, q_v, q, k, v, o, lse};
@@ -647,6 +852,10 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
   c.ctxV = static_cast<bf16*>(const_cast<void*>(ctx_v));
   c.qK = static_cast<bf16*>(q_k);
   c.qV = static_cast<bf16*>(q_v);
+  c.ctxK8 = nullptr;
+  c.ctxV8 = nullptr;
+  c.ctxKs = nullptr;
+  c.ctxVs = nullptr;
 
   DecodePlan pl;
   pl.ncta = decode_num_ctas(c, q_len, sms);
@@ -657,7 +866,11 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
                                   "(B*Hkv*G*D*(ceil(SMs/(B*Hkv))+2) must be <= 1048576 floats, "
                                   "B*Hkv <= 1024)");
   DecodeMaps maps;
-  if (!decode_make_maps(c, &maps)) return set_error(STAR_EINVAL, "TMA tensor maps rejected");
+  if (const char* bad = decode_make_maps(c, &maps)) {
+    char msg[96];
+    snprintf(msg, sizeof(msg), "TMA tensor map rejected by the driver: %s", bad);
+    return set_error(STAR_EINVAL, msg);
+  }
   Scratch sc;
   sc.partA = base;
   sc.partS = base + kNoAllocPartA;

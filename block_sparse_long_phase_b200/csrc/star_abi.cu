@@ -101,6 +101,7 @@ int validate_params(const star_params* p) {
   if (p->anchor < 0 || p->anchor > p->block)
     return fail(STAR_EINVAL, "anchor %d must satisfy 0 <= b_a <= b (%d)", p->anchor, p->block);
   if (p->q_cap < 1) return fail(STAR_EINVAL, "q_cap must be >= 1");
+  if (p->kv_fp8 != 0 && p->kv_fp8 != 1) return fail(STAR_EINVAL, "kv_fp8 must be 0 or 1");
   if (p->L + p->q_cap + 1 > 0x7fffffffLL) return fail(STAR_EINVAL, "L + q_cap too large");
   if ((p->L + p->block - 1) / p->block > 0x7fff) return fail(STAR_EINVAL, "too many blocks");
   return STAR_OK;
@@ -174,6 +175,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const size_t o_t = take(n_tickets * 4);
   const size_t o_e = take(sizeof(int));
   const size_t o_w = take(work.size() * sizeof(int4));
+  const bool fp8 = p->kv_fp8 != 0;
+  const long long ctx_rows = (long long)p->B * p->Hkv * p->L;
+  const size_t o_k8 = fp8 ? take(kv_ctx) : 0, o_v8 = fp8 ? take(kv_ctx) : 0;
+  const size_t o_ks = fp8 ? take(ctx_rows * 4) : 0, o_vs = fp8 ? take(ctx_rows * 4) : 0;
   e = cudaMalloc(&c->block, off);
   if (e != cudaSuccess) {
     delete c;
@@ -192,6 +197,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
   c->scratch.partS_elems = partS;
   c->scratch.n_tickets = (int)n_tickets;
   c->ctx_work = reinterpret_cast<int4*>(base + o_w);
+  v.ctxK8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_k8) : nullptr;
+  v.ctxV8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_v8) : nullptr;
+  v.ctxKs = fp8 ? reinterpret_cast<float*>(base + o_ks) : nullptr;
+  v.ctxVs = fp8 ? reinterpret_cast<float*>(base + o_vs) : nullptr;
   // Zero everything once: decode streams whole 128-row boxes and masks the
   // rows past the end, which must hold finite values.
   e = cudaMemset(c->block, 0, off);
@@ -204,10 +213,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
     delete c;
     return cuda_fail(e, "cache initialisation");
   }
-  if (!star::decode_make_maps(v, &c->dmaps)) {
+  if (const char* bad = star::decode_make_maps(v, &c->dmaps)) {
     cudaFree(c->block);
     delete c;
-    return fail(STAR_EINVAL, "TMA tensor maps of the cache rejected");
+    return fail(STAR_EINVAL, "TMA tensor map of the cache rejected by the driver: %s", bad);
   }
   e = star::decode_prepare(v.D);
   if (e == cudaSuccess) e = star::attn_tc_prepare(v.D);
@@ -266,6 +275,20 @@ int star_cache_segment(const star_cache* c, int seg, void** k, void** v, long lo
   return STAR_OK;
 }
 
+int star_cache_segment_fp8(const star_cache* c, int seg, void** k8, void** v8, float** k_scale,
+                           float** v_scale) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  const star::CacheView& w = c->view;
+  if (!w.ctxK8) return fail(STAR_EINVAL, "cache has no FP8 copy (kv_fp8 = 0)");
+  if (seg < 0 || seg >= w.n_seg) return fail(STAR_EINVAL, "context segment %d out of range", seg);
+  const long long rows = (long long)seg * w.B * w.Hkv * (long long)w.b;
+  if (k8) *k8 = w.ctxK8 + rows * w.D;
+  if (v8) *v8 = w.ctxV8 + rows * w.D;
+  if (k_scale) *k_scale = w.ctxKs + rows;
+  if (v_scale) *v_scale = w.ctxVs + rows;
+  return STAR_OK;
+}
+
 int star_cache_reset_query(star_cache* c) {
   if (!c) return fail(STAR_EINVAL, "cache is NULL");
   c->q_len = 0;
@@ -283,6 +306,7 @@ int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, 
       static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work,
       c->scratch.err, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
+  if (e == cudaSuccess && c->view.ctxK8) e = star::launch_quantize_ctx_fp8(c->view, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
   c->q_len = 0;
   return STAR_OK;

@@ -25,6 +25,12 @@ struct CacheView {
   bf16* ctxV;
   bf16* qK;  // query region [B][Hkv][q_cap][D]
   bf16* qV;
+  // optional FP8 (E4M3) copy of the context cache, same row order, and the
+  // per-row scales (null when the cache keeps bf16 only)
+  uint8_t* ctxK8;
+  uint8_t* ctxV8;
+  float* ctxKs;
+  float* ctxVs;
 };
 
 __host__ __device__ inline long long seg_len(const CacheView& c, int seg) {
@@ -90,8 +96,13 @@ int decode_num_ctas(const CacheView& c, long long len0, int num_sms);
 // TMA maps of the cache, built once per cache.
 struct DecodeMaps {
   CUtensorMap k_ctx, v_ctx, k_q, v_q;
+  CUtensorMap k8_ctx, v8_ctx, k_q64, v_q64;   // FP8 context rows; 64-row query boxes
+  CUtensorMap ks_ctx, vs_ctx;                 // FP8 per-row scales
 };
-bool decode_make_maps(const CacheView& c, DecodeMaps* m);
+cudaError_t launch_quantize_ctx_fp8(const CacheView& c, cudaStream_t st);
+// Builds the cache's TMA maps; returns nullptr, or the name of the map the
+// driver rejected.
+const char* decode_make_maps(const CacheView& c, DecodeMaps* m);
 cudaError_t decode_prepare(int D);   // one-time kernel attributes
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
                                const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,

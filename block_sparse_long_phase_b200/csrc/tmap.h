@@ -36,4 +36,37 @@ inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, unsigned long 
   return r == CUDA_SUCCESS;
 }
 
+// [rows][cols] bytes (cols = 64 or 128), box of box_rows whole rows, swizzled
+// to match the row length: 128-byte swizzle for 128-byte rows, 64-byte for 64.
+inline bool make_tmap_u8_2d(CUtensorMap* map, const void* base, unsigned long long rows,
+                            unsigned long long cols, unsigned box_rows) {
+  auto enc = tmap_encoder();
+  if (!enc || (cols != 64 && cols != 128)) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {(cuuint32_t)cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// [n] float32 as a one-row 2-D tensor, boxes of `box` elements (box * 4 a
+// multiple of 16); elements past the end read as zero.  The row stride only
+// has to satisfy the encoder (a multiple of 16 bytes): the tensor has one row.
+inline bool make_tmap_f32_row(CUtensorMap* map, const float* base, unsigned long long n, unsigned box) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {n, 1};
+  cuuint64_t strides[1] = {(n * 4 + 15) / 16 * 16};
+  cuuint32_t bx[2] = {box, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, bx,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace star

@@ -67,6 +67,13 @@ typedef struct {
   int anchor;       /* anchor size b_a, 0 <= b_a <= b (0 = no anchor)       */
   int q_cap;        /* query-region capacity: query tokens + decode steps   */
   float scale;      /* softmax scale; <= 0 selects 1/sqrt(D)                */
+  int kv_fp8;       /* 1: the cache also keeps an FP8 (E4M3) copy of the
+                       context K/V that star_decode_step streams (half the
+                       bytes); 0: bf16 only.  D = 64 or 128.  Quantisation
+                       (no counterpart in the pages, which call KV
+                       quantisation orthogonal): per cached row of one kv
+                       head, s = max|x| / 448 (1 if max|x| <= 1e-30), codes
+                       = e4m3_rn(x * (1/s)) in float32, value = code * s.   */
 } star_params;
 
 /* Opaque KV cache: n context segments + 1 query-region segment, the segment
@@ -82,6 +89,12 @@ STAR_API int star_cache_create(const star_params* p, star_cache** out);
 /* Frees everything the cache owns (synchronises the device first).  NULL is
  * accepted. */
 STAR_API int star_cache_destroy(star_cache* c);
+
+/* FP8 copy of context segment `seg` (kv_fp8 caches only): E4M3 codes of K and
+ * V as [B][Hkv][len][D] bytes and their per-row float32 scales [B][Hkv][len],
+ * device pointers.  STAR_EINVAL if the cache has no FP8 copy. */
+STAR_API int star_cache_segment_fp8(const star_cache* c, int seg, void** k8, void** v8,
+                                    float** k_scale, float** v_scale);
 
 /* Reads and clears the cache's device error word (synchronous: waits for
  * the work already queued on the device).  *flag is non-zero if a kernel
@@ -108,7 +121,8 @@ STAR_API int star_cache_reset_query(star_cache* c);
  * LSE [B][Hq][L] float32 out.  Token t of block i sees tokens j <= t of its
  * own block and, when i >= 1, the whole anchor [0, b_a).  Writes the cache:
  * segment i receives K/V rows of block i only (anchor KV discarded, every
- * context token cached exactly once).  Empties the query region. */
+ * context token cached exactly once), and with kv_fp8 also their FP8 copy.
+ * Empties the query region. */
 STAR_API int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V,
                     void* O, float* LSE, void* stream);
 
@@ -125,7 +139,10 @@ STAR_API int star_query_prefill(star_cache* c, int lq, const void* Q, const void
  * [B][Hkv][1][D] to the query region, then q [B][Hq][1][D] attends to every
  * context token and every query-region row (itself included): split-KV
  * partials merged on-chip.  o [B][Hq][1][D] bf16, lse [B][Hq] float32.
- * STAR_ENOSPC if the query region is full. */
+ * With kv_fp8 the context rows are read from the FP8 copy (dequantised on
+ * chip, fp16 MMA: q and the query region's bf16 K/V are rounded to fp16,
+ * so their magnitudes must stay within fp16 range); the query region stays
+ * bf16 in memory.  STAR_ENOSPC if the query region is full. */
 STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
                      void* o, float* lse, void* stream);
 
@@ -145,7 +162,8 @@ STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const flo
  * tickets, error word) lives in one static device array of the library,
  * 4.3 MiB, present on every GPU that loads the library until the process
  * exits.  Same arithmetic and kernel as star_decode_step.
- *   p          layer parameters, as for star_cache_create (scale <= 0: 1/sqrt(D))
+ *   p          layer parameters, as for star_cache_create (scale <= 0: 1/sqrt(D));
+ *              kv_fp8 must be 0 (bf16 context only)
  *   q_len      query-region rows in use before this step; this call writes
  *              row q_len of q_k / q_v with k / v
  *   ctx_k/v    context cache, the layout star_cache_create uses: segment i

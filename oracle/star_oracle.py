@@ -336,3 +336,44 @@ def phase2_partials(q_rows, segments, qk_region, qv_region, visible_q, scale):
             O[bi, h] = o
             LSE[bi, h] = lse
     return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) context cache for decode.
+#
+# The pages call KV-cache quantisation orthogonal to the method and fix no
+# scheme, so this is the build's own definition, stated once here and in the
+# C header: every cached K or V row (one token of one kv head) is scaled by
+# s = max|x| / 448 (s = 1 when max|x| <= 1e-30), each value x * (1/s) (float32,
+# round to nearest) is rounded to E4M3 (round to nearest even; |x/s| <= 448
+# so nothing saturates), and the dequantised value is e4m3 * s.  Attention
+# then runs on the dequantised rows exactly as before.
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def fp8_quantize_rows(x):
+    """Per-row E4M3 codes (uint8) and float32 scales of ``x`` [..., D]."""
+    import torch
+    x32 = _f64(x).astype(np.float32)
+    amax = np.abs(x32).max(axis=-1)
+    s = np.where(amax > np.float32(1e-30), amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    inv = (np.float32(1.0) / s).astype(np.float32)
+    y = (x32 * inv[..., None]).astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(y)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return codes, s
+
+
+def e4m3_value(codes):
+    """float64 value of E4M3 codes (no NaN codes are produced by the quantiser)."""
+    c = np.asarray(codes, np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = sign * (1.0 + m / 8.0) * np.exp2(e - 7.0)
+    sub = sign * (m / 8.0) * np.exp2(-6.0)
+    return np.where(e == 0, sub, normal)
+
+
+def fp8_dequantize_rows(codes, s):
+    return e4m3_value(codes) * np.asarray(s, np.float64)[..., None]

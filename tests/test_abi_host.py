@@ -51,6 +51,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
         _abi.StarParams(1, 4, 2, 64, 1024, 0, 0, 8, 0.0),        # b = 0
         _abi.StarParams(1, 4, 2, 64, 1024, 256, -1, 8, 0.0),     # b_a < 0
         _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 0, 0.0),    # q_cap = 0
+        _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 2), # kv_fp8 not 0/1
     ]
     for p in bad:
         assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EINVAL
@@ -65,6 +66,10 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.star_ctx_encode(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_decode_step(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_query_prefill(None, 4, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_cache_segment_fp8(None, 0, None, None, None, None) == _abi.STAR_EINVAL
+    p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 1)  # the no-alloc path is bf16 only
+    assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *([None] * 10)) == _abi.STAR_EINVAL
+    assert b"kv_fp8" in lib.star_last_error()
     assert lib.star_cache_destroy(None) == _abi.STAR_OK
     assert lib.star_cache_num_segments(None) == 0
 

@@ -136,6 +136,12 @@ template <int D>
 SM100_DEV uint32_t sw8(int row, int chunk) {
   return (uint32_t)(row * D + ((chunk ^ (D == 128 ? (row & 7) : ((row >> 1) & 3))) << 4));
 }
+// Transpose of an 8x8 matrix of 16-bit values held one row pair per thread.
+SM100_DEV uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(x));
+  return d;
+}
 SM100_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -144,11 +150,10 @@ SM100_DEV void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, int NG>   // NG: blocks of 8 heads per kv group (G <= 8 NG)
 __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
   using S = DSmem<D, FP8>;
   constexpr int NH = D / 64;
-  constexpr int NT_O = D / 8;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -261,107 +266,152 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   }
 
   // --------------------------------- consumers --------------------------------
+  // Keys are the MMA's M dimension: per warp and stage, S^T = K q^T over the
+  // warp's 16 keys (M = 16 keys, N = 8 heads of the group per block of NG,
+  // K = 16 columns of d) and O^T += V^T P^T (M = 16 rows of d, N = heads,
+  // K = the 16 keys).  With G <= 8 every key costs D/16 MMAs each way.
+  // Thread (t = lane/4, c = lane%4) holds, per head block nb, the heads
+  // g = 8nb + 2c + e (e = 0, 1): scores of keys t and t+8, O^T rows t and t+8
+  // of each 16-row block of d, and the running max / sum of those heads.
   const int cw = warp - 1;                       // consumer warp 0..7
   const int ctid = tid - 32;                     // 0..255
-  uint32_t qa[D / 16][4];
-  float o[NT_O][4];
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+  const int t4 = lane >> 2, c4 = lane & 3;
+  uint32_t qb[D / 16][NG][2];                    // B fragments of q^T
+  float oT[D / 16][NG][4];                       // C fragments of O^T
+  float mx[NG][2], ls[NG][2];                    // per head: max (log2 units), partial sum
   int cur_bg = -1;
   auto load_q = [&](int bg) {
     const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
-    const int r0 = lane >> 2, r1 = r0 + 8;
-    const bf16* qb = a.q + ((long long)bb * c.Hq + (long long)g * G) * D;
+    const bf16* qg = a.q + ((long long)bb * c.Hq + (long long)g * G) * D;
 #pragma unroll
     for (int kd = 0; kd < D / 16; ++kd) {
       // FP8 mode permutes the contraction index inside each 16-column step:
       // k-slots 2c, 2c+1 take columns 4c, 4c+1 and k-slots 2c+8, 2c+9 take
       // 4c+2, 4c+3, the order in which one 32-bit word of a key row holds them
-      const int col = FP8 ? 16 * kd + 4 * (lane & 3) : 16 * kd + 2 * (lane & 3);
+      const int col = FP8 ? 16 * kd + 4 * c4 : 16 * kd + 2 * c4;
       const int hi = FP8 ? 2 : 8;
-      qa[kd][0] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col) : 0u;
-      qa[kd][1] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col) : 0u;
-      qa[kd][2] = r0 < G ? *reinterpret_cast<const uint32_t*>(qb + r0 * D + col + hi) : 0u;
-      qa[kd][3] = r1 < G ? *reinterpret_cast<const uint32_t*>(qb + r1 * D + col + hi) : 0u;
-      if (FP8) {                                   // the FP8 path multiplies in f16
 #pragma unroll
-        for (int e = 0; e < 4; ++e) qa[kd][e] = bf16x2_to_f16x2(qa[kd][e]);
+      for (int nb = 0; nb < NG; ++nb) {
+        const int h = 8 * nb + t4;
+        uint32_t b0 = h < G ? *reinterpret_cast<const uint32_t*>(qg + h * D + col) : 0u;
+        uint32_t b1 = h < G ? *reinterpret_cast<const uint32_t*>(qg + h * D + col + hi) : 0u;
+        if (FP8) {                                 // the FP8 path multiplies in f16
+          b0 = bf16x2_to_f16x2(b0);
+          b1 = bf16x2_to_f16x2(b1);
+        }
+        qb[kd][nb][0] = b0;
+        qb[kd][nb][1] = b1;
       }
     }
   };
   auto reset_state = [&]() {
 #pragma unroll
-    for (int n = 0; n < NT_O; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    for (int m = 0; m < D / 16; ++m)
 #pragma unroll
-    for (int kd = 0; kd < D / 16; ++kd) qa[kd][0] = qa[kd][1] = qa[kd][2] = qa[kd][3] = 0u;
-    m_a = m_b = -INFINITY;
-    l_a = l_b = 0.f;
+      for (int nb = 0; nb < NG; ++nb) {
+        oT[m][nb][0] = oT[m][nb][1] = oT[m][nb][2] = oT[m][nb][3] = 0.f;
+        qb[m][nb][0] = qb[m][nb][1] = 0u;
+      }
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb) {
+      mx[nb][0] = mx[nb][1] = -INFINITY;
+      ls[nb][0] = ls[nb][1] = 0.f;
+    }
   };
   reset_state();
 
-  // Scale and mask the scores of this warp's 16 keys (sk: per-key factor on
-  // the log2 scale), update the running max / sum, turn scores into p.
-  auto softmax_update = [&](float (&s)[2][4], const float (&sk)[4], int kw, int n) {
+  // Scale and mask the scores (sk0, sk1: factor on the log2 scale of keys t
+  // and t+8), update the running max / sum per head, turn scores into p.
+  auto softmax_update = [&](float (&s)[NG][4], float sk0, float sk1, int kw, int n) {
+    const bool v0 = kw + t4 < n, v1 = kw + t4 + 8 < n;
 #pragma unroll
-    for (int nn = 0; nn < 2; ++nn)
+    for (int nb = 0; nb < NG; ++nb) {
+      s[nb][0] = v0 ? s[nb][0] * sk0 : -INFINITY;
+      s[nb][1] = v0 ? s[nb][1] * sk0 : -INFINITY;
+      s[nb][2] = v1 ? s[nb][2] * sk1 : -INFINITY;
+      s[nb][3] = v1 ? s[nb][3] * sk1 : -INFINITY;
+    }
+    float mn[NG][2];
+    bool up = false;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = kw + 8 * nn + 2 * (lane & 3) + (e & 1);
-        s[nn][e] = j < n ? s[nn][e] * sk[nn * 2 + (e & 1)] : -INFINITY;
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = fmaxf(s[nb][e], s[nb][2 + e]);
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        mn[nb][e] = v;
+        up |= v > mx[nb][e] + 8.f;
       }
-    float mx_a = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-    float mx_b = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    // The exponent base only moves up when a row's maximum grows by more
+    // The exponent base only moves up when a head's maximum grows by more
     // than 2^8, so the accumulator is rarely rescaled.
-    const bool up_a = mx_a > m_a + 8.f, up_b = mx_b > m_b + 8.f;
-    if (__any_sync(0xffffffffu, up_a || up_b)) {
-      const float al_a = up_a ? exp2f(m_a - mx_a) : 1.f;
-      const float al_b = up_b ? exp2f(m_b - mx_b) : 1.f;
-      if (up_a) m_a = mx_a;
-      if (up_b) m_b = mx_b;
-      l_a *= al_a;
-      l_b *= al_b;
+    if (__any_sync(0xffffffffu, up)) {
 #pragma unroll
-      for (int nn = 0; nn < NT_O; ++nn) {
-        o[nn][0] *= al_a;
-        o[nn][1] *= al_a;
-        o[nn][2] *= al_b;
-        o[nn][3] *= al_b;
+      for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const bool u = mn[nb][e] > mx[nb][e] + 8.f;
+          const float al = u ? exp2f(mx[nb][e] - mn[nb][e]) : 1.f;
+          if (u) mx[nb][e] = mn[nb][e];
+          ls[nb][e] *= al;
+#pragma unroll
+          for (int m = 0; m < D / 16; ++m) {
+            oT[m][nb][e] *= al;
+            oT[m][nb][2 + e] *= al;
+          }
+        }
+    }
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float base = mx[nb][e] == -INFINITY ? 0.f : mx[nb][e];
+        s[nb][e] = exp2f(s[nb][e] - base);
+        s[nb][2 + e] = exp2f(s[nb][2 + e] - base);
+        ls[nb][e] += s[nb][e] + s[nb][2 + e];
       }
-    }
-    const float base_a = m_a == -INFINITY ? 0.f : m_a;
-    const float base_b = m_b == -INFINITY ? 0.f : m_b;
-#pragma unroll
-    for (int nn = 0; nn < 2; ++nn) {
-      s[nn][0] = exp2f(s[nn][0] - base_a);
-      s[nn][1] = exp2f(s[nn][1] - base_a);
-      s[nn][2] = exp2f(s[nn][2] - base_b);
-      s[nn][3] = exp2f(s[nn][3] - base_b);
-    }
-    l_a += s[0][0] + s[0][1] + s[1][0] + s[1][1];
-    l_b += s[0][2] + s[0][3] + s[1][2] + s[1][3];
   };
 
-  // One stage of bf16 keys: 16 keys per warp, K and V fragments straight from
-  // the 128-byte-swizzled TMA tiles.
+  // P^T as the B operand of O^T += V^T P^T: the score fragment holds keys t,
+  // t+8 x heads 2c, 2c+1; a warp transpose of each 8x8 block gives keys 2c,
+  // 2c+1 (+8) x head t.  pv0 / pv1 scale keys t / t+8 (FP8: the V row scale).
+  auto p_fragments = [&](const float (&s)[NG][4], float pv0, float pv1, uint32_t (&pb)[NG][2]) {
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb) {
+      const uint32_t x0 = FP8 ? pack_f16(s[nb][0] * pv0, s[nb][1] * pv0) : pack_bf16(s[nb][0], s[nb][1]);
+      const uint32_t x1 = FP8 ? pack_f16(s[nb][2] * pv1, s[nb][3] * pv1) : pack_bf16(s[nb][2], s[nb][3]);
+      pb[nb][0] = movmatrix_trans(x0);
+      pb[nb][1] = movmatrix_trans(x1);
+    }
+  };
+
+  // One stage of bf16 keys: K and V fragments straight from the
+  // 128-byte-swizzled TMA tiles.
   auto bf16_stage = [&](uint32_t kb, uint32_t vb, int kw, int n, int slot) {
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float s[NG][4], s2[NG][4];                   // even / odd column steps: two short chains
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nb][e] = s2[nb][e] = 0.f;
 #pragma unroll
     for (int kd = 0; kd < D / 16; ++kd) {
-      uint32_t b0, b1, b2, b3;
-      const int ch = 2 * kd + ((lane >> 3) & 1);
-      const int row = kw + (lane & 7) + ((lane >> 4) << 3);
-      ldmatrix_x4(kb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b0, b1, b2, b3);
-      mma_bf16_16816(s[0], qa[kd], b0, b1);
-      mma_bf16_16816(s[1], qa[kd], b2, b3);
+      uint32_t af[4];
+      const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int ch = 2 * kd + (lane >> 4);
+      ldmatrix_x4(kb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), af[0], af[1], af[2],
+                  af[3]);
+#pragma unroll
+      for (int nb = 0; nb < NG; ++nb)
+        mma_bf16_16816((kd & 1) ? s2[nb] : s[nb], af, qb[kd][nb][0], qb[kd][nb][1]);
     }
-    const float sk[4] = {a.scale_log2, a.scale_log2, a.scale_log2, a.scale_log2};
-    softmax_update(s, sk, kw, n);
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nb][e] += s2[nb][e];
+    softmax_update(s, a.scale_log2, a.scale_log2, kw, n);
     if (kw + 16 > n) {
-      // Rows past the stage's valid count carry p = 0, but 0 * NaN is NaN:
+      // Keys past the stage's valid count carry p = 0, but 0 * NaN is NaN:
       // clear this warp's V rows there (bytes past the end of a buffer need
       // not be finite).  Each warp reads only its own 16 V rows.
       for (int i = lane; i < 16 * (D / 8); i += 32) {
@@ -374,36 +424,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       }
       __syncwarp();
     }
-    uint32_t pa[4];
-    pa[0] = pack_bf16(s[0][0], s[0][1]);
-    pa[1] = pack_bf16(s[0][2], s[0][3]);
-    pa[2] = pack_bf16(s[1][0], s[1][1]);
-    pa[3] = pack_bf16(s[1][2], s[1][3]);
+    uint32_t pb[NG][2];
+    p_fragments(s, 1.f, 1.f, pb);
 #pragma unroll
-    for (int j = 0; j < D / 16; ++j) {
-      const int ch = 2 * j + (lane >> 4);
-      uint32_t b0, b1, b2, b3;
-      const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
-      ldmatrix_x4_trans(vb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b0, b1, b2, b3);
-      mma_bf16_16816(o[2 * j], pa, b0, b1);
-      mma_bf16_16816(o[2 * j + 1], pa, b2, b3);
+    for (int m = 0; m < D / 16; ++m) {
+      uint32_t af[4];
+      const int row = kw + (lane & 7) + ((lane >> 4) << 3);
+      const int ch = 2 * m + ((lane >> 3) & 1);
+      ldmatrix_x4_trans(vb + (ch >> 3) * S::HALF + row * 128 + (((ch & 7) ^ (row & 7)) << 4), af[0], af[1],
+                        af[2], af[3]);
+#pragma unroll
+      for (int nb = 0; nb < NG; ++nb) mma_bf16_16816(oT[m][nb], af, pb[nb][0], pb[nb][1]);
     }
     // generic-proxy writes above must be ordered before the next TMA write
     if (kw + 16 > n) fence_proxy_async_smem();
   };
 
   // One stage in FP8 mode.  Context stages hold E4M3 codes: ldmatrix on the
-  // swizzled byte tile gives each thread one 32-bit word (4 codes) per 8x16-byte
-  // matrix, converted in registers to f16 MMA operands -- for K the word is a
-  // B fragment under the permuted contraction order of qa; for V (.trans) it
-  // holds two keys x two columns, regrouped by a byte permute.  The output
-  // columns of V are permuted too: accumulator block nb, column n holds
-  // d = 16 (nb / 2) + 2 n + nb % 2.  Query-region stages hold bf16 rows, read
-  // word-wise in the same orders.  Per-row scales: K's on the score, V's on p.
+  // swizzled byte tile gives each thread one 32-bit word (4 codes) per
+  // 8x16-byte matrix, converted in registers to f16 MMA operands.  For K the
+  // word holds 4 columns of one key, the A fragment under the permuted
+  // contraction order of q.  For V (.trans) it holds 2 keys x 2 columns; a
+  // byte permute regroups it into key pairs, and the rows of each 16-row
+  // block of O^T follow: row t <-> d = 16m + 2t, row t+8 <-> d = 16m + 2t + 1.
+  // Query-region stages hold bf16 rows, read word-wise in the same orders.
+  // Per-row scales: K's on the score, V's on p.
   auto fp8_stage = [&](const StageMeta& m, uint32_t kb, uint32_t vb, const uint8_t* sclp, int kw, int n) {
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float s[NG][4], s2[NG][4];
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nb][e] = s2[nb][e] = 0.f;
     const bool ctx8 = m.row0 >= 0;
-    const int t = lane >> 2, cq = lane & 3;
     const uint8_t* kp = smem + (kb - smem_u32(smem));
     const uint8_t* vp = kp + S::TILE;
     if (ctx8) {
@@ -412,38 +464,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4(kb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
-        mma_f16_16816(s[0], qa[2 * jp], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
-        mma_f16_16816(s[1], qa[2 * jp], e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
-        mma_f16_16816(s[0], qa[2 * jp + 1], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r2 >> 16));
-        mma_f16_16816(s[1], qa[2 * jp + 1], e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r3 >> 16));
+        const uint32_t af0[4] = {e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
+                                 e4m3x2_to_f16x2(r1 >> 16)};
+        const uint32_t af1[4] = {e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r2 >> 16),
+                                 e4m3x2_to_f16x2(r3 >> 16)};
+#pragma unroll
+        for (int nb = 0; nb < NG; ++nb) {
+          mma_f16_16816(s[nb], af0, qb[2 * jp][nb][0], qb[2 * jp][nb][1]);
+          mma_f16_16816(s2[nb], af1, qb[2 * jp + 1][nb][0], qb[2 * jp + 1][nb][1]);
+        }
       }
     } else {
 #pragma unroll
-      for (int kd = 0; kd < D / 16; ++kd)
+      for (int kd = 0; kd < D / 16; ++kd) {
+        const int r0 = kw + t4, r1 = r0 + 8;                    // < 64: kw < n <= 64
+        const int ch = 2 * (kd & 3) + (c4 >> 1);
+        const uint8_t* base = kp + (kd >> 2) * S::HALF64 + 8 * (c4 & 1);
+        const uint2 w0 = *reinterpret_cast<const uint2*>(base + r0 * 128 + ((ch ^ (r0 & 7)) << 4));
+        const uint2 w1 = *reinterpret_cast<const uint2*>(base + r1 * 128 + ((ch ^ (r1 & 7)) << 4));
+        const uint32_t af[4] = {bf16x2_to_f16x2(w0.x), bf16x2_to_f16x2(w1.x), bf16x2_to_f16x2(w0.y),
+                                bf16x2_to_f16x2(w1.y)};
 #pragma unroll
-        for (int nn = 0; nn < 2; ++nn) {
-          const int row = kw + 8 * nn + t;                       // < 64: kw < n <= 64
-          const int ch = 2 * (kd & 3) + (cq >> 1);
-          const uint2 w = *reinterpret_cast<const uint2*>(kp + (kd >> 2) * S::HALF64 + row * 128 +
-                                                          ((ch ^ (row & 7)) << 4) + 8 * (cq & 1));
-          mma_f16_16816(s[nn], qa[kd], bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y));
-        }
+        for (int nb = 0; nb < NG; ++nb)
+          mma_f16_16816((kd & 1) ? s2[nb] : s[nb], af, qb[kd][nb][0], qb[kd][nb][1]);
+      }
     }
-    const float* sks = reinterpret_cast<const float*>(sclp) + (ctx8 ? (m.row0 & 3) : 0);
-    const float* svs = reinterpret_cast<const float*>(sclp + S::SCL_SLOT) + (ctx8 ? (m.row0 & 3) : 0);
-    float sk[4], sv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int key = kw + (u >> 1) * 8 + 2 * cq + (u & 1);
-      sk[u] = ctx8 ? a.scale_log2 * sks[key] : a.scale_log2;
-      sv[u] = ctx8 ? svs[key] : 1.f;
-    }
-    softmax_update(s, sk, kw, n);
-    uint32_t pa[4];
-    pa[0] = pack_f16(s[0][0] * sv[0], s[0][1] * sv[1]);
-    pa[1] = pack_f16(s[0][2] * sv[0], s[0][3] * sv[1]);
-    pa[2] = pack_f16(s[1][0] * sv[2], s[1][1] * sv[3]);
-    pa[3] = pack_f16(s[1][2] * sv[2], s[1][3] * sv[3]);
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nb][e] += s2[nb][e];
+    const int so = ctx8 ? (m.row0 & 3) : 0;
+    const float* sks = reinterpret_cast<const float*>(sclp) + so;
+    const float* svs = reinterpret_cast<const float*>(sclp + S::SCL_SLOT) + so;
+    softmax_update(s, ctx8 ? a.scale_log2 * sks[kw + t4] : a.scale_log2,
+                   ctx8 ? a.scale_log2 * sks[kw + t4 + 8] : a.scale_log2, kw, n);
+    uint32_t pb[NG][2];
+    p_fragments(s, ctx8 ? svs[kw + t4] : 1.f, ctx8 ? svs[kw + t4 + 8] : 1.f, pb);
     if (ctx8) {
 #pragma unroll
       for (int jp = 0; jp < D / 32; ++jp) {
@@ -451,30 +507,37 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4_trans(vb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
         // r0: keys 2c, 2c+1 x columns 2t, 2t+1 of chunk 2jp; r1: keys 2c+8, 2c+9;
-        // r2, r3: the same of chunk 2jp+1.  Regroup to (key pair) per column.
+        // r2, r3: the same of chunk 2jp+1.  Regroup to key pairs per column.
         const uint32_t p0 = __byte_perm(r0, 0u, 0x3120), p1 = __byte_perm(r1, 0u, 0x3120);
         const uint32_t p2 = __byte_perm(r2, 0u, 0x3120), p3 = __byte_perm(r3, 0u, 0x3120);
-        mma_f16_16816(o[4 * jp], pa, e4m3x2_to_f16x2(p0), e4m3x2_to_f16x2(p1));
-        mma_f16_16816(o[4 * jp + 1], pa, e4m3x2_to_f16x2(p0 >> 16), e4m3x2_to_f16x2(p1 >> 16));
-        mma_f16_16816(o[4 * jp + 2], pa, e4m3x2_to_f16x2(p2), e4m3x2_to_f16x2(p3));
-        mma_f16_16816(o[4 * jp + 3], pa, e4m3x2_to_f16x2(p2 >> 16), e4m3x2_to_f16x2(p3 >> 16));
+        const uint32_t af0[4] = {e4m3x2_to_f16x2(p0), e4m3x2_to_f16x2(p0 >> 16), e4m3x2_to_f16x2(p1),
+                                 e4m3x2_to_f16x2(p1 >> 16)};
+        const uint32_t af1[4] = {e4m3x2_to_f16x2(p2), e4m3x2_to_f16x2(p2 >> 16), e4m3x2_to_f16x2(p3),
+                                 e4m3x2_to_f16x2(p3 >> 16)};
+#pragma unroll
+        for (int nb = 0; nb < NG; ++nb) {
+          mma_f16_16816(oT[2 * jp][nb], af0, pb[nb][0], pb[nb][1]);
+          mma_f16_16816(oT[2 * jp + 1][nb], af1, pb[nb][0], pb[nb][1]);
+        }
       }
     } else {
 #pragma unroll
-      for (int ch = 0; ch < D / 16; ++ch) {
-        const int cc = 2 * (ch & 3) + (t >> 2), by = 4 * (t & 3);
+      for (int mb = 0; mb < D / 16; ++mb) {
+        const int cc = 2 * (mb & 3) + (t4 >> 2), by = 4 * (t4 & 3);
         uint32_t w[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int kk = kw + 2 * cq + (q4 & 1) + 8 * (q4 >> 1);   // < 64
-          w[q4] = kk < n ? *reinterpret_cast<const uint32_t*>(vp + (ch >> 2) * S::HALF64 + kk * 128 +
+          const int kk = kw + 2 * c4 + (q4 & 1) + 8 * (q4 >> 1);   // < 64
+          w[q4] = kk < n ? *reinterpret_cast<const uint32_t*>(vp + (mb >> 2) * S::HALF64 + kk * 128 +
                                                               ((cc ^ (kk & 7)) << 4) + by)
                          : 0u;
         }
-        mma_f16_16816(o[2 * ch], pa, bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x5410)),
-                      bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x5410)));
-        mma_f16_16816(o[2 * ch + 1], pa, bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x7632)),
-                      bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x7632)));
+        const uint32_t af[4] = {bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x5410)),
+                                bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x7632)),
+                                bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x5410)),
+                                bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x7632))};
+#pragma unroll
+        for (int nb = 0; nb < NG; ++nb) mma_f16_16816(oT[mb][nb], af, pb[nb][0], pb[nb][1]);
       }
     }
   };
@@ -496,7 +559,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       const uint32_t kb = smem_u32(smem + slot * S::STAGE);
       const uint32_t vb = kb + S::TILE;
       const int kw = 16 * cw;   // first key of this warp in the stage
-      if (FP8 ? kw < n : true) {   // (FP8 mode: a warp past the valid keys adds nothing)
+      if (kw < n) {   // a warp past the stage's valid keys adds nothing
         if constexpr (FP8) fp8_stage(m, kb, vb, scl + slot * 2 * S::SCL_SLOT, kw, n);
         else bf16_stage(kb, vb, kw, n, slot);
       }
@@ -513,10 +576,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     const bool owns_new = (int)blockIdx.x == lastc;          // holds the piece's last cached row
     const int pslot = (int)blockIdx.x - first;
     const int count = lastc - first + 1;
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+#pragma unroll
+    for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = ls[nb][e];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        ls[nb][e] = v;
+      }
+    if (t4 == 0) {
+#pragma unroll
+      for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          wm[cw][8 * nb + 2 * c4 + e] = mx[nb][e];
+          wl[cw][8 * nb + 2 * c4 + e] = ls[nb][e];
+        }
+    }
     if (owns_new) {
       // score of the new token for every head of the group (warp r: head r)
       const bf16* kn = a.k + (long long)bg * D;
@@ -529,28 +607,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         if (lane == 0) s_new[r] = acc * a.scale_log2;
       }
     }
-    for (int rh = 0; rh < G; rh += 4) {            // rows rh .. rh+3 per round
-      const int ra = lane >> 2, rb = ra + 8;       // fragment rows of this thread
-      if ((lane & 3) == 0) {
-        wm[cw][ra] = m_a;
-        wm[cw][rb] = m_b;
-        wl[cw][ra] = l_a;
-        wl[cw][rb] = l_b;
-      }
+    for (int rh = 0; rh < G; rh += 4) {            // heads rh .. rh+3 per round
 #pragma unroll
-      for (int nn = 0; nn < NT_O; ++nn) {
-        // columns of accumulator block nn held by this thread (FP8 mode: permuted)
-        const int c0 = FP8 ? 16 * (nn >> 1) + 4 * (lane & 3) + (nn & 1) : 8 * nn + 2 * (lane & 3);
-        const int c1 = FP8 ? c0 + 2 : c0 + 1;
-        if (ra >= rh && ra < rh + 4) {
-          comb[(cw * 4 + ra - rh) * D + c0] = o[nn][0];
-          comb[(cw * 4 + ra - rh) * D + c1] = o[nn][1];
-        }
-        if (rb >= rh && rb < rh + 4) {
-          comb[(cw * 4 + rb - rh) * D + c0] = o[nn][2];
-          comb[(cw * 4 + rb - rh) * D + c1] = o[nn][3];
-        }
-      }
+      for (int mb = 0; mb < D / 16; ++mb)
+#pragma unroll
+        for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = 8 * nb + 2 * c4 + e;
+            // rows t, t+8 of O^T block mb (FP8 mode: permuted, see fp8_stage)
+            const int d0 = FP8 ? 16 * mb + 2 * t4 : 16 * mb + t4;
+            const int d1 = FP8 ? d0 + 1 : d0 + 8;
+            if (h >= rh && h < rh + 4) {
+              comb[(cw * 4 + h - rh) * D + d0] = oT[mb][nb][e];
+              comb[(cw * 4 + h - rh) * D + d1] = oT[mb][nb][2 + e];
+            }
+          }
       named_sync(1, 32 * NCW);
       const int rows = G - rh < 4 ? G - rh : 4;
       for (int idx = ctid; idx < rows * D; idx += 32 * NCW) {
@@ -715,14 +787,26 @@ const char* decode_make_maps(const CacheView& c, DecodeMaps* m) {
 
 template <int D, bool FP8>
 cudaError_t decode_prepare_one() {
-  return cudaFuncSetAttribute(decode_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              DSmem<D, FP8>::BYTES + 1024);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, FP8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DSmem<D, FP8>::BYTES + 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_kernel<D, FP8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             DSmem<D, FP8>::BYTES + 1024);
+  return e;
 }
 
 cudaError_t decode_prepare(int D) {
   cudaError_t e = D == 128 ? decode_prepare_one<128, false>() : decode_prepare_one<64, false>();
   if (e == cudaSuccess) e = D == 128 ? decode_prepare_one<128, true>() : decode_prepare_one<64, true>();
   return e;
+}
+
+template <int D, bool FP8>
+void launch_decode_kernel(const DecodeArgs& a, int G, int ncta, cudaStream_t st) {
+  if (G <= 8)
+    decode_kernel<D, FP8, 1><<<ncta, NTHREADS, DSmem<D, FP8>::BYTES + 1024, st>>>(a);
+  else
+    decode_kernel<D, FP8, 2><<<ncta, NTHREADS, DSmem<D, FP8>::BYTES + 1024, st>>>(a);
 }
 
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
@@ -756,13 +840,13 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.err = s.err;
   const bool fp8 = c.ctxK8 != nullptr;
   if (c.D == 128 && fp8)
-    decode_kernel<128, true><<<plan.ncta, NTHREADS, DSmem<128, true>::BYTES + 1024, st>>>(a);
+    launch_decode_kernel<128, true>(a, c.G, plan.ncta, st);
   else if (c.D == 128)
-    decode_kernel<128, false><<<plan.ncta, NTHREADS, DSmem<128, false>::BYTES + 1024, st>>>(a);
+    launch_decode_kernel<128, false>(a, c.G, plan.ncta, st);
   else if (fp8)
-    decode_kernel<64, true><<<plan.ncta, NTHREADS, DSmem<64, true>::BYTES + 1024, st>>>(a);
+    launch_decode_kernel<64, true>(a, c.G, plan.ncta, st);
   else
-    decode_kernel<64, false><<<plan.ncta, NTHREADS, DSmem<64, false>::BYTES + 1024, st>>>(a);
+    launch_decode_kernel<64, false>(a, c.G, plan.ncta, st);
   return cudaGetLastError();
 }
 

@@ -107,13 +107,14 @@ class StarCache:
         return out[0], out[1], seg
 
     def segment_fp8_tensors(self, i: int):
-        """FP8 copy of context segment ``i`` (``kv_fp8`` caches): E4M3 codes of K
-        and V as uint8 [B, Hkv, len, D] and their float32 row scales [B, Hkv, len]."""
+        """FP8 copy of segment ``i`` (``kv_fp8`` caches; ``i = num_segments - 1`` is
+        the query region): E4M3 codes of K and V as uint8 [B, Hkv, cap, D] and
+        their float32 row scales [B, Hkv, cap]."""
         k8, v8 = ctypes.c_void_p(), ctypes.c_void_p()
         ks, vs = ctypes.POINTER(ctypes.c_float)(), ctypes.POINTER(ctypes.c_float)()
         _abi.check(self.lib.star_cache_segment_fp8(self.handle, i, ctypes.byref(k8), ctypes.byref(v8),
                                                    ctypes.byref(ks), ctypes.byref(vs)))
-        n = self.segment(i).len
+        n = self.segment(i).cap
         shape = (self.B, self.Hkv, n)
         codes = [_view_from_ptr(p, self.B * self.Hkv * n * self.D, "|u1", self.device)
                  .view(*shape, self.D) for p in (k8.value, v8.value)]

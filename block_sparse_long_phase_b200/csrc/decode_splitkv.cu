@@ -25,12 +25,14 @@
 // another -- merges that head's partials and writes o and lse.
 #include <cuda_bf16.h>
 #include <stdio.h>
+#include <algorithm>
 #include <math.h>
 #include <string.h>
 
 #include <mutex>
 
 #include "../../include/star_attention.h"
+#include "fp8_row.cuh"
 #include "sm100_primitives.cuh"
 #include "star_common.cuh"
 #include "star_internal.h"
@@ -41,7 +43,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int KS = 128;                 // keys per stage
+constexpr int KS = 128;                 // keys per bf16 stage (16 per consumer warp)
+constexpr int KS8 = 256;                // keys per FP8 context stage (32 per consumer warp)
 constexpr int NSTAGE = 3;
 constexpr int NCW = 8;                  // consumer warps
 constexpr int NTHREADS = 32 * (NCW + 1);
@@ -49,17 +52,20 @@ constexpr int kMaxG = 16;
 
 struct StageMeta {
   int n;         // valid keys in the stage
-  int last;      // 1: the stage ends a (batch, kv head) piece of this span
   int bg;        // batch * Hkv + kv head
-  int row0;      // FP8 context stage: its first row in the context cache; else -1
+  int row0;      // first row of the stage in its region's cache (FP8: picks the scales)
+  int flush;     // 1: before this stage, flush the previous run (fbg, fslot, frows)
+  int end;       // 1: terminal stage (no keys): the CTA's work is done
+  int fbg, fslot, frows;
 };
 
 struct DecodeArgs {
   CUtensorMap tk_ctx, tv_ctx;   // context cache as [B*Hkv*L][D]
   CUtensorMap tk_q, tv_q;       // query region as [B*Hkv*q_cap][D]
-  CUtensorMap tk8, tv8;         // FP8 context cache as [B*Hkv*L][D] bytes
-  CUtensorMap tkq64, tvq64;     // query region in 64-row boxes (FP8 mode)
-  CUtensorMap tks, tvs;         // FP8 row scales: one row of B*Hkv*L float32
+  CUtensorMap tk8, tv8;         // FP8 context cache as [B*Hkv*L][D] bytes, 256-row boxes
+  CUtensorMap tkq8, tvq8;       // FP8 query region as [B*Hkv*q_cap][D] bytes
+  CUtensorMap tks, tvs;         // FP8 row scales as [ceil(B*Hkv*L / 4)][4] float32
+  CUtensorMap tkqs, tvqs;       // ... of the query region, [ceil(B*Hkv*q_cap / 4)][4]
   CacheView c;
   float scale_log2;
   int len0;                     // query-region rows before this step
@@ -73,14 +79,14 @@ struct DecodeArgs {
   float* lse;                   // [B][Hq]
   float* partA;                 // [B*Hkv][maxp][G][D]
   float* partS;                 // [B*Hkv][maxp][G]
-  unsigned* tickets;            // [B*Hkv]
+  unsigned* tickets;            // [B*Hkv] rows folded into parts (kept at 0 between steps)
   int* err;
 };
 
 __device__ __forceinline__ long long span_start(long long i, long long R, int n) {
   return i * R / n;
 }
-// CTA whose span holds global cached row x (largest i with span_start(i) <= x).
+// CTA whose span holds row x (largest i with span_start(i) <= x).
 __device__ __forceinline__ int cta_of(long long x, long long R, int n) {
   return (int)(((x + 1) * n - 1) / R);
 }
@@ -98,17 +104,16 @@ SM100_DEV void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"
 template <int D, bool FP8 = false>
 struct DSmem {
   static constexpr int HALF = KS * 128;               // one 64-column half of a bf16 stage tile
-  static constexpr int HALF64 = 64 * 128;             // ... of a 64-row bf16 tile (FP8 mode)
-  // K (or V) of one stage: 128 rows of bf16, or in FP8 mode 128 rows of E4M3
-  // codes (128- or 64-byte swizzled) / 64 query-region rows of bf16
-  static constexpr int TILE = FP8 ? KS * D : KS * D * 2;
+  // K (or V) of one stage: 128 rows of bf16, or in FP8 mode 256 rows of E4M3
+  // codes (128- or 64-byte swizzled)
+  static constexpr int TILE = FP8 ? KS8 * D : KS * D * 2;
   static constexpr int STAGE = 2 * TILE;
-  static constexpr int NST = FP8 ? 6 : NSTAGE;
-  // FP8 row scales of a stage: a box of 132 floats starting at the 4-aligned
-  // row at or below the stage's first row
-  static constexpr int SCL_BOX = KS + 4;
-  static constexpr int SCL_BYTES = SCL_BOX * 4;
-  static constexpr int SCL_SLOT = 640;
+  static constexpr int NST = FP8 ? (D == 128 ? 3 : 6) : NSTAGE;
+  // FP8 row scales of a stage: 65 groups of 4 floats starting at the group
+  // that holds the stage's first row (260 rows >= 256 + 3)
+  static constexpr int SCL_QUADS = KS8 / 4 + 1;
+  static constexpr int SCL_BYTES = SCL_QUADS * 16;
+  static constexpr int SCL_SLOT = 1152;
   static constexpr int SCL = FP8 ? NST * 2 * SCL_SLOT : 0;
   // 4 rows of O per warp per round; also holds the merge weights (<= 16 x 160)
   static constexpr int COMB = NCW * 4 * 128 * 4;
@@ -165,14 +170,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   __shared__ float wm[NCW][16], wl[NCW][16];
   __shared__ float s_new[kMaxG];
   __shared__ float s_lse[kMaxG];
-  __shared__ int s_last, abort_s;
+  __shared__ int s_last, abort_s, cons_abort;
 
   const CacheView& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = c.G;
-  const long long R = (long long)c.B * c.Hkv * a.rpb;
-  const long long x0 = span_start(blockIdx.x, R, a.ncta);
-  const long long x1 = span_start(blockIdx.x + 1, R, a.ncta);
 
   if (tid == 0) {
     for (int i = 0; i < S::NST; ++i) {
@@ -180,6 +182,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       mbar_init(smem_u32(&bar_empty[i]), NCW);
     }
     abort_s = 0;
+    cons_abort = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -191,6 +194,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
+    // The CTA's span of the cached rows (all (batch, kv head) pairs bg laid end
+    // to end, bg-major) is cut into runs of one bg each.  A run's partial is
+    // flushed at the first stage of the next run (or at the terminal stage),
+    // whose meta carries the run's bg, partial slot and row count.
     if (elect_one()) {
       prefetch_tmap(&a.tk_ctx);
       prefetch_tmap(&a.tv_ctx);
@@ -199,56 +206,82 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       if (FP8) {
         prefetch_tmap(&a.tk8);
         prefetch_tmap(&a.tv8);
-        prefetch_tmap(&a.tkq64);
-        prefetch_tmap(&a.tvq64);
+        prefetch_tmap(&a.tkq8);
+        prefetch_tmap(&a.tvq8);
         prefetch_tmap(&a.tks);
         prefetch_tmap(&a.tvs);
+        prefetch_tmap(&a.tkqs);
+        prefetch_tmap(&a.tvqs);
       }
+      const long long R = (long long)c.B * c.Hkv * a.rpb;
+      long long x = span_start(blockIdx.x, R, a.ncta);
+      const long long x1 = span_start(blockIdx.x + 1, R, a.ncta);
       int last_use[S::NST];
       for (int k = 0; k < S::NST; ++k) last_use[k] = -1;
-      long long x = x0;
-      for (int st = 0; x < x1; ++st) {
-        const int bg = (int)(x / a.rpb);
-        const long long off = x - (long long)bg * a.rpb;           // key index within (b, g)
-        const long long piece_end = ((long long)bg + 1) * a.rpb < x1 ? ((long long)bg + 1) * a.rpb : x1;
-        long long region_end;
-        int row;
-        bool ctx;
-        if (off < c.L) {
-          const int seg = (int)(off / c.b);
-          const long long len = seg_len(c, seg);
-          region_end = (long long)seg * c.b + len;
-          row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * len + (off - (long long)seg * c.b));
-          ctx = true;
-        } else {
-          region_end = a.rpb;
-          row = (int)((long long)bg * c.q_cap + (off - c.L));
-          ctx = false;
-        }
-        long long n = (FP8 && !ctx) ? 64 : KS;
-        if (region_end - off < n) n = region_end - off;
-        if (piece_end - x < n) n = piece_end - x;
-        const int slot = st % S::NST, use = st / S::NST;
-        if (use > 0 && !mbar_wait(smem_u32(&bar_empty[slot]), (use - 1) & 1)) { fail(); break; }
-        if (aborted()) break;
-        meta[slot].n = (int)n;
-        meta[slot].last = (x + n == piece_end) ? 1 : 0;
-        meta[slot].bg = bg;
-        meta[slot].row0 = (FP8 && ctx) ? row : -1;
-        const uint32_t fb = smem_u32(&bar_full[slot]);
-        mbar_arrive_expect_tx(fb, (FP8 && ctx) ? S::STAGE + 2 * S::SCL_BYTES : S::STAGE);
-        const uint32_t dst = smem_u32(smem + slot * S::STAGE);
-        if (FP8 && ctx) {
-          tma_load_2d(dst, &a.tk8, 0, row, fb);
-          tma_load_2d(dst + S::TILE, &a.tv8, 0, row, fb);
-          const uint32_t sd = smem_u32(scl + slot * 2 * S::SCL_SLOT);
-          tma_load_2d(sd, &a.tks, row & ~3, 0, fb);
-          tma_load_2d(sd + S::SCL_SLOT, &a.tvs, row & ~3, 0, fb);
-        } else if (FP8) {
-          for (int hf = 0; hf < NH; ++hf) {
-            tma_load_2d(dst + hf * S::HALF64, &a.tkq64, hf * 64, row, fb);
-            tma_load_2d(dst + S::TILE + hf * S::HALF64, &a.tvq64, hf * 64, row, fb);
+      int run_bg = -1, run_slot = 0, run_rows = 0;
+      bool broke = false;
+      for (int st = 0;; ++st) {
+        const bool have = x < x1;
+        int bg = -1, row = 0;
+        long long n = 0;
+        bool ctx = false;
+        if (have) {
+          bg = (int)(x / a.rpb);
+          const long long off = x - (long long)bg * a.rpb;         // key index within bg
+          const long long run_end = ((long long)bg + 1) * a.rpb < x1 ? ((long long)bg + 1) * a.rpb : x1;
+          long long region_end;
+          if (off < c.L) {
+            const int seg = (int)(off / c.b);
+            const long long len = seg_len(c, seg);
+            region_end = (long long)seg * c.b + len;
+            row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * len + (off - (long long)seg * c.b));
+            ctx = true;
+          } else {
+            region_end = a.rpb;
+            row = (int)((long long)bg * c.q_cap + (off - c.L));
           }
+          n = FP8 ? KS8 : KS;
+          if (region_end - off < n) n = region_end - off;
+          if (run_end - x < n) n = run_end - x;
+        }
+        const int slot = st % S::NST, use = st / S::NST;
+        if (use > 0 && !mbar_wait(smem_u32(&bar_empty[slot]), (use - 1) & 1)) {
+          fail();
+          broke = true;
+          break;
+        }
+        if (aborted()) {
+          broke = true;
+          break;
+        }
+        const bool new_run = !have || bg != run_bg;
+        StageMeta& md = meta[slot];
+        md.n = (int)n;
+        md.bg = bg;
+        md.row0 = row;
+        md.flush = (new_run && run_bg >= 0) ? 1 : 0;
+        md.end = have ? 0 : 1;
+        md.fbg = run_bg;
+        md.fslot = run_slot;
+        md.frows = run_rows;
+        const uint32_t fb = smem_u32(&bar_full[slot]);
+        if (!have) {
+          mbar_arrive(fb);                          // terminal stage: meta only
+          break;
+        }
+        if (new_run) {
+          run_bg = bg;
+          run_slot = (int)blockIdx.x - cta_of((long long)bg * a.rpb, R, a.ncta);   // rank among bg's CTAs
+          run_rows = 0;
+        }
+        mbar_arrive_expect_tx(fb, FP8 ? S::STAGE + 2 * S::SCL_BYTES : S::STAGE);
+        const uint32_t dst = smem_u32(smem + slot * S::STAGE);
+        if (FP8) {
+          const uint32_t sd = smem_u32(scl + slot * 2 * S::SCL_SLOT);
+          tma_load_2d(dst, ctx ? &a.tk8 : &a.tkq8, 0, row, fb);
+          tma_load_2d(dst + S::TILE, ctx ? &a.tv8 : &a.tvq8, 0, row, fb);
+          tma_load_2d(sd, ctx ? &a.tks : &a.tkqs, 0, row >> 2, fb);
+          tma_load_2d(sd + S::SCL_SLOT, ctx ? &a.tvs : &a.tvqs, 0, row >> 2, fb);
         } else {
           for (int hf = 0; hf < NH; ++hf) {
             tma_load_2d(dst + hf * S::HALF, ctx ? &a.tk_ctx : &a.tk_q, hf * 64, row, fb);
@@ -257,8 +290,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         }
         last_use[slot] = use;
         x += n;
+        run_rows += (int)n;
       }
-      if (aborted())
+      if (broke)
         for (int k = 0; k < S::NST; ++k)
           if (last_use[k] >= 0) mbar_wait(smem_u32(&bar_full[k]), last_use[k] & 1);
     }
@@ -273,6 +307,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   // Thread (t = lane/4, c = lane%4) holds, per head block nb, the heads
   // g = 8nb + 2c + e (e = 0, 1): scores of keys t and t+8, O^T rows t and t+8
   // of each 16-row block of d, and the running max / sum of those heads.
+  constexpr int SL = FP8 ? 2 : 1;                // slices of 16 keys per warp and stage
+  constexpr int KPW = 16 * SL;                   // keys per warp and stage
   const int cw = warp - 1;                       // consumer warp 0..7
   const int ctid = tid - 32;                     // 0..255
   const int t4 = lane >> 2, c4 = lane & 3;
@@ -320,16 +356,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   };
   reset_state();
 
-  // Scale and mask the scores (sk0, sk1: factor on the log2 scale of keys t
-  // and t+8), update the running max / sum per head, turn scores into p.
-  auto softmax_update = [&](float (&s)[NG][4], float sk0, float sk1, int kw, int n) {
-    const bool v0 = kw + t4 < n, v1 = kw + t4 + 8 < n;
+  // Scale and mask the scores of the warp's SL slices of 16 keys (sk[sl][0/1]:
+  // factor on the log2 scale of keys kw + 16 sl + t and + t + 8), update the
+  // running max / sum per head, turn scores into p.
+  auto softmax_update = [&](float (&s)[SL][NG][4], const float (&sk)[SL][2], int kw, int n) {
 #pragma unroll
-    for (int nb = 0; nb < NG; ++nb) {
-      s[nb][0] = v0 ? s[nb][0] * sk0 : -INFINITY;
-      s[nb][1] = v0 ? s[nb][1] * sk0 : -INFINITY;
-      s[nb][2] = v1 ? s[nb][2] * sk1 : -INFINITY;
-      s[nb][3] = v1 ? s[nb][3] * sk1 : -INFINITY;
+    for (int sl = 0; sl < SL; ++sl) {
+      const bool v0 = kw + 16 * sl + t4 < n, v1 = kw + 16 * sl + t4 + 8 < n;
+#pragma unroll
+      for (int nb = 0; nb < NG; ++nb) {
+        s[sl][nb][0] = v0 ? s[sl][nb][0] * sk[sl][0] : -INFINITY;
+        s[sl][nb][1] = v0 ? s[sl][nb][1] * sk[sl][0] : -INFINITY;
+        s[sl][nb][2] = v1 ? s[sl][nb][2] * sk[sl][1] : -INFINITY;
+        s[sl][nb][3] = v1 ? s[sl][nb][3] * sk[sl][1] : -INFINITY;
+      }
     }
     float mn[NG][2];
     bool up = false;
@@ -337,7 +377,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     for (int nb = 0; nb < NG; ++nb)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float v = fmaxf(s[nb][e], s[nb][2 + e]);
+        float v = fmaxf(s[0][nb][e], s[0][nb][2 + e]);
+#pragma unroll
+        for (int sl = 1; sl < SL; ++sl) v = fmaxf(v, fmaxf(s[sl][nb][e], s[sl][nb][2 + e]));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
         v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
@@ -367,9 +409,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const float base = mx[nb][e] == -INFINITY ? 0.f : mx[nb][e];
-        s[nb][e] = exp2f(s[nb][e] - base);
-        s[nb][2 + e] = exp2f(s[nb][2 + e] - base);
-        ls[nb][e] += s[nb][e] + s[nb][2 + e];
+#pragma unroll
+        for (int sl = 0; sl < SL; ++sl) {
+          s[sl][nb][e] = exp2f(s[sl][nb][e] - base);
+          s[sl][nb][2 + e] = exp2f(s[sl][nb][2 + e] - base);
+          ls[nb][e] += s[sl][nb][e] + s[sl][nb][2 + e];
+        }
       }
   };
 
@@ -389,11 +434,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   // One stage of bf16 keys: K and V fragments straight from the
   // 128-byte-swizzled TMA tiles.
   auto bf16_stage = [&](uint32_t kb, uint32_t vb, int kw, int n, int slot) {
-    float s[NG][4], s2[NG][4];                   // even / odd column steps: two short chains
+    float s[SL][NG][4], s2[NG][4];               // even / odd column steps: two short chains
 #pragma unroll
     for (int nb = 0; nb < NG; ++nb)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nb][e] = s2[nb][e] = 0.f;
+      for (int e = 0; e < 4; ++e) s[0][nb][e] = s2[nb][e] = 0.f;
 #pragma unroll
     for (int kd = 0; kd < D / 16; ++kd) {
       uint32_t af[4];
@@ -403,13 +448,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
                   af[3]);
 #pragma unroll
       for (int nb = 0; nb < NG; ++nb)
-        mma_bf16_16816((kd & 1) ? s2[nb] : s[nb], af, qb[kd][nb][0], qb[kd][nb][1]);
+        mma_bf16_16816((kd & 1) ? s2[nb] : s[0][nb], af, qb[kd][nb][0], qb[kd][nb][1]);
     }
 #pragma unroll
     for (int nb = 0; nb < NG; ++nb)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nb][e] += s2[nb][e];
-    softmax_update(s, a.scale_log2, a.scale_log2, kw, n);
+      for (int e = 0; e < 4; ++e) s[0][nb][e] += s2[nb][e];
+    float sk[SL][2];
+#pragma unroll
+    for (int sl = 0; sl < SL; ++sl) sk[sl][0] = sk[sl][1] = a.scale_log2;
+    softmax_update(s, sk, kw, n);
     if (kw + 16 > n) {
       // Keys past the stage's valid count carry p = 0, but 0 * NaN is NaN:
       // clear this warp's V rows there (bytes past the end of a buffer need
@@ -425,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       __syncwarp();
     }
     uint32_t pb[NG][2];
-    p_fragments(s, 1.f, 1.f, pb);
+    p_fragments(s[0], 1.f, 1.f, pb);
 #pragma unroll
     for (int m = 0; m < D / 16; ++m) {
       uint32_t af[4];
@@ -440,28 +488,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     if (kw + 16 > n) fence_proxy_async_smem();
   };
 
-  // One stage in FP8 mode.  Context stages hold E4M3 codes: ldmatrix on the
-  // swizzled byte tile gives each thread one 32-bit word (4 codes) per
-  // 8x16-byte matrix, converted in registers to f16 MMA operands.  For K the
-  // word holds 4 columns of one key, the A fragment under the permuted
-  // contraction order of q.  For V (.trans) it holds 2 keys x 2 columns; a
-  // byte permute regroups it into key pairs, and the rows of each 16-row
-  // block of O^T follow: row t <-> d = 16m + 2t, row t+8 <-> d = 16m + 2t + 1.
-  // Query-region stages hold bf16 rows, read word-wise in the same orders.
-  // Per-row scales: K's on the score, V's on p.
+  // One stage in FP8 mode (context segments and query region alike); each
+  // warp takes SL = 2 slices of 16 keys (kw + 16 sl ...), whose softmax shares
+  // one reduction.  ldmatrix on the swizzled byte tile gives each thread one
+  // 32-bit word (4 codes) per 8x16-byte matrix, converted in registers to f16
+  // MMA operands.  For K the word holds 4 columns of one key, the A fragment
+  // under the permuted contraction order of q.  For V (.trans) it holds 2 keys
+  // x 2 columns; a byte permute regroups it into key pairs, and the rows of
+  // each 16-row block of O^T follow: row t <-> d = 16m + 2t, row t+8 <->
+  // d = 16m + 2t + 1.  Per-row scales: K's on the score, V's on p.
   auto fp8_stage = [&](const StageMeta& m, uint32_t kb, uint32_t vb, const uint8_t* sclp, int kw, int n) {
-    float s[NG][4], s2[NG][4];
+    float s[SL][NG][4], s2[SL][NG][4];
 #pragma unroll
-    for (int nb = 0; nb < NG; ++nb)
+    for (int sl = 0; sl < SL; ++sl)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nb][e] = s2[nb][e] = 0.f;
-    const bool ctx8 = m.row0 >= 0;
-    const uint8_t* kp = smem + (kb - smem_u32(smem));
-    const uint8_t* vp = kp + S::TILE;
-    if (ctx8) {
+      for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[sl][nb][e] = s2[sl][nb][e] = 0.f;
+#pragma unroll
+    for (int sl = 0; sl < SL; ++sl) {
+      const int k0 = kw + 16 * sl;
 #pragma unroll
       for (int jp = 0; jp < D / 32; ++jp) {
-        const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4(kb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
         const uint32_t af0[4] = {e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r0 >> 16),
@@ -470,40 +519,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
                                  e4m3x2_to_f16x2(r3 >> 16)};
 #pragma unroll
         for (int nb = 0; nb < NG; ++nb) {
-          mma_f16_16816(s[nb], af0, qb[2 * jp][nb][0], qb[2 * jp][nb][1]);
-          mma_f16_16816(s2[nb], af1, qb[2 * jp + 1][nb][0], qb[2 * jp + 1][nb][1]);
+          mma_f16_16816(s[sl][nb], af0, qb[2 * jp][nb][0], qb[2 * jp][nb][1]);
+          mma_f16_16816(s2[sl][nb], af1, qb[2 * jp + 1][nb][0], qb[2 * jp + 1][nb][1]);
         }
-      }
-    } else {
-#pragma unroll
-      for (int kd = 0; kd < D / 16; ++kd) {
-        const int r0 = kw + t4, r1 = r0 + 8;                    // < 64: kw < n <= 64
-        const int ch = 2 * (kd & 3) + (c4 >> 1);
-        const uint8_t* base = kp + (kd >> 2) * S::HALF64 + 8 * (c4 & 1);
-        const uint2 w0 = *reinterpret_cast<const uint2*>(base + r0 * 128 + ((ch ^ (r0 & 7)) << 4));
-        const uint2 w1 = *reinterpret_cast<const uint2*>(base + r1 * 128 + ((ch ^ (r1 & 7)) << 4));
-        const uint32_t af[4] = {bf16x2_to_f16x2(w0.x), bf16x2_to_f16x2(w1.x), bf16x2_to_f16x2(w0.y),
-                                bf16x2_to_f16x2(w1.y)};
-#pragma unroll
-        for (int nb = 0; nb < NG; ++nb)
-          mma_f16_16816((kd & 1) ? s2[nb] : s[nb], af, qb[kd][nb][0], qb[kd][nb][1]);
       }
     }
 #pragma unroll
-    for (int nb = 0; nb < NG; ++nb)
+    for (int sl = 0; sl < SL; ++sl)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[nb][e] += s2[nb][e];
-    const int so = ctx8 ? (m.row0 & 3) : 0;
-    const float* sks = reinterpret_cast<const float*>(sclp) + so;
-    const float* svs = reinterpret_cast<const float*>(sclp + S::SCL_SLOT) + so;
-    softmax_update(s, ctx8 ? a.scale_log2 * sks[kw + t4] : a.scale_log2,
-                   ctx8 ? a.scale_log2 * sks[kw + t4 + 8] : a.scale_log2, kw, n);
-    uint32_t pb[NG][2];
-    p_fragments(s, ctx8 ? svs[kw + t4] : 1.f, ctx8 ? svs[kw + t4 + 8] : 1.f, pb);
-    if (ctx8) {
+      for (int nb = 0; nb < NG; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[sl][nb][e] += s2[sl][nb][e];
+    // scales: a box of 4-row groups from the group holding row0
+    const float* sks = reinterpret_cast<const float*>(sclp) + (m.row0 & 3);
+    const float* svs = reinterpret_cast<const float*>(sclp + S::SCL_SLOT) + (m.row0 & 3);
+    float sk[SL][2];
+#pragma unroll
+    for (int sl = 0; sl < SL; ++sl) {
+      const int k0 = kw + 16 * sl + t4;
+      sk[sl][0] = a.scale_log2 * sks[k0];
+      sk[sl][1] = a.scale_log2 * sks[k0 + 8];
+    }
+    softmax_update(s, sk, kw, n);
+#pragma unroll
+    for (int sl = 0; sl < SL; ++sl) {
+      const int k0 = kw + 16 * sl;
+      uint32_t pb[NG][2];
+      p_fragments(s[sl], svs[k0 + t4], svs[k0 + t4 + 8], pb);
 #pragma unroll
       for (int jp = 0; jp < D / 32; ++jp) {
-        const int row = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int row = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
         uint32_t r0, r1, r2, r3;
         ldmatrix_x4_trans(vb + sw8<D>(row, 2 * jp + (lane >> 4)), r0, r1, r2, r3);
         // r0: keys 2c, 2c+1 x columns 2t, 2t+1 of chunk 2jp; r1: keys 2c+8, 2c+9;
@@ -520,62 +565,118 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           mma_f16_16816(oT[2 * jp + 1][nb], af1, pb[nb][0], pb[nb][1]);
         }
       }
-    } else {
-#pragma unroll
-      for (int mb = 0; mb < D / 16; ++mb) {
-        const int cc = 2 * (mb & 3) + (t4 >> 2), by = 4 * (t4 & 3);
-        uint32_t w[4];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int kk = kw + 2 * c4 + (q4 & 1) + 8 * (q4 >> 1);   // < 64
-          w[q4] = kk < n ? *reinterpret_cast<const uint32_t*>(vp + (mb >> 2) * S::HALF64 + kk * 128 +
-                                                              ((cc ^ (kk & 7)) << 4) + by)
-                         : 0u;
-        }
-        const uint32_t af[4] = {bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x5410)),
-                                bf16x2_to_f16x2(__byte_perm(w[0], w[1], 0x7632)),
-                                bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x5410)),
-                                bf16x2_to_f16x2(__byte_perm(w[2], w[3], 0x7632))};
-#pragma unroll
-        for (int nb = 0; nb < NG; ++nb) mma_f16_16816(oT[mb][nb], af, pb[nb][0], pb[nb][1]);
-      }
     }
   };
 
-  long long x = x0;
-  for (int st = 0; x < x1; ++st) {
-    const int slot = st % S::NST, use = st / S::NST;
-    bool ok = !aborted() && mbar_wait(smem_u32(&bar_full[slot]), use & 1);
-    if (!ok) fail();
-    const StageMeta m = meta[slot];
-    const int n = ok ? m.n : (int)(x1 - x < KS ? x1 - x : KS);
-    const int bg = ok ? m.bg : (int)(x / a.rpb);
-    const bool last = ok ? (m.last != 0) : true;
-    if (bg != cur_bg) {
-      load_q(bg);
-      cur_bg = bg;
-    }
-    if (ok) {
-      const uint32_t kb = smem_u32(smem + slot * S::STAGE);
-      const uint32_t vb = kb + S::TILE;
-      const int kw = 16 * cw;   // first key of this warp in the stage
-      if (kw < n) {   // a warp past the stage's valid keys adds nothing
-        if constexpr (FP8) fp8_stage(m, kb, vb, scl + slot * 2 * S::SCL_SLOT, kw, n);
-        else bf16_stage(kb, vb, kw, n, slot);
-      }
-      if (lane == 0) mbar_arrive(smem_u32(&bar_empty[slot]));
-    }
-    x += n;
-    if (!last) continue;
+  // [B*Hkv] rows of each (batch, kv head) folded into parts (the new token
+  // counts as one): the CTA that completes rpb + 1 rows merges
+  unsigned* const done = a.tickets;
+  const int newslot = a.maxp - 1;                 // the new token's part
 
-    // ---- piece epilogue: one partial (A, s) for (bg, this CTA) ---------------
+  // ---- merge of bg's parts: one per CTA whose span holds rows of bg (slots
+  // 0..nspan-1) and the new token (slot maxp-1) -----------------------------
+  auto merge_bg = [&](int bg) {
     const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
-    const long long first_row = (long long)bg * a.rpb;
-    const int first = cta_of(first_row, R, a.ncta);
-    const int lastc = cta_of(first_row + a.rpb - 1, R, a.ncta);
-    const bool owns_new = (int)blockIdx.x == lastc;          // holds the piece's last cached row
-    const int pslot = (int)blockIdx.x - first;
-    const int count = lastc - first + 1;
+    const long long R = (long long)c.B * c.Hkv * a.rpb;
+    const int nspan = cta_of((long long)bg * a.rpb + a.rpb - 1, R, a.ncta) - cta_of((long long)bg * a.rpb, R, a.ncta) + 1;
+    const int cnt = nspan + 1;
+    auto slot_of = [&](int p) { return p < nspan ? p : newslot; };
+    // A thread owns one float4 column of one row and every npg-th part; its
+    // part loads are issued before the s_h loads and the weights, so the merge
+    // costs about one L2 round trip when cnt <= KMAX * npg.
+    constexpr int NT = 32 * NCW;
+    constexpr int KMAX = 11;
+    const int nout = G * (D / 4);
+    float* sv = comb;                              // [G][cnt] s_h, then weights
+    float4* red = reinterpret_cast<float4*>(comb + kMaxG * 160);   // [npg][nb]
+    bool have_w = false;
+    for (int ob = 0; ob < nout; ob += NT) {
+      const int nb = nout - ob < NT ? nout - ob : NT;
+      const int npg = NT / nb;
+      const bool active = ctid < nb * npg;
+      const int oi = ob + ctid % nb, pg = ctid / nb;
+      const int r = oi / (D / 4), d4 = oi - (oi / (D / 4)) * (D / 4);
+      const float4* pa = reinterpret_cast<const float4*>(a.partA + ((long long)bg * a.maxp * G + r) * D) + d4;
+      const long long pstride = (long long)G * D / 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int p0 = 0; p0 < cnt; p0 += KMAX * npg) {
+        float4 v[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+          const int p = p0 + pg + k * npg;
+          v[k] = (active && p < cnt) ? __ldcg(pa + slot_of(p) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (!have_w) {
+          for (int i = ctid; i < G * cnt; i += NT) {
+            const int rr = i / cnt, p = i - (i / cnt) * cnt;
+            sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + slot_of(p)) * G + rr);
+          }
+          named_sync(1, NT);
+          for (int rr = cw; rr < G; rr += NCW) {    // per-row log-sum-exp, then weights (warp rr)
+            float M = -INFINITY;
+            for (int p = lane; p < cnt; p += 32) M = fmaxf(M, sv[rr * cnt + p]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            const float base = M == -INFINITY ? 0.f : M;
+            float tot = 0.f;
+            for (int p = lane; p < cnt; p += 32) tot += __expf(sv[rr * cnt + p] - base);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+            const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
+            if (lane == 0) s_lse[rr] = l;
+            for (int p = lane; p < cnt; p += 32) {
+              const float sp = sv[rr * cnt + p];
+              sv[rr * cnt + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
+            }
+          }
+          named_sync(1, NT);
+          have_w = true;
+        }
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+          const int p = p0 + pg + k * npg;
+          const float wgt = (active && p < cnt) ? sv[r * cnt + p] : 0.f;
+          acc.x += wgt * v[k].x;
+          acc.y += wgt * v[k].y;
+          acc.z += wgt * v[k].z;
+          acc.w += wgt * v[k].w;
+        }
+      }
+      if (active) red[pg * nb + (oi - ob)] = acc;   // sum the npg partial sums of each column
+      named_sync(1, NT);
+      if (active && pg == 0) {
+        for (int q2 = 1; q2 < npg; ++q2) {
+          const float4 u = red[q2 * nb + (oi - ob)];
+          acc.x += u.x;
+          acc.y += u.y;
+          acc.z += u.z;
+          acc.w += u.w;
+        }
+        const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
+        uint2 pk;
+        pk.x = pack_bf16(acc.x, acc.y);
+        pk.y = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+        if (d4 == 0) a.lse[orow] = s_lse[r];
+      }
+      named_sync(1, NT);
+    }
+    if (ctid == 0) done[bg] = 0u;                  // ready for the next step
+  };
+
+  // ---- rows of bg now live in partials: count them; the CTA that completes
+  // bg merges.  The barrier orders every consumer's partial stores before
+  // thread 0's gpu-scope release (cumulative), which precedes the count.
+  auto complete = [&](int bg, int rows) {
+    named_sync(1, 32 * NCW);
+    if (ctid == 0)
+      s_last = atom_add_acq_rel_gpu(&done[bg], (unsigned)rows) + (unsigned)rows == (unsigned)a.rpb + 1u;
+    named_sync(1, 32 * NCW);
+    if (s_last) merge_bg(bg);
+  };
+
+  // ---- flush: this CTA's run of bg becomes part `pslot` ---------------------
+  auto flush_run = [&](int bg, int pslot, int rows) {
 #pragma unroll
     for (int nb = 0; nb < NG; ++nb)
 #pragma unroll
@@ -595,18 +696,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           wl[cw][8 * nb + 2 * c4 + e] = ls[nb][e];
         }
     }
-    if (owns_new) {
-      // score of the new token for every head of the group (warp r: head r)
-      const bf16* kn = a.k + (long long)bg * D;
-      for (int r = cw; r < G; r += NCW) {
-        const bf16* qr = a.q + (((long long)bb * c.Hq + (long long)g * G + r) * D);
-        float acc = 0.f;
-        for (int d = lane; d < D; d += 32) acc += __bfloat162float(qr[d]) * __bfloat162float(kn[d]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) s_new[r] = acc * a.scale_log2;
-      }
-    }
     for (int rh = 0; rh < G; rh += 4) {            // heads rh .. rh+3 per round
 #pragma unroll
       for (int mb = 0; mb < D / 16; ++mb)
@@ -624,13 +713,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
             }
           }
       named_sync(1, 32 * NCW);
-      const int rows = G - rh < 4 ? G - rh : 4;
-      for (int idx = ctid; idx < rows * D; idx += 32 * NCW) {
+      const int nrow = G - rh < 4 ? G - rh : 4;
+      for (int idx = ctid; idx < nrow * D; idx += 32 * NCW) {
         const int r = idx / D, d = idx - (idx / D) * D, rr = rh + r;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) M = fmaxf(M, wm[w][rr]);
-        if (owns_new) M = fmaxf(M, s_new[rr]);
         const float base = M == -INFINITY ? 0.f : M;
         float Ls = 0.f, acc = 0.f;
 #pragma unroll
@@ -639,128 +727,91 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           Ls += f * wl[w][rr];
           acc += f * comb[(w * 4 + r) * D + d];
         }
-        if (owns_new) {
-          const float f = exp2f(s_new[rr] - base);
-          Ls += f;
-          acc += f * __bfloat162float(a.v[(long long)bg * D + d]);
-        }
         const long long pr = ((long long)bg * a.maxp + pslot) * G + rr;
         a.partA[pr * D + d] = Ls > 0.f ? acc / Ls : 0.f;
         if (d == 0) a.partS[pr] = Ls > 0.f ? (base + log2f(Ls)) * kLn2 : -INFINITY;
       }
       named_sync(1, 32 * NCW);
     }
-    reset_state();                             // the piece's state now lives in the partial
+    reset_state();                             // the run's state now lives in the partial
     cur_bg = -1;
-    if (owns_new && ctid < D / 8) {
-      // append the new token to the query region (row len0); no reader in this launch
+    complete(bg, rows);
+  };
+
+  // ---- the new token of bg = this CTA's index (+ k ncta): its own part (score
+  // q.k per head, value v) and its row of the query region (row len0, which
+  // no reader of this launch touches) ------------------------------------------
+  for (int bg = blockIdx.x; bg < c.B * c.Hkv; bg += a.ncta) {
+    const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+    const bf16* kn = a.k + (long long)bg * D;
+    const bf16* vn = a.v + (long long)bg * D;
+    for (int r = cw; r < G; r += NCW) {
+      const bf16* qr = a.q + (((long long)bb * c.Hq + (long long)g * G + r) * D);
+      float acc = 0.f;
+      for (int d = lane; d < D; d += 32) acc += __bfloat162float(qr[d]) * __bfloat162float(kn[d]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) a.partS[((long long)bg * a.maxp + newslot) * G + r] = acc * a.scale_log2 * kLn2;
+    }
+    for (int i = ctid; i < G * D; i += 32 * NCW)
+      a.partA[(((long long)bg * a.maxp + newslot) * G) * D + i] = __bfloat162float(vn[i % D]);
+    if (ctid < D / 8) {
       const long long qo = q_row_offset(c, bb, g, a.len0);
-      reinterpret_cast<uint4*>(c.qK + qo)[ctid] = reinterpret_cast<const uint4*>(a.k + (long long)bg * D)[ctid];
-      reinterpret_cast<uint4*>(c.qV + qo)[ctid] = reinterpret_cast<const uint4*>(a.v + (long long)bg * D)[ctid];
+      reinterpret_cast<uint4*>(c.qK + qo)[ctid] = reinterpret_cast<const uint4*>(kn)[ctid];
+      reinterpret_cast<uint4*>(c.qV + qo)[ctid] = reinterpret_cast<const uint4*>(vn)[ctid];
     }
-    // ticket: the last CTA of this (batch, kv head) merges its partials.  The
-    // barrier orders every consumer's partial stores before thread 0's
-    // gpu-scope release fence (cumulative), which precedes the ticket.
-    named_sync(1, 32 * NCW);
-    if (ctid == 0) s_last = (atom_add_acq_rel_gpu(&a.tickets[bg], 1u) == (unsigned)(count - 1));
-    named_sync(1, 32 * NCW);
-    if (s_last) {
-      // Merge this head's `count` partials.  A thread owns one float4 column of
-      // one row and every npg-th partial; its partial loads are issued before
-      // the s_h loads and the weights, so the merge costs about one L2 round
-      // trip when count <= KMAX * npg.
-      constexpr int NT = 32 * NCW;
-      constexpr int KMAX = 11;
-      const int nout = G * (D / 4);
-      float* sv = comb;                              // [G][count] s_h, then weights
-      float4* red = reinterpret_cast<float4*>(comb + kMaxG * 160);   // [npg][nb]
-      bool have_w = false;
-      for (int ob = 0; ob < nout; ob += NT) {
-        const int nb = nout - ob < NT ? nout - ob : NT;
-        const int npg = NT / nb;
-        const bool active = ctid < nb * npg;
-        const int oi = ob + ctid % nb, pg = ctid / nb;
-        const int r = oi / (D / 4), d4 = oi - (oi / (D / 4)) * (D / 4);
-        const float4* pa = reinterpret_cast<const float4*>(a.partA + ((long long)bg * a.maxp * G + r) * D) + d4;
-        const long long pstride = (long long)G * D / 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p0 = 0; p0 < count; p0 += KMAX * npg) {
-          float4 v[KMAX];
-#pragma unroll
-          for (int k = 0; k < KMAX; ++k) {
-            const int p = p0 + pg + k * npg;
-            v[k] = (active && p < count) ? __ldcg(pa + p * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-          if (!have_w) {
-            for (int i = ctid; i < G * count; i += NT) {
-              const int rr = i / count, p = i - (i / count) * count;
-              sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + p) * G + rr);
-            }
-            named_sync(1, NT);
-            if (ctid < G) {                           // per-row log-sum-exp, then weights
-              float M = -INFINITY;
-              for (int p = 0; p < count; ++p) M = fmaxf(M, sv[ctid * count + p]);
-              const float base = M == -INFINITY ? 0.f : M;
-              float tot = 0.f;
-              for (int p = 0; p < count; ++p) tot += __expf(sv[ctid * count + p] - base);
-              const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
-              s_lse[ctid] = l;
-              for (int p = 0; p < count; ++p) {
-                const float sp = sv[ctid * count + p];
-                sv[ctid * count + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
-              }
-            }
-            named_sync(1, NT);
-            have_w = true;
-          }
-#pragma unroll
-          for (int k = 0; k < KMAX; ++k) {
-            const int p = p0 + pg + k * npg;
-            const float wgt = (active && p < count) ? sv[r * count + p] : 0.f;
-            acc.x += wgt * v[k].x;
-            acc.y += wgt * v[k].y;
-            acc.z += wgt * v[k].z;
-            acc.w += wgt * v[k].w;
-          }
-        }
-        if (active) red[pg * nb + (oi - ob)] = acc;   // sum the npg partial sums of each column
-        named_sync(1, NT);
-        if (active && pg == 0) {
-          for (int q2 = 1; q2 < npg; ++q2) {
-            const float4 u = red[q2 * nb + (oi - ob)];
-            acc.x += u.x;
-            acc.y += u.y;
-            acc.z += u.z;
-            acc.w += u.w;
-          }
-          const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
-          uint2 pk;
-          pk.x = pack_bf16(acc.x, acc.y);
-          pk.y = pack_bf16(acc.z, acc.w);
-          *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
-          if (d4 == 0) a.lse[orow] = s_lse[r];
-        }
-        named_sync(1, NT);
-      }
-      if (ctid == 0) a.tickets[bg] = 0u;   // ready for the next step
+    if (FP8 && cw < 2) {                        // its FP8 copy, for the steps after this one
+      const long long qrow = (long long)bg * c.q_cap + a.len0;
+      if (cw == 0) quantize_row_warp<D>(kn, c.qK8 + qrow * D, c.qKs + qrow, lane);
+      else quantize_row_warp<D>(vn, c.qV8 + qrow * D, c.qVs + qrow, lane);
     }
+    complete(bg, 1);
+  }
+
+  for (int st = 0;; ++st) {
+    const int slot = st % S::NST, use = st / S::NST;
+    // every consumer warp takes the same path: a warp whose bounded wait gave
+    // up says so before the barrier, and all of them stop after it
+    if (!mbar_wait(smem_u32(&bar_full[slot]), use & 1)) {
+      fail();
+      if (lane == 0) cons_abort = 1;
+    }
+    named_sync(2, 32 * NCW);
+    if (cons_abort) break;
+    const StageMeta m = meta[slot];
+    if (m.flush) flush_run(m.fbg, m.fslot, m.frows);
+    if (m.end) break;
+    if (m.bg != cur_bg) {
+      load_q(m.bg);
+      cur_bg = m.bg;
+    }
+    const uint32_t kb = smem_u32(smem + slot * S::STAGE);
+    const uint32_t vb = kb + S::TILE;
+    const int kw = KPW * cw;   // first key of this warp in the stage
+    if (kw < m.n) {            // a warp past the stage's valid keys adds nothing
+      if constexpr (FP8) fp8_stage(m, kb, vb, scl + slot * 2 * S::SCL_SLOT, kw, m.n);
+      else bf16_stage(kb, vb, kw, m.n, slot);
+    }
+    if (lane == 0) mbar_arrive(smem_u32(&bar_empty[slot]));
   }
 }
 
 }  // namespace
 
 int decode_max_partials(const CacheView& c, int ncta) {
-  // a (batch, kv head) of R/(B*Hkv) rows is touched by at most this many spans
+  // spans that touch one (batch, kv head), + the new token's part
   const int bgs = c.B * c.Hkv;
-  return (ncta + bgs - 1) / bgs + 2;
+  return (ncta + bgs - 1) / bgs + 3;
 }
 
-int decode_num_ctas(const CacheView& c, long long len0, int num_sms) {
-  const long long R = (long long)c.B * c.Hkv * (c.L + len0);
-  long long n = R / 512;                    // at least 512 cached rows per span
+DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms) {
+  DecodePlan pl;
+  long long n = (long long)c.B * c.Hkv * (c.L + len0) / 512;   // at least 512 cached rows per CTA
   if (n < 1) n = 1;
   if (n > num_sms) n = num_sms;
-  return (int)n;
+  pl.ncta = (int)n;
+  pl.maxp = decode_max_partials(c, pl.ncta);
+  return pl;
 }
 
 const char* decode_make_maps(const CacheView& c, DecodeMaps* m) {
@@ -773,15 +824,19 @@ const char* decode_make_maps(const CacheView& c, DecodeMaps* m) {
       !make_tmap_bf16_2d(&m->v_q, c.qV, q_rows, c.D, KS, 64))
     return "query region K/V";
   if (!c.ctxK8) return nullptr;
-  if (!make_tmap_u8_2d(&m->k8_ctx, c.ctxK8, ctx_rows, c.D, KS) ||
-      !make_tmap_u8_2d(&m->v8_ctx, c.ctxV8, ctx_rows, c.D, KS))
+  if (!make_tmap_u8_2d(&m->k8_ctx, c.ctxK8, ctx_rows, c.D, KS8) ||
+      !make_tmap_u8_2d(&m->v8_ctx, c.ctxV8, ctx_rows, c.D, KS8))
     return "FP8 context K/V";
-  if (!make_tmap_f32_row(&m->ks_ctx, c.ctxKs, ctx_rows, DSmem<128, true>::SCL_BOX) ||
-      !make_tmap_f32_row(&m->vs_ctx, c.ctxVs, ctx_rows, DSmem<128, true>::SCL_BOX))
+  // the scale arrays are padded (with zeros) to whole groups of 4 rows
+  if (!make_tmap_f32_quads(&m->ks_ctx, c.ctxKs, (ctx_rows + 3) / 4, DSmem<128, true>::SCL_QUADS) ||
+      !make_tmap_f32_quads(&m->vs_ctx, c.ctxVs, (ctx_rows + 3) / 4, DSmem<128, true>::SCL_QUADS))
     return "FP8 row scales";
-  if (!make_tmap_bf16_2d(&m->k_q64, c.qK, q_rows, c.D, 64, 64) ||
-      !make_tmap_bf16_2d(&m->v_q64, c.qV, q_rows, c.D, 64, 64))
-    return "64-row query region K/V";
+  if (!make_tmap_u8_2d(&m->k8_q, c.qK8, q_rows, c.D, KS8) ||
+      !make_tmap_u8_2d(&m->v8_q, c.qV8, q_rows, c.D, KS8))
+    return "FP8 query region K/V";
+  if (!make_tmap_f32_quads(&m->ks_q, c.qKs, (q_rows + 3) / 4, DSmem<128, true>::SCL_QUADS) ||
+      !make_tmap_f32_quads(&m->vs_q, c.qVs, (q_rows + 3) / 4, DSmem<128, true>::SCL_QUADS))
+    return "FP8 query region row scales";
   return nullptr;
 }
 
@@ -819,10 +874,12 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.tv_q = maps.v_q;
   a.tk8 = maps.k8_ctx;
   a.tv8 = maps.v8_ctx;
-  a.tkq64 = maps.k_q64;
-  a.tvq64 = maps.v_q64;
+  a.tkq8 = maps.k8_q;
+  a.tvq8 = maps.v8_q;
   a.tks = maps.ks_ctx;
   a.tvs = maps.vs_ctx;
+  a.tkqs = maps.ks_q;
+  a.tvqs = maps.vs_q;
   a.c = c;
   a.scale_log2 = scale * kLog2e;
   a.len0 = len0;
@@ -868,7 +925,7 @@ namespace {
 
 constexpr long long kNoAllocPartA = 1LL << 20;    // floats of partial outputs (4 MiB)
 constexpr long long kNoAllocPartS = 1LL << 14;    // floats of partial log-sum-exps (64 KiB)
-constexpr long long kNoAllocTickets = 1024;       // merge tickets (one per batch x kv head)
+constexpr long long kNoAllocTickets = 1024;       // merge counters (one per batch x kv head)
 constexpr long long kNoAllocFloats = kNoAllocPartA + kNoAllocPartS + kNoAllocTickets + 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
@@ -940,14 +997,16 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
   c.ctxV8 = nullptr;
   c.ctxKs = nullptr;
   c.ctxVs = nullptr;
+  c.qK8 = nullptr;
+  c.qV8 = nullptr;
+  c.qKs = nullptr;
+  c.qVs = nullptr;
 
-  DecodePlan pl;
-  pl.ncta = decode_num_ctas(c, q_len, sms);
-  pl.maxp = decode_max_partials(c, sms);
+  const DecodePlan pl = decode_plan(c, q_len, sms);
   const long long rows = (long long)c.B * c.Hkv * pl.maxp * c.G;
   if (rows * c.D > kNoAllocPartA || rows > kNoAllocPartS || (long long)c.B * c.Hkv > kNoAllocTickets)
     return set_error(STAR_EINVAL, "problem too large for the static decode scratch "
-                                  "(B*Hkv*G*D*(ceil(SMs/(B*Hkv))+2) must be <= 1048576 floats, "
+                                  "(B*Hkv*G*D*(ceil(SMs/(B*Hkv))+3) must be <= 1048576 floats, "
                                   "B*Hkv <= 1024)");
   DecodeMaps maps;
   if (const char* bad = decode_make_maps(c, &maps)) {

@@ -1,52 +1,43 @@
-// FP8 (E4M3) copy of the context KV cache, read by the decode step.
+// FP8 (E4M3) copy of the KV cache, read by the decode step.
 //
 // The pages call KV-cache quantisation orthogonal to the method and define
-// none; this is the build's own scheme.  Every cached row (one token of one kv
-// head) gets the scale s = max|x| / 448 (1 when max|x| <= 1e-30) and codes
-// e4m3_rn(x * (1/s)), computed in float32 with IEEE division and rounding to
-// nearest even, so |x/s| <= 448 and nothing saturates.  HBM-bound: one warp
-// per row reads the bf16 row once and writes D bytes and one scale.
+// none; this is the build's own scheme (fp8_row.cuh): one float32 scale per
+// cached row (one token of one kv head).  The context rows are quantised once
+// after phase 1; query-region rows as a prefill appends them (a decode step
+// quantises its own new row).  HBM-bound: one warp per row reads the bf16 row
+// once and writes D bytes and one scale.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "fp8_row.cuh"
 #include "star_common.cuh"
 #include "star_internal.h"
 
 namespace star {
 namespace {
 
-__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
-  uint16_t d;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(d) : "f"(hi), "f"(lo));
-  return d;
-}
-
+// rows [0, rows) of src -> same rows of dst / scale
 template <int D>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const bf16* __restrict__ src,
                                                             uint8_t* __restrict__ dst,
                                                             float* __restrict__ scale, long long rows) {
-  constexpr int PER = D / 32;                     // values per lane (4 or 2)
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  float x[PER];
-  const bf16* r = src + row * D + lane * PER;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) x[i] = __bfloat162float(r[i]);
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) amax = fmaxf(amax, fabsf(x[i]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float s = amax > 1e-30f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  const float inv = __fdiv_rn(1.0f, s);
-  uint8_t* o = dst + row * D + lane * PER;
-#pragma unroll
-  for (int i = 0; i < PER; i += 2) {
-    const uint16_t c = e4m3x2(__fmul_rn(x[i], inv), __fmul_rn(x[i + 1], inv));
-    *reinterpret_cast<uint16_t*>(o + i) = c;
-  }
-  if (lane == 0) scale[row] = s;
+  quantize_row_warp<D>(src + row * D, dst + row * D, scale + row, threadIdx.x & 31);
+}
+
+// prefill rows: input row (bg, r) of [B*Hkv][lq][D] -> query-region row
+// bg * q_cap + len0 + r
+template <int D>
+__global__ void __launch_bounds__(256) quantize_qrows_kernel(const bf16* __restrict__ src,
+                                                             uint8_t* __restrict__ dst,
+                                                             float* __restrict__ scale, int bgs, int lq,
+                                                             int q_cap, int len0) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= (long long)bgs * lq) return;
+  const long long bg = row / lq, r = row - bg * lq;
+  const long long out = bg * q_cap + len0 + r;
+  quantize_row_warp<D>(src + row * D, dst + out * D, scale + out, threadIdx.x & 31);
 }
 
 }  // namespace
@@ -60,6 +51,21 @@ cudaError_t launch_quantize_ctx_fp8(const CacheView& c, cudaStream_t st) {
   } else {
     quantize_rows_kernel<64><<<grid, 256, 0, st>>>(c.ctxK, c.ctxK8, c.ctxKs, rows);
     quantize_rows_kernel<64><<<grid, 256, 0, st>>>(c.ctxV, c.ctxV8, c.ctxVs, rows);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_qregion_fp8(const CacheView& c, const bf16* K, const bf16* V, int len0, int lq,
+                                        cudaStream_t st) {
+  const int bgs = c.B * c.Hkv;
+  const unsigned grid = (unsigned)(((long long)bgs * lq + 7) / 8);
+  if (grid == 0) return cudaSuccess;
+  if (c.D == 128) {
+    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0);
+    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0);
+  } else {
+    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0);
+    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0);
   }
   return cudaGetLastError();
 }

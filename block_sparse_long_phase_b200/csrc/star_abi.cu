@@ -85,8 +85,7 @@ star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
 
 star::DecodePlan plan_decode(const star_cache* c, long long len0) {
   star::DecodePlan pl;
-  pl.ncta = star::decode_num_ctas(c->view, len0, c->num_sms);
-  pl.maxp = star::decode_max_partials(c->view, c->num_sms);
+  pl = star::decode_plan(c->view, len0, c->num_sms);
   return pl;
 }
 
@@ -178,7 +177,13 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const bool fp8 = p->kv_fp8 != 0;
   const long long ctx_rows = (long long)p->B * p->Hkv * p->L;
   const size_t o_k8 = fp8 ? take(kv_ctx) : 0, o_v8 = fp8 ? take(kv_ctx) : 0;
-  const size_t o_ks = fp8 ? take(ctx_rows * 4) : 0, o_vs = fp8 ? take(ctx_rows * 4) : 0;
+  // scales padded to whole groups of 4 rows (zeroed below): decode loads them 4 rows at a time
+  const size_t scl_bytes = (size_t)((ctx_rows + 3) / 4) * 16;
+  const size_t o_ks = fp8 ? take(scl_bytes) : 0, o_vs = fp8 ? take(scl_bytes) : 0;
+  const long long q_rows = (long long)p->B * p->Hkv * p->q_cap;
+  const size_t qscl_bytes = (size_t)((q_rows + 3) / 4) * 16;
+  const size_t o_qk8 = fp8 ? take(kv_q) : 0, o_qv8 = fp8 ? take(kv_q) : 0;
+  const size_t o_qks = fp8 ? take(qscl_bytes) : 0, o_qvs = fp8 ? take(qscl_bytes) : 0;
   e = cudaMalloc(&c->block, off);
   if (e != cudaSuccess) {
     delete c;
@@ -201,6 +206,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
   v.ctxV8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_v8) : nullptr;
   v.ctxKs = fp8 ? reinterpret_cast<float*>(base + o_ks) : nullptr;
   v.ctxVs = fp8 ? reinterpret_cast<float*>(base + o_vs) : nullptr;
+  v.qK8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_qk8) : nullptr;
+  v.qV8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_qv8) : nullptr;
+  v.qKs = fp8 ? reinterpret_cast<float*>(base + o_qks) : nullptr;
+  v.qVs = fp8 ? reinterpret_cast<float*>(base + o_qvs) : nullptr;
   // Zero everything once: decode streams whole 128-row boxes and masks the
   // rows past the end, which must hold finite values.
   e = cudaMemset(c->block, 0, off);
@@ -246,6 +255,8 @@ int star_cache_device_error(star_cache* c, int* flag) {
   int h = 0;
   cudaError_t e = cudaMemcpy(&h, c->scratch.err, sizeof(int), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && h) e = cudaMemset(c->scratch.err, 0, sizeof(int));
+  // a step that gave up may have left its decode counters behind
+  if (e == cudaSuccess && h) e = cudaMemset(c->scratch.tickets, 0, (size_t)c->scratch.n_tickets * 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flag = h;
   return STAR_OK;
@@ -280,7 +291,14 @@ int star_cache_segment_fp8(const star_cache* c, int seg, void** k8, void** v8, f
   if (!c) return fail(STAR_EINVAL, "cache is NULL");
   const star::CacheView& w = c->view;
   if (!w.ctxK8) return fail(STAR_EINVAL, "cache has no FP8 copy (kv_fp8 = 0)");
-  if (seg < 0 || seg >= w.n_seg) return fail(STAR_EINVAL, "context segment %d out of range", seg);
+  if (seg < 0 || seg > w.n_seg) return fail(STAR_EINVAL, "segment %d out of range", seg);
+  if (seg == w.n_seg) {                     // the query region
+    if (k8) *k8 = w.qK8;
+    if (v8) *v8 = w.qV8;
+    if (k_scale) *k_scale = w.qKs;
+    if (v_scale) *v_scale = w.qVs;
+    return STAR_OK;
+  }
   const long long rows = (long long)seg * w.B * w.Hkv * (long long)w.b;
   if (k8) *k8 = w.ctxK8 + rows * w.D;
   if (v8) *v8 = w.ctxV8 + rows * w.D;
@@ -326,6 +344,9 @@ int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K, cons
       c->view, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
       static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
       c->scratch, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && c->view.qK8)
+    e = star::launch_quantize_qregion_fp8(c->view, static_cast<const bf16*>(K), static_cast<const bf16*>(V),
+                                          (int)c->q_len, lq, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_query_prefill launch");
   c->q_len += lq;
   return STAR_OK;

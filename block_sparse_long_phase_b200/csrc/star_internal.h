@@ -31,6 +31,11 @@ struct CacheView {
   uint8_t* ctxV8;
   float* ctxKs;
   float* ctxVs;
+  // ... and of the query region ([B][Hkv][q_cap] rows)
+  uint8_t* qK8;
+  uint8_t* qV8;
+  float* qKs;
+  float* qVs;
 };
 
 __host__ __device__ inline long long seg_len(const CacheView& c, int seg) {
@@ -60,7 +65,7 @@ __host__ __device__ inline long long q_row_offset(const CacheView& c, int bb, in
 struct Scratch {
   float* partA;        // partial outputs A_h
   float* partS;        // partial log-sum-exp s_h
-  unsigned* tickets;   // per (batch, kv head) arrival counters, kept at 0 between calls
+  unsigned* tickets;   // per (batch, kv head) rows folded into parts, kept at 0 between calls
   int* err;            // device error word: set by a kernel whose bounded wait gave up
   long long partA_elems;
   long long partS_elems;
@@ -86,20 +91,26 @@ struct PrefillPlan {
   PrefillChunk chunk[kMaxPrefillChunks];
 };
 
+// Decode work split: the cached rows of all (batch, kv head) pairs, laid end
+// to end, are cut into one balanced span per CTA; each span leaves one part
+// per (batch, kv head) it touches, and the new token one more.
 struct DecodePlan {
-  int ncta;   // CTAs (one balanced span of cached rows each)
-  int maxp;   // partial slots per (batch, kv head)
+  int ncta;   // CTAs
+  int maxp;   // part slots per (batch, kv head)
 };
 int decode_max_partials(const CacheView& c, int ncta);
-int decode_num_ctas(const CacheView& c, long long len0, int num_sms);
+DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms);
 
 // TMA maps of the cache, built once per cache.
 struct DecodeMaps {
   CUtensorMap k_ctx, v_ctx, k_q, v_q;
-  CUtensorMap k8_ctx, v8_ctx, k_q64, v_q64;   // FP8 context rows; 64-row query boxes
-  CUtensorMap ks_ctx, vs_ctx;                 // FP8 per-row scales
+  CUtensorMap k8_ctx, v8_ctx, k8_q, v8_q;     // FP8 rows: context, query region
+  CUtensorMap ks_ctx, vs_ctx, ks_q, vs_q;     // their per-row scales
 };
 cudaError_t launch_quantize_ctx_fp8(const CacheView& c, cudaStream_t st);
+// FP8 copy of prefill rows: K, V [B][Hkv][lq][D] -> query-region rows len0..len0+lq-1
+cudaError_t launch_quantize_qregion_fp8(const CacheView& c, const bf16* K, const bf16* V, int len0, int lq,
+                                        cudaStream_t st);
 // Builds the cache's TMA maps; returns nullptr, or the name of the map the
 // driver rejected.
 const char* decode_make_maps(const CacheView& c, DecodeMaps* m);

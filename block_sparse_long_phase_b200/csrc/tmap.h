@@ -53,15 +53,15 @@ inline bool make_tmap_u8_2d(CUtensorMap* map, const void* base, unsigned long lo
   return r == CUDA_SUCCESS;
 }
 
-// [n] float32 as a one-row 2-D tensor, boxes of `box` elements (box * 4 a
-// multiple of 16); elements past the end read as zero.  The row stride only
-// has to satisfy the encoder (a multiple of 16 bytes): the tensor has one row.
-inline bool make_tmap_f32_row(CUtensorMap* map, const float* base, unsigned long long n, unsigned box) {
+// float32 array of n_quads * 4 elements viewed as [n_quads][4] (16-byte
+// rows), boxes of box_quads whole rows; rows past the end read as zero.
+inline bool make_tmap_f32_quads(CUtensorMap* map, const float* base, unsigned long long n_quads,
+                                unsigned box_quads) {
   auto enc = tmap_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {n, 1};
-  cuuint64_t strides[1] = {(n * 4 + 15) / 16 * 16};
-  cuuint32_t bx[2] = {box, 1};
+  cuuint64_t dims[2] = {4, n_quads};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t bx[2] = {4, box_quads};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, bx,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

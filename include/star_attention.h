@@ -67,9 +67,11 @@ typedef struct {
   int anchor;       /* anchor size b_a, 0 <= b_a <= b (0 = no anchor)       */
   int q_cap;        /* query-region capacity: query tokens + decode steps   */
   float scale;      /* softmax scale; <= 0 selects 1/sqrt(D)                */
-  int kv_fp8;       /* 1: the cache also keeps an FP8 (E4M3) copy of the
-                       context K/V that star_decode_step streams (half the
-                       bytes); 0: bf16 only.  D = 64 or 128.  Quantisation
+  int kv_fp8;       /* 1: the cache also keeps an FP8 (E4M3) copy of every
+                       cached K/V row (context and query region), which
+                       star_decode_step streams instead of the bf16 rows
+                       (about half the bytes); 0: bf16 only.  D = 64 or
+                       128.  Quantisation
                        (no counterpart in the pages, which call KV
                        quantisation orthogonal): per cached row of one kv
                        head, s = max|x| / 448 (1 if max|x| <= 1e-30), codes
@@ -90,9 +92,11 @@ STAR_API int star_cache_create(const star_params* p, star_cache** out);
  * accepted. */
 STAR_API int star_cache_destroy(star_cache* c);
 
-/* FP8 copy of context segment `seg` (kv_fp8 caches only): E4M3 codes of K and
- * V as [B][Hkv][len][D] bytes and their per-row float32 scales [B][Hkv][len],
- * device pointers.  STAR_EINVAL if the cache has no FP8 copy. */
+/* FP8 copy of segment `seg` (kv_fp8 caches only): E4M3 codes of K and V and
+ * their per-row float32 scales, device pointers.  Context segment seg < n:
+ * [B][Hkv][len][D] bytes and [B][Hkv][len] scales; seg = n, the query
+ * region: [B][Hkv][q_cap][D] and [B][Hkv][q_cap] (rows in use as for
+ * star_cache_segment).  STAR_EINVAL if the cache has no FP8 copy. */
 STAR_API int star_cache_segment_fp8(const star_cache* c, int seg, void** k8, void** v8,
                                     float** k_scale, float** v_scale);
 
@@ -139,10 +143,10 @@ STAR_API int star_query_prefill(star_cache* c, int lq, const void* Q, const void
  * [B][Hkv][1][D] to the query region, then q [B][Hq][1][D] attends to every
  * context token and every query-region row (itself included): split-KV
  * partials merged on-chip.  o [B][Hq][1][D] bf16, lse [B][Hq] float32.
- * With kv_fp8 the context rows are read from the FP8 copy (dequantised on
- * chip, fp16 MMA: q and the query region's bf16 K/V are rounded to fp16,
- * so their magnitudes must stay within fp16 range); the query region stays
- * bf16 in memory.  STAR_ENOSPC if the query region is full. */
+ * With kv_fp8 every cached row is read from the FP8 copy (dequantised on
+ * chip, fp16 MMA: q is rounded to fp16, so its magnitude must stay within
+ * fp16 range); the step's own new token enters exactly (bf16), and its FP8
+ * copy is written for the steps after it.  STAR_ENOSPC if the query region is full. */
 STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
                      void* o, float* lse, void* stream);
 
@@ -170,7 +174,7 @@ STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const flo
  *              as [B][Hkv][len_i][D] bf16, segments back to back
  *   q_k/v      query region [B][Hkv][q_cap][D] bf16
  *   q, k, v, o, lse   as for star_decode_step
- * Limits: B*Hkv*G*D*(ceil(SMs/(B*Hkv)) + 2) <= 1048576 and B*Hkv <= 1024,
+ * Limits: B*Hkv*G*D*(ceil(SMs/(B*Hkv)) + 3) <= 1048576 and B*Hkv <= 1024,
  * else STAR_EINVAL.  The first call on a device looks up the array's device
  * address (make it before any stream capture).  Every call shares the one
  * array, so calls that overlap on the GPU (other streams, other threads) race;

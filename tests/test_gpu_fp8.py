@@ -1,17 +1,18 @@
-"""GPU parity of the FP8 (E4M3) context cache and the decode step that streams it.
+"""GPU parity of the FP8 (E4M3) KV cache and the decode step that streams it.
 
 What is compared, and against what:
-  * the FP8 copy of every context segment -- codes and per-row float32
-    scales -- bit-exact against the oracle's quantiser applied to the input
-    K/V (cache contents are integer/byte work);
+  * the FP8 copy of every context segment and of the query region -- codes
+    and per-row float32 scales -- bit-exact against the oracle's quantiser
+    applied to the input K/V rows (cache contents are integer/byte work);
   * phase 1, the bf16 cache and the query prefill are unchanged by the
     option: bit-identical to a bf16-only cache;
-  * each decode step against the fp64 oracle run on the DEQUANTISED context
-    (the oracle's own codes times its own scales) with the bf16 query region:
-    max-abs 1e-2, mean-abs 1e-3, LSE 1e-3, as for the bf16 path.  The kernel
-    multiplies in fp16 (E4M3 codes are exact in fp16; q and the query region
-    are rounded from bf16 to fp16 -- exact for normal fp16 magnitudes -- and
-    p * s_v is rounded to fp16, a relative 2^-11 per term).
+  * each decode step against the fp64 oracle run on the DEQUANTISED cache
+    (the oracle's own codes times its own scales) for every row cached
+    before the step, and on the step's own new token exactly (the kernel
+    folds it in from its bf16 input): max-abs 1e-2, mean-abs 1e-3, LSE 1e-3,
+    as for the bf16 path.  The kernel multiplies in fp16 (E4M3 codes are
+    exact in fp16; q is rounded from bf16 to fp16 -- exact for normal fp16
+    magnitudes -- and p * s_v is rounded to fp16, a relative 2^-11 per term).
 """
 
 import numpy as np
@@ -59,8 +60,8 @@ def dequantised(Kc):
 
 
 def check_fp8_copy(cache, w, Kc, Vc, rows_of_block=None):
-    """Codes and scales of each segment bit-exact against the oracle quantiser
-    (every row, or the given rows of each block)."""
+    """Codes and scales of each context segment bit-exact against the oracle
+    quantiser (every row, or the given rows of each block)."""
     for i, (s, n) in enumerate(so.block_table(w.L, w.b)):
         k8, v8, ks, vs = cache.segment_fp8_tensors(i)
         sel = np.arange(n) if rows_of_block is None else rows_of_block[i] - s
@@ -70,6 +71,37 @@ def check_fp8_copy(cache, w, Kc, Vc, rows_of_block=None):
             got_s = scales[:, :, sel].cpu().numpy()
             assert np.array_equal(got_c, ref_c), f"segment {i}: E4M3 codes differ"
             assert np.array_equal(got_s.view(np.uint32), ref_s.view(np.uint32)), f"segment {i}: scales differ"
+
+
+def check_fp8_region(cache, qk, qv):
+    """FP8 copy of the query region's rows in use bit-exact (qk, qv: the bf16
+    rows appended so far, [B, Hkv, rows, D])."""
+    n = qk.shape[2]
+    k8, v8, ks, vs = cache.segment_fp8_tensors(cache.num_segments - 1)
+    for codes, scales, src in ((k8, ks, qk), (v8, vs, qv)):
+        ref_c, ref_s = so.fp8_quantize_rows(src)
+        assert np.array_equal(codes[:, :, :n].cpu().numpy(), ref_c), "query region: E4M3 codes differ"
+        assert np.array_equal(scales[:, :, :n].cpu().numpy().view(np.uint32), ref_s.view(np.uint32)), \
+            "query region: scales differ"
+
+
+def region_rows(x, t):
+    """bf16 query-region K, V rows in use before decode step t (prefill rows,
+    then the earlier decode tokens)."""
+    qk = torch.cat([x["Kq"]] + [x["kd"][i] for i in range(t)], dim=2)
+    qv = torch.cat([x["Vq"]] + [x["vd"][i] for i in range(t)], dim=2)
+    return qk, qv
+
+
+def decode_reference(x, segs_deq, t, lq, scale, bs=slice(None), gs=slice(None), hs=slice(None)):
+    """Oracle of decode step t on an FP8 cache: earlier rows dequantised, the
+    step's own token exact."""
+    qk, qv = region_rows(x, t)
+    qk, qv = qk[bs, gs].cpu(), qv[bs, gs].cpu()
+    kd, vd = so._f64(x["kd"][t][bs, gs]), so._f64(x["vd"][t][bs, gs])
+    rk = np.concatenate([dequantised(qk), kd], axis=2)
+    rv = np.concatenate([dequantised(qv), vd], axis=2)
+    return so.query_attend(x["qd"][t][bs, hs].cpu(), segs_deq, rk, rv, np.array([lq + t + 1]), scale)
 
 
 VARIANTS = {
@@ -100,13 +132,11 @@ def test_fp8_small_cases(variant):
         k, v, _ = cache.segment_tensors(i)
         k2, v2, _ = ref[0].segment_tensors(i)
         assert torch.equal(bits(k), bits(k2)) and torch.equal(bits(v), bits(v2))
-    # decode on the dequantised context, chained through the oracle's query region
+    # the query region's FP8 copy, and decode on the dequantised cache
+    check_fp8_region(cache, *[t.cpu() for t in region_rows(cpu, w.T)])
     segs = so.cache_segments(dequantised(cpu["Kc"]), dequantised(cpu["Vc"]), w.b)
-    region = np.zeros((w.B, w.Hkv, w.lq + w.T, w.D))
-    _, _, qk, qv = so.query_prefill(cpu["Qq"], cpu["Kq"], cpu["Vq"], segs, region, region, 0, w.scale)
     for t in range(w.T):
-        o_ref, l_ref, qk, qv = so.decode_step(cpu["qd"][t], cpu["kd"][t], cpu["vd"][t], segs, qk, qv,
-                                             w.lq + t, w.scale)
+        o_ref, l_ref = decode_reference(cpu, segs, t, w.lq, w.scale)
         assert_close(dec[t][0], o_ref, dec[t][1], l_ref[:, :, 0], f"{variant} fp8 decode {t}")
     cache.close()
     ref[0].close()
@@ -128,11 +158,8 @@ def test_fp8_zero_rows_and_wide_range():
     _, _, _, vs = cache.segment_fp8_tensors(1)
     assert (ks[:, :, 5] == 1.0).all() and (vs[:, :, 300 - 256] == 1.0).all()
     segs = so.cache_segments(dequantised(cpu["Kc"]), dequantised(cpu["Vc"]), w.b)
-    region = np.zeros((w.B, w.Hkv, w.lq + w.T, w.D))
-    _, _, qk, qv = so.query_prefill(cpu["Qq"], cpu["Kq"], cpu["Vq"], segs, region, region, 0, w.scale)
     for t in range(w.T):
-        o_ref, l_ref, qk, qv = so.decode_step(cpu["qd"][t], cpu["kd"][t], cpu["vd"][t], segs, qk, qv,
-                                             w.lq + t, w.scale)
+        o_ref, l_ref = decode_reference(cpu, segs, t, w.lq, w.scale)
         assert_close(dec[t][0], o_ref, dec[t][1], l_ref[:, :, 0], f"zero/wide rows decode {t}")
     cache.close()
 
@@ -159,12 +186,8 @@ def test_fp8_full_size_sampled(name):
             kc = dequantised(x["Kc"][bs, gs].cpu())
             vc = dequantised(x["Vc"][bs, gs].cpu())
             segs = so.cache_segments(kc, vc, w.b)
-            qk = torch.cat([x["Kq"][bs, gs]] + [x["kd"][t][bs, gs] for t in range(w.T)], dim=2)
-            qv = torch.cat([x["Vq"][bs, gs]] + [x["vd"][t][bs, gs] for t in range(w.T)], dim=2)
-            qk, qv = so._f64(qk), so._f64(qv)
             for t in sorted({0, 1, w.T // 2, w.T - 1}):
-                ref, lref = so.query_attend(x["qd"][t][bs, hs], segs, qk, qv,
-                                            np.array([w.lq + t + 1]), w.scale)
+                ref, lref = decode_reference(x, segs, t, w.lq, w.scale, bs, gs, hs)
                 assert_close(dec[t][0][bs, hs], ref, dec[t][1][bs, hs], lref[:, :, 0],
                              f"{name} fp8 decode {t} kv{g} b{bi}")
     if w.needle:

@@ -121,8 +121,10 @@ def test_small_cases_every_element(variant):
     cache.close()
 
 
-def test_deterministic_and_reset():
-    w = wl.get("tiny")
+@pytest.mark.parametrize("name", ["tiny", "d128-gqa8"])
+def test_deterministic_and_reset(name):
+    """Every output is bit-identical run to run (fixed work split and merge order)."""
+    w = wl.get("tiny").with_(**TINY_VARIANTS[name])
     x = {k: v.cuda() for k, v in wl.make_inputs(w, "cpu").items()}
     a = run_path(w, x)
     b = run_path(w, x)
@@ -137,6 +139,19 @@ def test_deterministic_and_reset():
     o0, l0 = cache.star_decode_step(x["qd"][0], x["kd"][0], x["vd"][0])
     assert torch.equal(bits(Oq), bits(a[3])) and torch.equal(LSEq, a[4])
     assert torch.equal(bits(o0), bits(a[5][0][0]))
+    a[0].close()
+    b[0].close()
+
+
+def test_full_size_decode_is_deterministic():
+    """Bit-identical decode at a full size, where every (batch, kv head) is
+    split over many CTAs."""
+    w = wl.get("8b-32k").with_(T=4)
+    x = wl.make_inputs(w, "cuda")
+    a = run_path(w, x)
+    b = run_path(w, x)
+    for (o1, l1), (o2, l2) in zip(a[5], b[5]):
+        assert torch.equal(bits(o1), bits(o2)) and torch.equal(l1, l2)
     a[0].close()
     b[0].close()
 

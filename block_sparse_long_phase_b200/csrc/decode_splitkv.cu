@@ -168,8 +168,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   __shared__ __align__(8) uint64_t bar_empty[S::NST];
   __shared__ StageMeta meta[S::NST];
   __shared__ float wm[NCW][16], wl[NCW][16];
-  __shared__ float s_new[kMaxG];
-  __shared__ float s_lse[kMaxG];
   __shared__ int s_last, abort_s, cons_abort;
 
   const CacheView& c = a.c;
@@ -574,22 +572,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   const int newslot = a.maxp - 1;                 // the new token's part
 
   // ---- merge of bg's parts: one per CTA whose span holds rows of bg (slots
-  // 0..nspan-1) and the new token (slot maxp-1) -----------------------------
+  // 0..nspan-1) and the new token (slot maxp-1).  A thread owns one float4
+  // column of one row and every npg-th part: it loads their A_h and s_h
+  // together (one L2 round trip), folds them with a running maximum, and
+  // the npg threads of a column combine through shared memory. -------------
   auto merge_bg = [&](int bg) {
     const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
     const long long R = (long long)c.B * c.Hkv * a.rpb;
     const int nspan = cta_of((long long)bg * a.rpb + a.rpb - 1, R, a.ncta) - cta_of((long long)bg * a.rpb, R, a.ncta) + 1;
     const int cnt = nspan + 1;
     auto slot_of = [&](int p) { return p < nspan ? p : newslot; };
-    // A thread owns one float4 column of one row and every npg-th part; its
-    // part loads are issued before the s_h loads and the weights, so the merge
-    // costs about one L2 round trip when cnt <= KMAX * npg.
     constexpr int NT = 32 * NCW;
     constexpr int KMAX = 11;
     const int nout = G * (D / 4);
-    float* sv = comb;                              // [G][cnt] s_h, then weights
-    float4* red = reinterpret_cast<float4*>(comb + kMaxG * 160);   // [npg][nb]
-    bool have_w = false;
+    float4* red = reinterpret_cast<float4*>(comb);             // [npg][nb] partial sums
+    float* redm = comb + 4 * NT;                               // [npg][nb] their maxima
+    float* redl = redm + NT;                                   // [npg][nb] their sums
     for (int ob = 0; ob < nout; ob += NT) {
       const int nb = nout - ob < NT ? nout - ob : NT;
       const int npg = NT / nb;
@@ -597,67 +595,70 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       const int oi = ob + ctid % nb, pg = ctid / nb;
       const int r = oi / (D / 4), d4 = oi - (oi / (D / 4)) * (D / 4);
       const float4* pa = reinterpret_cast<const float4*>(a.partA + ((long long)bg * a.maxp * G + r) * D) + d4;
+      const float* ps = a.partS + (long long)bg * a.maxp * G + r;
       const long long pstride = (long long)G * D / 4;
+      float M = -INFINITY, L = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int p0 = 0; p0 < cnt; p0 += KMAX * npg) {
         float4 v[KMAX];
+        float sp[KMAX];
 #pragma unroll
         for (int k = 0; k < KMAX; ++k) {
           const int p = p0 + pg + k * npg;
-          v[k] = (active && p < cnt) ? __ldcg(pa + slot_of(p) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const bool ok = active && p < cnt;
+          v[k] = ok ? __ldcg(pa + slot_of(p) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+          sp[k] = ok ? __ldcg(ps + (long long)slot_of(p) * G) : -INFINITY;
         }
-        if (!have_w) {
-          for (int i = ctid; i < G * cnt; i += NT) {
-            const int rr = i / cnt, p = i - (i / cnt) * cnt;
-            sv[i] = __ldcg(a.partS + ((long long)bg * a.maxp + slot_of(p)) * G + rr);
+        float Mn = M;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) Mn = fmaxf(Mn, sp[k]);
+        if (Mn != -INFINITY) {
+          const float al = M == -INFINITY ? 0.f : __expf(M - Mn);
+          L *= al;
+          acc.x *= al;
+          acc.y *= al;
+          acc.z *= al;
+          acc.w *= al;
+#pragma unroll
+          for (int k = 0; k < KMAX; ++k) {
+            const float wk = sp[k] == -INFINITY ? 0.f : __expf(sp[k] - Mn);
+            L += wk;
+            acc.x += wk * v[k].x;
+            acc.y += wk * v[k].y;
+            acc.z += wk * v[k].z;
+            acc.w += wk * v[k].w;
           }
-          named_sync(1, NT);
-          for (int rr = cw; rr < G; rr += NCW) {    // per-row log-sum-exp, then weights (warp rr)
-            float M = -INFINITY;
-            for (int p = lane; p < cnt; p += 32) M = fmaxf(M, sv[rr * cnt + p]);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-            const float base = M == -INFINITY ? 0.f : M;
-            float tot = 0.f;
-            for (int p = lane; p < cnt; p += 32) tot += __expf(sv[rr * cnt + p] - base);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
-            const float l = M == -INFINITY ? -INFINITY : base + __logf(tot);
-            if (lane == 0) s_lse[rr] = l;
-            for (int p = lane; p < cnt; p += 32) {
-              const float sp = sv[rr * cnt + p];
-              sv[rr * cnt + p] = sp == -INFINITY ? 0.f : __expf(sp - l);
-            }
-          }
-          named_sync(1, NT);
-          have_w = true;
-        }
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-          const int p = p0 + pg + k * npg;
-          const float wgt = (active && p < cnt) ? sv[r * cnt + p] : 0.f;
-          acc.x += wgt * v[k].x;
-          acc.y += wgt * v[k].y;
-          acc.z += wgt * v[k].z;
-          acc.w += wgt * v[k].w;
+          M = Mn;
         }
       }
-      if (active) red[pg * nb + (oi - ob)] = acc;   // sum the npg partial sums of each column
+      if (active) {
+        red[pg * nb + (oi - ob)] = acc;
+        redm[pg * nb + (oi - ob)] = M;
+        redl[pg * nb + (oi - ob)] = L;
+      }
       named_sync(1, NT);
       if (active && pg == 0) {
-        for (int q2 = 1; q2 < npg; ++q2) {
+        float Mt = M;
+        for (int q2 = 1; q2 < npg; ++q2) Mt = fmaxf(Mt, redm[q2 * nb + (oi - ob)]);
+        float Lt = 0.f;
+        float4 at = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q2 = 0; q2 < npg; ++q2) {
+          const float mq = redm[q2 * nb + (oi - ob)];
+          const float f = mq == -INFINITY ? 0.f : __expf(mq - Mt);
           const float4 u = red[q2 * nb + (oi - ob)];
-          acc.x += u.x;
-          acc.y += u.y;
-          acc.z += u.z;
-          acc.w += u.w;
+          Lt += f * redl[q2 * nb + (oi - ob)];
+          at.x += f * u.x;
+          at.y += f * u.y;
+          at.z += f * u.z;
+          at.w += f * u.w;
         }
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
         const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
         uint2 pk;
-        pk.x = pack_bf16(acc.x, acc.y);
-        pk.y = pack_bf16(acc.z, acc.w);
+        pk.x = pack_bf16(at.x * inv, at.y * inv);
+        pk.y = pack_bf16(at.z * inv, at.w * inv);
         *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
-        if (d4 == 0) a.lse[orow] = s_lse[r];
+        if (d4 == 0) a.lse[orow] = Lt > 0.f ? Mt + __logf(Lt) : -INFINITY;
       }
       named_sync(1, NT);
     }
@@ -809,6 +810,12 @@ DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms) {
   long long n = (long long)c.B * c.Hkv * (c.L + len0) / 512;   // at least 512 cached rows per CTA
   if (n < 1) n = 1;
   if (n > num_sms) n = num_sms;
+  // A whole number of CTAs per (batch, kv head), if that idles at most 4 % of
+  // the SMs: no span then crosses from one (batch, kv head) into the next,
+  // which would cost it a second flush.
+  const long long bgs = (long long)c.B * c.Hkv;
+  const long long aligned = n / bgs * bgs;
+  if (n == num_sms && aligned > 0 && aligned * 25 >= n * 24) n = aligned;
   pl.ncta = (int)n;
   pl.maxp = decode_max_partials(c, pl.ncta);
   return pl;

@@ -43,6 +43,22 @@ WORKLOAD = "8b-32k"
 METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roofline"
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu captures summarised under profiles/, valid only for the kernel source they
+# were taken on (first 16 hex digits of its sha256); null otherwise.
+TRAFFIC = {
+    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3d5aa39a55201982", 2335043256),
+    "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "7f675125a444770d", 144934912),
+}
+
+
+def traffic(key):
+    import hashlib
+    path, sha, nbytes = TRAFFIC[key]
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return nbytes if hashlib.sha256(f.read()).hexdigest()[:16] == sha else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -68,9 +84,10 @@ def decode_bytes(w, t):
 
 
 def decode_bytes_fp8(w, t):
-    """Same, FP8 context cache: one byte per context element plus a float32
-    scale per context row, for K and for V; the query region stays bf16."""
-    return w.B * w.Hkv * (w.L * (w.D + 4) * 2 + (w.lq + t + 1) * w.D * 2 * 2)
+    """Same, FP8 cache: one byte per element plus a float32 scale per row, for K
+    and for V, of every row cached before the step; the step's own token is
+    read in bf16."""
+    return w.B * w.Hkv * ((w.L + w.lq + t) * (w.D + 4) * 2 + w.D * 2 * 2)
 
 
 class Clocks:
@@ -499,10 +516,12 @@ def main():
                    "us_per_step": dec_avg_s / w.T * 1e6,
                    "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"],
                                 "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
-                                "traffic": None, "peak_source": pk["source"]}},
+                                "traffic": traffic("decode 8b-32k") if w.name == "8b-32k" else None,
+                                "peak_source": pk["source"]}},
         "prefill_ms": sum(pre_ms) / args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"], "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"],
+                     "traffic": traffic("phase1 8b-32k") if w.name == "8b-32k" else None,
                      "kernel": "phase-1 context encode", "flops_per_launch": flops,
                      "peak_source": pk["source"] + " burst bf16 dense"},
         "clocks": clk,
@@ -530,7 +549,7 @@ def main():
         wl3, t3 = long_dec_fp8
         gbs = decode_bytes_fp8(wl3, 0) / (t3 * 1e-6) / 1e9
         line["decode_long_fp8"] = {
-            "workload": wl3.name, "kv_cache": "context K/V in E4M3 with a float32 scale per row",
+            "workload": wl3.name, "kv_cache": "K/V rows in E4M3 with a float32 scale per row",
             "value": world * wl3.B / (t3 * 1e-6), "unit": "decode tok/s", "us_per_step": t3,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": None,

@@ -49,6 +49,7 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 TRAFFIC = {
     "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3d5aa39a55201982", 2335043256),
     "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "7f675125a444770d", 144934912),
+    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "7f675125a444770d", 287263232),
 }
 
 
@@ -552,7 +553,7 @@ def main():
             "workload": wl3.name, "kv_cache": "K/V rows in E4M3 with a float32 scale per row",
             "value": world * wl3.B / (t3 * 1e-6), "unit": "decode tok/s", "us_per_step": t3,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic("decode fp8 8b-128k"),
                          "bytes_per_step": decode_bytes_fp8(wl3, 0)}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, d, sample, threads = cpu_oracle_sample(w, x)

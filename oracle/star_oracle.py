@@ -377,3 +377,99 @@ def e4m3_value(codes):
 
 def fp8_dequantize_rows(codes, s):
     return e4m3_value(codes) * np.asarray(s, np.float64)[..., None]
+
+
+# ---------------------------------------------------------------------------
+# RoPE front end and anchor position IDs (NEXT-1).
+#
+# [P2] "Phase 1: Context Encoding with Anchor Blocks", Step 2: the anchor
+# tokens prepended to block i keep their original position IDs 0..b-1 while
+# the block's own tokens keep theirs; [P2] ablation of section 4.1 (Table 4):
+# anchor position IDs taken from the first block (proposed), from the block
+# just before block i, or sampled at random from [0, start of block i).
+# Readings (listed in the design doc): rotary embedding in the RoFormer form on
+# adjacent pairs (2k, 2k+1) with inverse frequencies base^(-2k/D), base
+# 500000 (Llama 3) and no frequency rescaling; "previous" = the b_a positions
+# right before block i; random positions are drawn by the caller; query-region
+# row r sits at position L + r.  Pinned by tests/test_oracle_rope.py.
+# ---------------------------------------------------------------------------
+ROPE_BASE = 500000.0
+
+
+def rope_inv_freq(D: int, base: float = ROPE_BASE) -> np.ndarray:
+    """Inverse frequencies base^(-2k/D), k = 0..D/2-1 (float64)."""
+    k = np.arange(D // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * k / D)
+
+
+def rope(x, pos, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotary embedding of x [..., n, D] at integer positions pos [n]:
+    each pair (x_2k, x_2k+1) is rotated by the angle pos * base^(-2k/D)."""
+    x = _f64(x)
+    D = x.shape[-1]
+    ang = np.asarray(pos, np.float64)[:, None] * rope_inv_freq(D, base)[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = x0 * c - x1 * s
+    y[..., 1::2] = x0 * s + x1 * c
+    return y
+
+
+def anchor_positions(mode: str, n_blocks: int, b: int, b_a: int, given=None) -> np.ndarray:
+    """Position IDs [n_blocks - 1, b_a] of the anchor keys prepended to blocks
+    1..n-1: "first" -> 0..b_a-1 (the proposed method); "previous" -> the b_a
+    positions right before block i, i*b - b_a .. i*b - 1; "given" -> the
+    caller's array (e.g. random draws from [0, i*b))."""
+    i = np.arange(1, n_blocks, dtype=np.int64)[:, None]
+    j = np.arange(b_a, dtype=np.int64)[None, :]
+    if mode == "first":
+        return np.broadcast_to(j, (n_blocks - 1, b_a)).copy()
+    if mode == "previous":
+        return i * b - b_a + j
+    if mode == "given":
+        return np.asarray(given, np.int64).reshape(n_blocks - 1, b_a)
+    raise ValueError(mode)
+
+
+def ctx_encode_rope(Q, K, V, b: int, b_a: int, scale: float, anchor_pos, base: float = ROPE_BASE,
+                    rows=None):
+    """Phase 1 on un-rotated Q, K [B, H, L, D] with rotary positions.
+
+    Token t of block i is at position t (positions preserved, [P2] Phase 1
+    Step 2).  Block 0 attends causally to itself; block i >= 1 attends to the
+    whole anchor -- K rows 0..b_a-1 rotated at anchor_pos[i-1] -- and causally
+    to its own block.  V is not rotated.  Returns (O, LSE) for ``rows``
+    (default all), like ``ctx_encode``.
+    """
+    Bn, Hq, L, D = Q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    rows = np.arange(L) if rows is None else np.asarray(rows, np.int64)
+    O = np.zeros((Bn, Hq, len(rows), D))
+    LSE = np.zeros((Bn, Hq, len(rows)))
+    for i, (s, n) in enumerate(block_table(L, b)):
+        sel = np.nonzero((rows >= s) & (rows < s + n))[0]
+        if len(sel) == 0:
+            continue
+        t = rows[sel]
+        own = np.arange(s, s + n)
+        if i == 0:
+            kpos = own
+            mask = own[None, :] <= t[:, None]
+        else:
+            kpos = np.concatenate([np.asarray(anchor_pos[i - 1], np.int64), own])
+            mask = np.concatenate([np.ones((len(t), b_a), bool), own[None, :] <= t[:, None]], axis=1)
+        for bi in range(Bn):
+            for g in range(Hkv):
+                kraw = _f64(K[bi, g])
+                kk = np.concatenate([rope(kraw[:b_a], kpos[:b_a], base), rope(kraw[s:s + n], own, base)]) \
+                    if i > 0 else rope(kraw[s:s + n], own, base)
+                vv = _f64(V[bi, g])
+                vv = np.concatenate([vv[:b_a], vv[s:s + n]]) if i > 0 else vv[s:s + n]
+                for h in range(g * G, (g + 1) * G):
+                    q = rope(_f64(Q[bi, h])[t], t, base)
+                    o, lse = masked_attention(q, kk, vv, mask, scale)
+                    O[bi, h, sel] = o
+                    LSE[bi, h, sel] = lse
+    return O, LSE

@@ -23,6 +23,7 @@ EXPORTS = (
     "star_cache_segment", "star_cache_segment_fp8", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
+    "star_rope", "star_anchor_keys", "star_ctx_encode_anchored",
 )
 
 
@@ -66,6 +67,9 @@ def load(path: str = LIB_PATH):
     lib.star_query_prefill.argtypes = [vp, i, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_lse_merge.argtypes = [i, ll, i, vp, vp, vp, vp, vp]
+    lib.star_rope.argtypes = [i, i, ll, i, ctypes.c_double, vp, ll, vp, vp, vp]
+    lib.star_anchor_keys.argtypes = [vp, i, vp, ctypes.c_double, vp, vp, vp]
+    lib.star_ctx_encode_anchored.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step_noalloc.argtypes = [ctypes.POINTER(StarParams), ll, vp, vp, vp, vp,
                                              vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:

@@ -16,6 +16,10 @@ import torch
 from . import _abi
 
 
+# Rotary base of the Llama 3 family (no frequency rescaling).
+ROPE_THETA = 500000.0
+
+
 def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr())
 
@@ -136,20 +140,67 @@ class StarCache:
         _abi.check(self.lib.star_cache_reset_query(self.handle))
 
     # -- the hot path --------------------------------------------------------
-    def star_ctx_encode(self, Q, K, V, O=None, LSE=None):
+    def star_ctx_encode(self, Q, K, V, O=None, LSE=None, Ka=None):
+        """Phase 1.  ``Ka`` (optional, from ``star_anchor_keys``): per-block anchor keys."""
         B, Hq, Hkv, D, L = self.B, self.Hq, self.Hkv, self.D, self.L
         _need(Q, (B, Hq, L, D), torch.bfloat16, "Q")
         _need(K, (B, Hkv, L, D), torch.bfloat16, "K")
         _need(V, (B, Hkv, L, D), torch.bfloat16, "V")
+        if Ka is not None:
+            _need(Ka, (self.num_segments - 2, B, Hkv, self.anchor, D), torch.bfloat16, "Ka")
         if O is None:
             O = torch.empty((B, Hq, L, D), dtype=torch.bfloat16, device=Q.device)
         if LSE is None:
             LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
         _need(O, (B, Hq, L, D), torch.bfloat16, "O")
         _need(LSE, (B, Hq, L), torch.float32, "LSE")
-        _abi.check(self.lib.star_ctx_encode(self.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
-                                            _ptr(LSE), _stream(Q.device)))
+        _abi.check(self.lib.star_ctx_encode_anchored(self.handle, _ptr(Q), _ptr(K), _ptr(V),
+                                                     _ptr(Ka) if Ka is not None else None, _ptr(O),
+                                                     _ptr(LSE), _stream(Q.device)))
         return O, LSE
+
+    def star_anchor_keys(self, K, anchor="first", theta=ROPE_THETA, Ka=None):
+        """Anchor keys of blocks 1..n-1 from un-rotated K [B, Hkv, L, D]:
+        ``anchor`` = "first" (IDs 0..b_a-1), "previous" (the b_a positions before
+        each block) or an int32 CUDA tensor [n-1, b_a] of IDs.  Returns Ka
+        [n-1, B, Hkv, b_a, D] bf16."""
+        B, Hkv, D, L = self.B, self.Hkv, self.D, self.L
+        _need(K, (B, Hkv, L, D), torch.bfloat16, "K")
+        nb = self.num_segments - 1
+        if Ka is None:
+            Ka = torch.empty((max(nb - 1, 0), B, Hkv, self.anchor, D), dtype=torch.bfloat16, device=K.device)
+        pos = None
+        if isinstance(anchor, str):
+            mode = {"first": 0, "previous": 1}[anchor]
+        else:
+            mode = 2
+            pos = anchor
+            _need(pos, (nb - 1, self.anchor), torch.int32, "anchor positions")
+        _abi.check(self.lib.star_anchor_keys(self.handle, mode, _ptr(pos) if pos is not None else None,
+                                             float(theta), _ptr(K), _ptr(Ka) if Ka.numel() else None,
+                                             _stream(K.device)))
+        return Ka
+
+    def star_ctx_encode_rope(self, Q, K, V, anchor="first", theta=ROPE_THETA, O=None, LSE=None):
+        """Phase 1 on un-rotated Q, K: rotates them at positions 0..L-1, builds the
+        anchor keys of the chosen position-ID variant (none needed for "first"),
+        encodes.  Returns (O, LSE)."""
+        Qr = star_rope(Q, theta=theta)
+        Kr = star_rope(K, theta=theta)
+        Ka = None if (isinstance(anchor, str) and anchor == "first") else self.star_anchor_keys(K, anchor, theta)
+        return self.star_ctx_encode(Qr, Kr, V, O, LSE, Ka=Ka)
+
+    def star_query_prefill_rope(self, Q, K, V, theta=ROPE_THETA, O=None, LSE=None):
+        """Query prefill on un-rotated Q, K: query row r sits at position L + q_len + r."""
+        p0 = self.L + self.q_len
+        return self.star_query_prefill(star_rope(Q, pos0=p0, theta=theta), star_rope(K, pos0=p0, theta=theta),
+                                       V, O, LSE)
+
+    def star_decode_step_rope(self, q, k, v, theta=ROPE_THETA, o=None, lse=None):
+        """Decode step on un-rotated q, k: the token sits at position L + q_len."""
+        p0 = self.L + self.q_len
+        return self.star_decode_step(star_rope(q, pos0=p0, theta=theta), star_rope(k, pos0=p0, theta=theta),
+                                     v, o, lse)
 
     def star_query_prefill(self, Q, K, V, O=None, LSE=None):
         B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
@@ -181,6 +232,22 @@ class StarCache:
         _abi.check(self.lib.star_decode_step(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                              _ptr(lse), _stream(q.device)))
         return o, lse
+
+
+def star_rope(x: torch.Tensor, positions=None, pos0=0, theta=ROPE_THETA, out=None):
+    """Rotary embedding of x [B, H, L, D] bf16 (CUDA) at positions
+    ``positions`` (int32 CUDA tensor [L]) or pos0 + t; ``out`` may be ``x``."""
+    lib = _abi.load()
+    B, H, L, D = x.shape
+    _need(x, (B, H, L, D), torch.bfloat16, "x")
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, (B, H, L, D), torch.bfloat16, "out")
+    if positions is not None:
+        _need(positions, (L,), torch.int32, "positions")
+    _abi.check(lib.star_rope(B, H, L, D, float(theta), _ptr(positions) if positions is not None else None,
+                             int(pos0), _ptr(x), _ptr(out), _stream(x.device)))
+    return out
 
 
 def star_lse_merge(A: torch.Tensor, s: torch.Tensor, out_A=None, out_s=None):

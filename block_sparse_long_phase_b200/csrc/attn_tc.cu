@@ -60,7 +60,8 @@ struct CtxTcArgs {
   CUtensorMap tq;   // phase 1: Q as [B*Hq*L][D]; prefill: query rows as [B*Hq*lq][D]
   CUtensorMap tk;   // phase 1: K as [B*Hkv*L][D]; prefill: context cache as [B*Hkv*L][D]
   CUtensorMap tv;
-  CUtensorMap tkq;  // prefill: query region as [B*Hkv*q_cap][D]
+  CUtensorMap tkq;  // prefill: query region as [B*Hkv*q_cap][D]; phase 1: anchor keys as
+                    // [(n-1)*B*Hkv*b_a][D] when anchor_keys is set
   CUtensorMap tvq;
   CacheView c;
   float scale_log2;
@@ -70,6 +71,7 @@ struct CtxTcArgs {
   float* LSE;
   const int4* work;   // phase 1: (b*Hkv + g, head pair, block, q tile)
   int* err;
+  int anchor_keys;    // phase 1: block i >= 1 reads its anchor's K tiles from tkq
   // prefill
   int lq, len0, row_pairs;
   float* partA;
@@ -207,6 +209,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       prefetch_tmap(&a.tq);
       prefetch_tmap(mk);
       prefetch_tmap(mv);
+      const bool own_anchor = !PF && a.anchor_keys && blk > 0;   // per-block anchor keys
+      if (own_anchor) prefetch_tmap(&a.tkq);
       const uint32_t qb = smem_u32(&bar_q_full);
       mbar_arrive_expect_tx(qb, nq * S::TILE);
       for (int q = 0; q < nq; ++q) {
@@ -223,10 +227,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         if (*(volatile int*)&abort_s) break;
         const long long tok = PF ? (long long)j * BN
                                  : (j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN);
-        const int row = (int)(kv_row0 + tok);
+        int row = (int)(kv_row0 + tok);
+        const CUtensorMap* m = (i & 1) ? mv : mk;
+        if (own_anchor && !(i & 1) && j < n_anchor) {
+          // K of block blk's anchor: rows of Ka[blk - 1] for this (batch, kv head)
+          m = &a.tkq;
+          row = (int)((((long long)(blk - 1) * c.B * c.Hkv) + bg) * c.b_a + tok);
+        }
         const uint32_t fb = smem_u32(&bar_kv_full[slot]);
         mbar_arrive_expect_tx(fb, S::TILE);
-        const CUtensorMap* m = (i & 1) ? mv : mk;
         for (int hf = 0; hf < NH; ++hf)
           tma_load_2d(smem_u32(smem + S::RING + slot * S::TILE + hf * S::HALF), m, hf * 64, row, fb);
         last_use[slot] = use;
@@ -502,7 +511,7 @@ cudaError_t attn_tc_prepare(int D) {
 
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
-                                 int* err, cudaStream_t st) {
+                                 int* err, cudaStream_t st, const bf16* Ka) {
   if (n_work == 0) return cudaSuccess;
   CtxTcArgs a;
   memset(&a, 0, sizeof(a));
@@ -511,6 +520,11 @@ cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q,
   if (!make_tmap_bf16_2d(&a.tq, Q, qrows, c.D, BM, 64) || !make_tmap_bf16_2d(&a.tk, K, kvrows, c.D, BN, 64) ||
       !make_tmap_bf16_2d(&a.tv, V, kvrows, c.D, BN, 64))
     return cudaErrorInvalidValue;
+  if (Ka && c.n_seg > 1 && c.b_a > 0) {
+    const unsigned long long karows = (unsigned long long)(c.n_seg - 1) * c.B * c.Hkv * c.b_a;
+    if (!make_tmap_bf16_2d(&a.tkq, Ka, karows, c.D, BN, 64)) return cudaErrorInvalidValue;
+    a.anchor_keys = 1;
+  }
   a.c = c;
   a.scale_log2 = scale * kLog2e;
   a.K = K;

@@ -313,20 +313,82 @@ int star_cache_reset_query(star_cache* c) {
   return STAR_OK;
 }
 
-int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
-                    float* LSE, void* stream) {
+int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const void* V, const void* Ka,
+                             void* O, float* LSE, void* stream) {
   if (!c) return fail(STAR_EINVAL, "cache is NULL");
   if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+      (Ka && !aligned16(Ka)))
     return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
   cudaError_t e = star::launch_ctx_encode_tc(
       c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
       static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work,
-      c->scratch.err, static_cast<cudaStream_t>(stream));
+      c->scratch.err, static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka));
   if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
   if (e == cudaSuccess && c->view.ctxK8) e = star::launch_quantize_ctx_fp8(c->view, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
   c->q_len = 0;
+  return STAR_OK;
+}
+
+int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
+                    float* LSE, void* stream) {
+  return star_ctx_encode_anchored(c, Q, K, V, nullptr, O, LSE, stream);
+}
+
+int star_rope(int B, int H, long long L, int D, double theta, const int* pos, long long pos0, const void* x,
+              void* y, void* stream) {
+  if (B < 1 || H < 1 || L < 0) return fail(STAR_EINVAL, "need B, H >= 1 and L >= 0");
+  if (D != 64 && D != 128) return fail(STAR_EUNSUPPORTED, "head dim %d: RoPE supports D = 64 or 128", D);
+  if (!(theta > 1.0)) return fail(STAR_EINVAL, "theta must be > 1");
+  if (B > 65535) return fail(STAR_EINVAL, "B must be <= 65535");
+  if (pos0 < 0) return fail(STAR_EINVAL, "pos0 must be >= 0");
+  if (L == 0) return STAR_OK;
+  if (!x || !y) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(x) || !aligned16(y)) return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  star::RopeJob j;
+  j.x = static_cast<const bf16*>(x);
+  j.y = static_cast<bf16*>(y);
+  j.x_seq = j.y_seq = L;
+  j.x_grp = j.y_grp = 0;
+  j.n = L;
+  j.H = H;
+  j.pos = pos;
+  j.pos_grp = 0;
+  j.pos0 = pos0;
+  j.pos0_grp = 0;
+  star::rope_inv_freq(D, theta, j.inv_freq);
+  cudaError_t e = star::launch_rope(j, D, B, 1, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_rope launch");
+  return STAR_OK;
+}
+
+int star_anchor_keys(const star_cache* c, int mode, const int* pos, double theta, const void* K, void* Ka,
+                     void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  const star::CacheView& w = c->view;
+  if (mode < 0 || mode > 2) return fail(STAR_EINVAL, "mode must be 0 (first), 1 (previous) or 2 (given)");
+  if (!(theta > 1.0)) return fail(STAR_EINVAL, "theta must be > 1");
+  if (w.n_seg < 2 || w.b_a == 0) return STAR_OK;          // no block has an anchor
+  if (mode == 2 && !pos) return fail(STAR_EINVAL, "mode 2 needs the position array");
+  if (!K || !Ka) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(K) || !aligned16(Ka)) return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  star::RopeJob j;
+  j.x = static_cast<const bf16*>(K);
+  j.y = static_cast<bf16*>(Ka);
+  j.x_seq = w.L;                                      // K [B][Hkv][L][D]: rows 0..b_a-1 of each (b, g)
+  j.x_grp = 0;                                        // every block reads the same anchor rows
+  j.y_seq = w.b_a;                                    // Ka [n-1][B][Hkv][b_a][D]
+  j.y_grp = (long long)w.B * w.Hkv * w.b_a;
+  j.n = w.b_a;
+  j.H = w.Hkv;
+  j.pos = mode == 2 ? pos : nullptr;
+  j.pos_grp = w.b_a;                                  // pos [n-1][b_a]
+  j.pos0 = mode == 1 ? (long long)w.b - w.b_a : 0;    // block i = z + 1: positions i*b - b_a + t
+  j.pos0_grp = mode == 1 ? w.b : 0;
+  star::rope_inv_freq(w.D, theta, j.inv_freq);
+  cudaError_t e = star::launch_rope(j, w.D, w.B, w.n_seg - 1, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_anchor_keys launch");
   return STAR_OK;
 }
 

@@ -75,9 +75,29 @@ struct Scratch {
 // ---- launchers (defined in the .cu files) --------------------------------
 size_t ctx_tc_work_count(const CacheView& c);
 void ctx_tc_fill_work(const CacheView& c, int4* out);
+// Ka (may be null): anchor keys of blocks 1..n-1 as [n-1][B][Hkv][b_a][D];
+// block i >= 1 then reads its anchor keys from Ka[i-1] instead of K rows 0..b_a-1.
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
-                                 int* err, cudaStream_t st);
+                                 int* err, cudaStream_t st, const bf16* Ka = nullptr);
+
+// Rotary embedding of rows: for group z < groups, batch b < B, head h < H and
+// t < n, row (z*x_grp + (b*H + h)*x_seq + t) of x is rotated at position
+// pos[z*pos_grp + t] (pos non-null) or pos0 + z*pos0_grp + t, and written to
+// row (z*y_grp + (b*H + h)*y_seq + t) of y.
+struct RopeJob {
+  const bf16* x;
+  bf16* y;
+  long long x_seq, y_seq, x_grp, y_grp;
+  long long n;
+  int H;
+  const int* pos;
+  long long pos_grp;
+  long long pos0, pos0_grp;
+  double inv_freq[64];
+};
+void rope_inv_freq(int D, double base, double* out);
+cudaError_t launch_rope(const RopeJob& j, int D, int B, int groups, cudaStream_t st);
 
 struct PrefillChunk {
   int seg;     // context segment, or -1 for the query region

@@ -130,6 +130,35 @@ STAR_API int star_cache_reset_query(star_cache* c);
 STAR_API int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V,
                     void* O, float* LSE, void* stream);
 
+/* RoPE front end ("Star Attention", Phase 1 Step 2: every token keeps its
+ * position ID; anchor tokens keep theirs).  Rotary embedding of
+ * x [B][H][L][D] bf16 into y (y == x allowed): each adjacent pair
+ * (x_2k, x_2k+1) of row t turns by p_t * theta^(-2k/D), p_t = pos[t] when
+ * pos (device, int32 [L]) is given, else pos0 + t.  Angles are formed and
+ * reduced in double, rotated in float32, rounded once to bf16.  D = 64 or
+ * 128 (else STAR_EUNSUPPORTED); theta > 1; B <= 65535; positions >= 0. */
+STAR_API int star_rope(int B, int H, long long L, int D, double theta, const int* pos,
+                       long long pos0, const void* x, void* y, void* stream);
+
+/* Anchor keys of blocks 1..n-1 under a position-ID variant ("Star
+ * Attention", Section 4.1, Table 4): Ka[i-1] = the anchor rows 0..b_a-1 of
+ * K (un-rotated, [B][Hkv][L][D] bf16) rotated at the IDs block i gives its
+ * anchor -- mode 0: 0..b_a-1 (first block, the method); 1: i*b - b_a ..
+ * i*b - 1 (the positions just before block i); 2: pos[(i-1)*b_a + j]
+ * (device int32 [n-1][b_a], e.g. random draws from [0, i*b)).
+ * Ka: [n-1][B][Hkv][b_a][D] bf16, caller-owned.  Nothing to do when n = 1
+ * or b_a = 0. */
+STAR_API int star_anchor_keys(const star_cache* c, int mode, const int* pos, double theta,
+                              const void* K, void* Ka, void* stream);
+
+/* Phase 1 as star_ctx_encode, except that block i >= 1 attends to the
+ * anchor keys Ka[i-1] (from star_anchor_keys) instead of K rows
+ * 0..b_a-1; the anchor's values are V rows 0..b_a-1 as before.  Q and K are
+ * the rotated inputs (star_rope at positions 0..L-1); Ka = NULL is
+ * star_ctx_encode.  The cache receives the rotated K rows of each block. */
+STAR_API int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const void* V,
+                                      const void* Ka, void* O, float* LSE, void* stream);
+
 /* Phase 2 -- query prefill ([P2] Phase 2 Steps 3, 5, 7).  Appends K, V
  * [B][Hkv][lq][D] bf16 to the query region, then every query row r of
  * Q [B][Hq][lq][D] attends to all context segments and to query-region rows

@@ -432,16 +432,25 @@ def anchor_positions(mode: str, n_blocks: int, b: int, b_a: int, given=None) -> 
     raise ValueError(mode)
 
 
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), as float64."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
 def ctx_encode_rope(Q, K, V, b: int, b_a: int, scale: float, anchor_pos, base: float = ROPE_BASE,
-                    rows=None):
+                    rows=None, rotated_bf16: bool = False):
     """Phase 1 on un-rotated Q, K [B, H, L, D] with rotary positions.
 
     Token t of block i is at position t (positions preserved, [P2] Phase 1
     Step 2).  Block 0 attends causally to itself; block i >= 1 attends to the
     whole anchor -- K rows 0..b_a-1 rotated at anchor_pos[i-1] -- and causally
-    to its own block.  V is not rotated.  Returns (O, LSE) for ``rows``
-    (default all), like ``ctx_encode``.
+    to its own block.  V is not rotated.  ``rotated_bf16`` rounds the rotated
+    q and k to bf16 before the attention (the precision of a path whose
+    attention operands are bf16).  Returns (O, LSE) for ``rows`` (default
+    all), like ``ctx_encode``.
     """
+    rnd = round_bf16 if rotated_bf16 else (lambda a: a)
     Bn, Hq, L, D = Q.shape
     Hkv = K.shape[1]
     G = Hq // Hkv
@@ -465,10 +474,11 @@ def ctx_encode_rope(Q, K, V, b: int, b_a: int, scale: float, anchor_pos, base: f
                 kraw = _f64(K[bi, g])
                 kk = np.concatenate([rope(kraw[:b_a], kpos[:b_a], base), rope(kraw[s:s + n], own, base)]) \
                     if i > 0 else rope(kraw[s:s + n], own, base)
+                kk = rnd(kk)
                 vv = _f64(V[bi, g])
                 vv = np.concatenate([vv[:b_a], vv[s:s + n]]) if i > 0 else vv[s:s + n]
                 for h in range(g * G, (g + 1) * G):
-                    q = rope(_f64(Q[bi, h])[t], t, base)
+                    q = rnd(rope(_f64(Q[bi, h])[t], t, base))
                     o, lse = masked_attention(q, kk, vv, mask, scale)
                     O[bi, h, sel] = o
                     LSE[bi, h, sel] = lse

@@ -70,6 +70,13 @@ def test_argument_errors_are_caught_on_the_host(lib):
     p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 1)  # the no-alloc path is bf16 only
     assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *([None] * 10)) == _abi.STAR_EINVAL
     assert b"kv_fp8" in lib.star_last_error()
+    assert lib.star_rope(1, 1, 8, 96, 500000.0, None, 0, None, None, None) == _abi.STAR_EUNSUPPORTED
+    assert lib.star_rope(1, 1, 8, 64, 1.0, None, 0, None, None, None) == _abi.STAR_EINVAL     # theta <= 1
+    assert lib.star_rope(1, 1, 8, 64, 500000.0, None, -1, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_rope(1, 1, 8, 64, 500000.0, None, 0, None, None, None) == _abi.STAR_EINVAL  # NULL x
+    assert lib.star_rope(1, 1, 0, 64, 500000.0, None, 0, None, None, None) == _abi.STAR_OK      # nothing to do
+    assert lib.star_anchor_keys(None, 0, None, 500000.0, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_ctx_encode_anchored(None, None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_cache_destroy(None) == _abi.STAR_OK
     assert lib.star_cache_num_segments(None) == 0
 

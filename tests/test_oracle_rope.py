@@ -150,3 +150,8 @@ def test_planted_position_mistake_is_caught(rng, monkeypatch):
     monkeypatch.setattr(so, "ctx_encode_rope", ignores_anchor_ids)
     with pytest.raises(AssertionError):
         test_ctx_encode_rope_matches_the_augmented_sequence(rng, "previous", 12, 4, 4)
+
+
+def test_round_bf16_is_round_to_nearest_even():
+    x = np.array([1 + 2 ** -8, 1 + 2 ** -8 + 2 ** -20, 1 + 3 * 2 ** -8, -(2 + 2 ** -7), 3.0])
+    np.testing.assert_array_equal(so.round_bf16(x), [1.0, 1 + 2 ** -7, 1 + 2 ** -6, -2.0, 3.0])

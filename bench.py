@@ -321,6 +321,54 @@ def measure_phase1_variants(dev, flush, warmup, steps, world):
     return out
 
 
+def measure_rope(dev, flush, warmup, steps, world):
+    """RoPE front end on the 8B-32K shape: the rotation of Q and K (HBM-bound),
+    and phase 1 on un-rotated inputs with the previous-block anchor IDs
+    (rotation + anchor keys + phase 1 on per-block anchor keys)."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, star_rope, workloads as wl
+    w = wl.get(WORKLOAD)
+    g = torch.Generator(device=dev).manual_seed(w.seed + 11)
+    Q = torch.randn((w.B, w.Hq, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+    K = torch.randn((w.B, w.Hkv, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn((w.B, w.Hkv, w.L, w.D), generator=g, device=dev).to(torch.bfloat16)
+    Qr, Kr = torch.empty_like(Q), torch.empty_like(K)
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, 1, w.scale)
+    nb = cache.num_segments - 1
+    Ka = torch.empty((nb - 1, w.B, w.Hkv, w.b_a, w.D), dtype=torch.bfloat16, device=dev)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    rope_ms, all_ms = [], []
+    for it in range(warmup + steps):
+        flush.flush(7.0)
+        a, b, c = ev(), ev(), ev()
+        a.record(stream)
+        star_rope(Q, out=Qr)
+        star_rope(K, out=Kr)
+        b.record(stream)
+        cache.star_anchor_keys(K, "previous", Ka=Ka)
+        cache.star_ctx_encode(Qr, Kr, V, O, LSE, Ka=Ka)
+        c.record(stream)
+        if it >= warmup:
+            rope_ms.append((a, b))
+            all_ms.append((a, c))
+    torch.cuda.synchronize(dev)
+    t_rope = sum(x.elapsed_time(y) for x, y in rope_ms) / steps
+    t_all = sum(x.elapsed_time(y) for x, y in all_ms) / steps
+    t_rope, t_all = max_over_ranks([t_rope, t_all], dev, world)
+    nbytes = 2 * 2 * (Q.numel() + K.numel())          # read + write, bf16
+    flops, _ = phase1_flops(w)
+    cache.close()
+    del Q, K, V, Qr, Kr, Ka, O, LSE
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "rotation_us": t_rope * 1e3, "rotation_bytes": nbytes,
+            "rotation_gbs": nbytes / (t_rope / 1e3) / 1e9,
+            "phase1_previous_ids_ms": t_all, "ctx_tok_s": world * w.B * w.L / (t_all / 1e3),
+            "phase1_tflops_incl_rope": flops / (t_all / 1e3) / 1e12}
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -488,13 +536,24 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "what": "H2D of Q,K,V from pinned host + star_ctx_encode + D2H of O,LSE"}
 
-    variants = None
-    if not args.no_variants:
-        variants = measure_phase1_variants(dev, flush, args.warmup, min(args.steps, 10), world)
+    def settle():
+        # each further section starts from an idle GPU rather than under the
+        # power and thermal state the section before it left behind
+        torch.cuda.synchronize(dev)
+        time.sleep(1.0)
+
     long_dec = None
     if not args.no_long_decode:
+        settle()
         long_dec = measure_long_decode(dev, flush, args.warmup, args.steps, world)
+        settle()
         long_dec_fp8 = measure_long_decode(dev, flush, args.warmup, args.steps, world, kv_fp8=True)
+    rope = variants = None
+    if not args.no_variants:
+        settle()
+        rope = measure_rope(dev, flush, args.warmup, min(args.steps, 10), world)
+        settle()
+        variants = measure_phase1_variants(dev, flush, args.warmup, min(args.steps, 10), world)
 
     pk = peaks()
     flops, _ = phase1_flops(w)
@@ -531,6 +590,9 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
+    if rope:
+        rope["rotation_frac"] = rope["rotation_gbs"] / pk["hbm_gbs"]
+        line["rope"] = rope
     if variants:
         for v in variants.values():
             # burst peak for a launch of a few ms; a launch of 10+ ms runs under

@@ -489,7 +489,14 @@ void ctx_tc_fill_work(const CacheView& c, int4* out) {
         for (int hp = 0; hp < pairs; ++hp)
           items.push_back({anchor_tiles + qt + 1, make_int4(bg, hp, blk, qt)});
   }
-  std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) { return x.cost > y.cost; });
+  // Blocks one after another (last block first), longest tile first inside a
+  // block: the CTAs that run together share one block's K/V and anchor keys
+  // (measured 1 % faster than one global longest-first order), and the short
+  // tiles of block 0 close the launch.
+  std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) {
+    if (x.v.z != y.v.z) return x.v.z > y.v.z;
+    return x.cost > y.cost;
+  });
   for (size_t i = 0; i < items.size(); ++i) out[i] = items[i].v;
 }
 

@@ -22,7 +22,7 @@ struct star_cache {
   int device;
   int num_sms;
   void* block;              // the one cudaMalloc holding everything below
-  int4* ctx_work;           // phase-1 work list, longest first
+  int4* ctx_work;           // phase-1 work list, block by block, longest tile first
   int n_ctx_work;
   star::DecodeMaps dmaps;   // TMA maps of the cache (built once)
 };
@@ -322,8 +322,8 @@ int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const 
     return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
   cudaError_t e = star::launch_ctx_encode_tc(
       c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
-      static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work,
-      c->scratch.err, static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka));
+      static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work, c->scratch.err,
+      static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka));
   if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
   if (e == cudaSuccess && c->view.ctxK8) e = star::launch_quantize_ctx_fp8(c->view, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");

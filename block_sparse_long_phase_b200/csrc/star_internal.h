@@ -74,6 +74,7 @@ struct Scratch {
 
 // ---- launchers (defined in the .cu files) --------------------------------
 size_t ctx_tc_work_count(const CacheView& c);
+// phase-1 work list (b*Hkv + g, head pair, block, q tile), block by block
 void ctx_tc_fill_work(const CacheView& c, int4* out);
 // Ka (may be null): anchor keys of blocks 1..n-1 as [n-1][B][Hkv][b_a][D];
 // block i >= 1 then reads its anchor keys from Ka[i-1] instead of K rows 0..b_a-1.

@@ -157,3 +157,28 @@ def test_prefill_and_decode_with_rope():
         ref, lref = so.query_attend(q, segs, Kreg, Vreg, np.array([w.lq + t + 1]), w.scale)
         assert_close(dec[t][0], ref, dec[t][1], lref[:, :, 0], f"decode {t}")
     cache.close()
+
+
+def test_phase1_with_rope_full_size_sampled():
+    """8B-32K in the benchmark's launch configuration, previous-block anchor
+    IDs: sampled rows of every block (first, last, tile edges) of two kv groups."""
+    from block_sparse_long_phase_b200 import StarCache
+    w = wl.get("8b-32k")
+    rng = np.random.default_rng(w.seed + 3)
+    x = wl.make_inputs(w, "cuda")
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+    O, LSE = cache.star_ctx_encode_rope(x["Qc"], x["Kc"], x["Vc"], anchor="previous", theta=THETA)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    ap = anchor_ids("previous", w)
+    rows = []
+    for s, n in so.block_table(w.L, w.b):
+        cand = {0, n - 1, 127, 128, n // 2} | set(rng.integers(0, n, 3).tolist())
+        rows += [s + c for c in sorted(cand)]
+    rows = np.array(rows)
+    for g in (0, w.Hkv - 1):
+        hs, gs = slice(g * w.G, (g + 1) * w.G), slice(g, g + 1)
+        ref, lref = so.ctx_encode_rope(x["Qc"][:, hs].cpu(), x["Kc"][:, gs].cpu(), x["Vc"][:, gs].cpu(),
+                                       w.b, w.b_a, w.scale, ap, THETA, rows=rows, rotated_bf16=True)
+        assert_close(O[:, hs][:, :, rows], ref, LSE[:, hs][:, :, rows], lref, f"8b-32k previous kv{g}")
+    cache.close()

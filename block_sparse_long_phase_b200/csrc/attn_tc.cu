@@ -479,22 +479,46 @@ size_t ctx_tc_work_count(const CacheView& c) {
 
 void ctx_tc_fill_work(const CacheView& c, int4* out) {
   const int pairs = (c.G + 1) / 2;
-  struct Item { long long cost; int4 v; };
+  const int BG = c.B * c.Hkv;
+  // Work units (block, batch x kv head), last block first, are packed into
+  // groups whose K/V (the block's rows plus the anchor rows it reads) stays
+  // under kGroupBytes, about two thirds of the 126 MB L2.  Inside a group the
+  // longest tile goes first.  The CTAs that run together then re-read one
+  // group's K/V from L2 instead of streaming every head's from HBM (one
+  // global longest-first order spans all heads of all batch entries: 268 MB
+  // of K/V at four 32K-token sequences), and the short tiles of block 0 close
+  // the launch.
+  constexpr long long kGroupBytes = 80ll << 20;
+  std::vector<int> group((size_t)c.n_seg * BG);
+  int g = 0;
+  long long used = 0;
+  for (int blk = c.n_seg - 1; blk >= 0; --blk) {
+    const long long unit = (seg_len(c, blk) + (blk > 0 ? c.b_a : 0)) * c.D * 2ll * (long long)sizeof(bf16);
+    if (used > 0 && used + unit * BG > kGroupBytes && unit * BG <= kGroupBytes) {
+      ++g;                                   // a block that fits a group of its own is not split
+      used = 0;
+    }
+    for (int bg = 0; bg < BG; ++bg) {
+      if (used > 0 && used + unit > kGroupBytes) {
+        ++g;
+        used = 0;
+      }
+      used += unit;
+      group[(size_t)blk * BG + bg] = g;
+    }
+  }
+  struct Item { int group; long long cost; int4 v; };
   std::vector<Item> items;
   for (int blk = 0; blk < c.n_seg; ++blk) {
     const long long tiles = (seg_len(c, blk) + BM - 1) / BM;
     const long long anchor_tiles = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
     for (int qt = 0; qt < tiles; ++qt)
-      for (int bg = 0; bg < c.B * c.Hkv; ++bg)
+      for (int bg = 0; bg < BG; ++bg)
         for (int hp = 0; hp < pairs; ++hp)
-          items.push_back({anchor_tiles + qt + 1, make_int4(bg, hp, blk, qt)});
+          items.push_back({group[(size_t)blk * BG + bg], anchor_tiles + qt + 1, make_int4(bg, hp, blk, qt)});
   }
-  // Blocks one after another (last block first), longest tile first inside a
-  // block: the CTAs that run together share one block's K/V and anchor keys
-  // (measured 1 % faster than one global longest-first order), and the short
-  // tiles of block 0 close the launch.
   std::stable_sort(items.begin(), items.end(), [](const Item& x, const Item& y) {
-    if (x.v.z != y.v.z) return x.v.z > y.v.z;
+    if (x.group != y.group) return x.group < y.group;
     return x.cost > y.cost;
   });
   for (size_t i = 0; i < items.size(); ++i) out[i] = items[i].v;

@@ -12,8 +12,9 @@
 // and reduced to [-pi, pi] in double (positions reach 2^20 and beyond, where
 // a float angle would be off by a large fraction of a radian), and only the
 // reduced angle goes through sincosf.  HBM-bound: every element is read and
-// written once; a CTA holds the cos/sin of 16 positions in shared memory and
-// applies them to every head of its batch entry.
+// written once; a thread computes the cos/sin of its 4 pairs at one position
+// and applies them to that slice of every head of its batch entry (of every
+// other head at D = 64).
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -24,44 +25,59 @@
 namespace star {
 namespace {
 
-constexpr int kTP = 16;                      // positions per CTA
+// A CTA turns 16 positions of every head: one thread per (position, 16-byte
+// vector) slot at D = 128, two heads side by side at D = 64.  (Four-position
+// CTAs, for a shorter last wave, measured slower: 107 registers, 2 CTAs/SM.)
+template <int D>
+constexpr int kTP = 16;
 constexpr double kTwoPi = 6.283185307179586476925286766559;
 
 template <int D>
 __global__ void __launch_bounds__(256) rope_kernel(const __grid_constant__ RopeJob j) {
-  __shared__ float2 cs[kTP][D / 2];
-  const long long t0 = (long long)blockIdx.x * kTP;
+  // Thread = (position t, 16-byte vector v of 4 pairs); it turns that vector
+  // of every head, so its 4 (cos, sin) pairs are computed once, in registers.
+  constexpr int VPR = D / 8;                 // 16-byte vectors per row
+  constexpr int TV = kTP<D> * VPR;           // (position, vector) slots of a CTA
+  constexpr int HS = 256 / TV;               // heads taken side by side
+  constexpr int kU = 8;                      // loads in flight per thread
+  const int tv = threadIdx.x % TV, hs = threadIdx.x / TV;
+  const int t = tv / VPR, v = tv % VPR;
+  const long long tok = (long long)blockIdx.x * kTP<D> + t;
   const int b = blockIdx.y, grp = blockIdx.z;
-  const int np = (int)(j.n - t0 < kTP ? j.n - t0 : kTP);
-  for (int i = threadIdx.x; i < kTP * (D / 2); i += blockDim.x) {
-    const int t = i / (D / 2), k = i - (i / (D / 2)) * (D / 2);
-    if (t < np) {
-      const long long p = j.pos ? (long long)j.pos[(long long)grp * j.pos_grp + t0 + t]
-                                : j.pos0 + (long long)grp * j.pos0_grp + t0 + t;
-      const double a = (double)p * j.inv_freq[k];
-      const double r = a - kTwoPi * rint(a * (1.0 / kTwoPi));
-      float s, c;
-      sincosf((float)r, &s, &c);
-      cs[t][k] = make_float2(c, s);
-    }
-  }
-  __syncthreads();
-  constexpr int VPR = D / 8;                 // 16-byte vectors (4 pairs) per row
-  const int total = j.H * np * VPR;
-  for (int i = threadIdx.x; i < total; i += blockDim.x) {
-    const int v = i % VPR, r = i / VPR, t = r % np, h = r / np;
-    const long long xrow = (long long)grp * j.x_grp + ((long long)b * j.H + h) * j.x_seq + t0 + t;
-    const long long yrow = (long long)grp * j.y_grp + ((long long)b * j.H + h) * j.y_seq + t0 + t;
-    const uint4 u = *reinterpret_cast<const uint4*>(j.x + xrow * D + v * 8);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[4];
+  if (tok >= j.n) return;
+  const long long p = j.pos ? (long long)j.pos[(long long)grp * j.pos_grp + tok]
+                            : j.pos0 + (long long)grp * j.pos0_grp + tok;
+  float2 cv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = cs[t][v * 4 + e];
-      const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
-      o[e] = pack_bf16(x0 * f.x - x1 * f.y, x0 * f.y + x1 * f.x);
+  for (int e = 0; e < 4; ++e) {
+    const double a = (double)p * j.inv_freq[4 * v + e];
+    const double r = a - kTwoPi * rint(a * (1.0 / kTwoPi));
+    sincosf((float)r, &cv[e].y, &cv[e].x);
+  }
+  const bf16* x = j.x + ((long long)grp * j.x_grp + (long long)b * j.H * j.x_seq + tok) * D + v * 8;
+  bf16* y = j.y + ((long long)grp * j.y_grp + (long long)b * j.H * j.y_seq + tok) * D + v * 8;
+  const long long xs = j.x_seq * D, ys = j.y_seq * D;
+  for (int h0 = hs; h0 < j.H; h0 += kU * HS) {
+    uint4 u[kU];
+#pragma unroll
+    for (int q = 0; q < kU; ++q) {
+      const int h = h0 + q * HS;
+      if (h < j.H) u[q] = *reinterpret_cast<const uint4*>(x + h * xs);
     }
-    *reinterpret_cast<uint4*>(j.y + yrow * D + v * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int q = 0; q < kU; ++q) {
+      const int h = h0 + q * HS;
+      if (h < j.H) {
+        const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __uint_as_float(w[e] << 16), x1 = __uint_as_float(w[e] & 0xffff0000u);
+          o[e] = pack_bf16(x0 * cv[e].x - x1 * cv[e].y, x0 * cv[e].y + x1 * cv[e].x);
+        }
+        *reinterpret_cast<uint4*>(y + h * ys) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
   }
 }
 
@@ -73,7 +89,8 @@ void rope_inv_freq(int D, double base, double* out) {
 
 cudaError_t launch_rope(const RopeJob& j, int D, int B, int groups, cudaStream_t st) {
   if (j.n <= 0 || B <= 0 || groups <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)((j.n + kTP - 1) / kTP), (unsigned)B, (unsigned)groups);
+  const int tp = D == 128 ? kTP<128> : kTP<64>;
+  const dim3 grid((unsigned)((j.n + tp - 1) / tp), (unsigned)B, (unsigned)groups);
   if (D == 128)
     rope_kernel<128><<<grid, 256, 0, st>>>(j);
   else

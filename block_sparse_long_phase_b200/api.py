@@ -218,6 +218,32 @@ class StarCache:
                                                _ptr(O), _ptr(LSE), _stream(Q.device)))
         return O, LSE
 
+    def star_query_prefill_partials(self, Q, K, V, fp32_out=True):
+        """Debug form of :meth:`star_query_prefill`: one partial per context
+        segment plus one for the query region, returned with the outputs.
+
+        Returns ``(O, LSE, Ah, sh, O32)``: Ah [n+1, B, Hq, lq, D] and sh
+        [n+1, B, Hq, lq] float32 (part n is the query region), O32 the merged
+        rows in float32 (None unless ``fp32_out``).  With lq = 1 it is a
+        generation step on the bf16 cache.
+        """
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        lq = Q.shape[2]
+        _need(Q, (B, Hq, lq, D), torch.bfloat16, "Q")
+        _need(K, (B, Hkv, lq, D), torch.bfloat16, "K")
+        _need(V, (B, Hkv, lq, D), torch.bfloat16, "V")
+        P = self.num_segments
+        dev = Q.device
+        O = torch.empty((B, Hq, lq, D), dtype=torch.bfloat16, device=dev)
+        LSE = torch.empty((B, Hq, lq), dtype=torch.float32, device=dev)
+        Ah = torch.empty((P, B, Hq, lq, D), dtype=torch.float32, device=dev)
+        sh = torch.empty((P, B, Hq, lq), dtype=torch.float32, device=dev)
+        O32 = torch.empty((B, Hq, lq, D), dtype=torch.float32, device=dev) if fp32_out else None
+        _abi.check(self.lib.star_query_prefill_partials(
+            self.handle, lq, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(Ah), _ptr(sh),
+            _ptr(O32) if O32 is not None else None, _stream(dev)))
+        return O, LSE, Ah, sh, O32
+
     def star_decode_step(self, q, k, v, o=None, lse=None):
         B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
         _need(q, (B, Hq, 1, D), torch.bfloat16, "q")

@@ -78,6 +78,7 @@ struct CtxTcArgs {
   float* partS;
   PrefillPlan plan;
 };
+static_assert(sizeof(CtxTcArgs) <= 4096, "kernel parameters beyond 4 KB");
 
 SM100_DEV float ex2(float x) {
   float y;
@@ -592,12 +593,17 @@ __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, 
 }
 
 // Merge the chunks' partials of every packed query row and scatter to O / LSE.
+// Debug outputs (null in the normal path): O32, the merged rows in float32;
+// Ah / sh, every chunk's partial in [chunk][B][Hq][lq] row order.
 template <int D>
 __global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq, int n_chunks,
                                                             const float* __restrict__ partA,
                                                             const float* __restrict__ partS,
                                                             bf16* __restrict__ O,
-                                                            float* __restrict__ LSE) {
+                                                            float* __restrict__ LSE,
+                                                            float* __restrict__ O32,
+                                                            float* __restrict__ Ah,
+                                                            float* __restrict__ sh) {
   const int rows_total = c.G * lq;
   const long long gw = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -605,6 +611,9 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq,
   const long long bg = gw / rows_total;
   const int m = (int)(gw - bg * rows_total);
   const int bb = (int)(bg / c.Hkv), g = (int)(bg - (long long)bb * c.Hkv);
+  const int h = g * c.G + m / lq;
+  const int rr = m % lq;
+  const long long orow_i = ((long long)bb * c.Hq + h) * lq + rr;   // row of O / LSE
   float mx = -INFINITY;
   for (int p = 0; p < n_chunks; ++p) mx = fmaxf(mx, partS[(bg * n_chunks + p) * rows_total + m]);
   const float base = mx == -INFINITY ? 0.f : mx;
@@ -615,20 +624,28 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq,
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  const long long prow_stride = (long long)c.B * c.Hq * lq;        // rows per chunk in Ah / sh
   for (int p = 0; p < n_chunks; ++p) {
     const long long r = (bg * n_chunks + p) * rows_total + m;
     const float s = partS[r];
+    if (Ah) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i) Ah[(p * prow_stride + orow_i) * D + lane + 32 * i] = partA[r * D + lane + 32 * i];
+      if (lane == 0) sh[p * prow_stride + orow_i] = s;
+    }
     if (s == -INFINITY) continue;
     const float w = __expf(s - lse);
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] += w * partA[r * D + lane + 32 * i];
   }
-  const int h = g * c.G + m / lq;
-  const int rr = m % lq;
-  bf16* orow = O + (((long long)bb * c.Hq + h) * lq + rr) * D;
+  bf16* orow = O + orow_i * D;
 #pragma unroll
   for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
-  if (lane == 0) LSE[((long long)bb * c.Hq + h) * lq + rr] = lse;
+  if (O32) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) O32[orow_i * D + lane + 32 * i] = acc[i];
+  }
+  if (lane == 0) LSE[orow_i] = lse;
 }
 
 }  // namespace
@@ -638,7 +655,7 @@ int prefill_row_pairs(const CacheView& c, int lq) { return (c.G * lq + 2 * BM - 
 cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, float scale, int lq,
                                     int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, float* O32, float* Ah, float* sh) {
   CtxTcArgs a;
   memset(&a, 0, sizeof(a));
   const unsigned long long qrows = (unsigned long long)c.B * c.Hq * lq;
@@ -668,9 +685,9 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
   const int mgrid = (int)((rows + 3) / 4);
   if (c.D == 128)
-    prefill_merge_kernel<128><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE);
+    prefill_merge_kernel<128><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
   else
-    prefill_merge_kernel<64><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE);
+    prefill_merge_kernel<64><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
   return cudaGetLastError();
 }
 

@@ -83,6 +83,17 @@ star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
   return pl;
 }
 
+// One chunk per context segment and one for the query region: the partials
+// are then exactly the per-segment (A_h, s_h) of the method.
+star::PrefillPlan plan_prefill_per_segment(const star_cache* c, int lq, long long len0) {
+  const star::CacheView& v = c->view;
+  star::PrefillPlan pl{};
+  for (int s = 0; s < v.n_seg; ++s) pl.chunk[s] = {s, 0, (int)star::seg_len(v, s)};
+  pl.chunk[v.n_seg] = {-1, 0, (int)(len0 + lq)};
+  pl.n_chunks = v.n_seg + 1;
+  return pl;
+}
+
 star::DecodePlan plan_decode(const star_cache* c, long long len0) {
   star::DecodePlan pl;
   pl = star::decode_plan(c->view, len0, c->num_sms);
@@ -102,7 +113,9 @@ int validate_params(const star_params* p) {
   if (p->q_cap < 1) return fail(STAR_EINVAL, "q_cap must be >= 1");
   if (p->kv_fp8 != 0 && p->kv_fp8 != 1) return fail(STAR_EINVAL, "kv_fp8 must be 0 or 1");
   if (p->L + p->q_cap + 1 > 0x7fffffffLL) return fail(STAR_EINVAL, "L + q_cap too large");
-  if ((p->L + p->block - 1) / p->block > 0x7fff) return fail(STAR_EINVAL, "too many blocks");
+  if ((p->L + p->block - 1) / p->block > star::kMaxPrefillChunks - 1)
+    return fail(STAR_EUNSUPPORTED, "%lld blocks: at most %d", (p->L + p->block - 1) / p->block,
+                star::kMaxPrefillChunks - 1);
   return STAR_OK;
 }
 
@@ -115,6 +128,33 @@ int set_error(int code, const char* msg) {
 }
 int check_params(const star_params* p) { return validate_params(p); }
 }  // namespace star
+
+namespace {
+// star_query_prefill and its debug form with per-segment partials.
+int query_prefill(star_cache* c, int lq, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                  void* stream, bool per_segment, float* Ah, float* sh, float* O32) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (lq < 1) return fail(STAR_EINVAL, "lq must be >= 1");
+  if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (per_segment && (!Ah || !sh)) return fail(STAR_EINVAL, "NULL partials pointer");
+  if (c->q_len + lq > c->view.q_cap)
+    return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, c->view.q_cap);
+  const star::PrefillPlan pl =
+      per_segment ? plan_prefill_per_segment(c, lq, c->q_len) : plan_prefill(c, lq, c->q_len);
+  cudaError_t e = star::launch_query_prefill_tc(
+      c->view, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
+      static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
+      c->scratch, static_cast<cudaStream_t>(stream), O32, Ah, sh);
+  if (e == cudaSuccess && c->view.qK8)
+    e = star::launch_quantize_qregion_fp8(c->view, static_cast<const bf16*>(K), static_cast<const bf16*>(V),
+                                          (int)c->q_len, lq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_query_prefill launch");
+  c->q_len += lq;
+  return STAR_OK;
+}
+}  // namespace
 
 extern "C" {
 
@@ -394,24 +434,12 @@ int star_anchor_keys(const star_cache* c, int mode, const int* pos, double theta
 
 int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K, const void* V,
                        void* O, float* LSE, void* stream) {
-  if (!c) return fail(STAR_EINVAL, "cache is NULL");
-  if (lq < 1) return fail(STAR_EINVAL, "lq must be >= 1");
-  if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
-    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
-  if (c->q_len + lq > c->view.q_cap)
-    return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, c->view.q_cap);
-  star::PrefillPlan pl = plan_prefill(c, lq, c->q_len);
-  cudaError_t e = star::launch_query_prefill_tc(
-      c->view, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
-      static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
-      c->scratch, static_cast<cudaStream_t>(stream));
-  if (e == cudaSuccess && c->view.qK8)
-    e = star::launch_quantize_qregion_fp8(c->view, static_cast<const bf16*>(K), static_cast<const bf16*>(V),
-                                          (int)c->q_len, lq, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "star_query_prefill launch");
-  c->q_len += lq;
-  return STAR_OK;
+  return query_prefill(c, lq, Q, K, V, O, LSE, stream, false, nullptr, nullptr, nullptr);
+}
+
+int star_query_prefill_partials(star_cache* c, int lq, const void* Q, const void* K, const void* V,
+                                void* O, float* LSE, float* Ah, float* sh, float* O32, void* stream) {
+  return query_prefill(c, lq, Q, K, V, O, LSE, stream, true, Ah, sh, O32);
 }
 
 int star_decode_step(star_cache* c, const void* q, const void* k, const void* v, void* o,

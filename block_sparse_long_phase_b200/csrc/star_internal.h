@@ -105,7 +105,10 @@ struct PrefillChunk {
   int start;   // first row inside the segment
   int len;     // rows
 };
-constexpr int kMaxPrefillChunks = 96;
+// Chunk table size of a prefill launch (kernel parameter): every context
+// segment takes at least one chunk, so a cache has at most kMaxPrefillChunks - 1
+// segments.
+constexpr int kMaxPrefillChunks = 192;
 
 struct PrefillPlan {
   int n_chunks;
@@ -145,7 +148,8 @@ int prefill_row_pairs(const CacheView& c, int lq);   // 256-row pairs of packed 
 cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, float scale, int lq,
                                     int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
-                                    cudaStream_t st);
+                                    cudaStream_t st, float* O32 = nullptr, float* Ah = nullptr,
+                                    float* sh = nullptr);
 
 cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,
                              float* outA, float* outS, cudaStream_t st);

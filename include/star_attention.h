@@ -52,7 +52,7 @@ extern "C" {
 #define STAR_EINVAL       -1   /* bad shape, ratio, b_a > b, null or misaligned pointer */
 #define STAR_ENOSPC       -2   /* query region full (q_cap reached)                      */
 #define STAR_ECUDA        -3   /* CUDA runtime / launch error                            */
-#define STAR_EUNSUPPORTED -4   /* head_dim not 64/128, device not sm_100                 */
+#define STAR_EUNSUPPORTED -4   /* head_dim not 64/128, device not sm_100, > 191 blocks   */
 #define STAR_ENOMEM       -5   /* cudaMalloc failed in star_cache_create                 */
 
 /* Problem statement of one attention layer ([P2] Phase 1 Step 1, Phase 2
@@ -63,7 +63,7 @@ typedef struct {
   int Hkv;          /* key/value heads                                      */
   int D;            /* head dim: 64 or 128                                  */
   long long L;      /* context length, >= 1                                 */
-  int block;        /* block size b >= 1; n = ceil(L / b) blocks            */
+  int block;        /* block size b >= 1; n = ceil(L / b) blocks, n <= 191 */
   int anchor;       /* anchor size b_a, 0 <= b_a <= b (0 = no anchor)       */
   int q_cap;        /* query-region capacity: query tokens + decode steps   */
   float scale;      /* softmax scale; <= 0 selects 1/sqrt(D)                */
@@ -167,6 +167,24 @@ STAR_API int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* 
  * [B][Hq][lq] float32.  STAR_ENOSPC if len0 + lq > q_cap. */
 STAR_API int star_query_prefill(star_cache* c, int lq, const void* Q, const void* K,
                        const void* V, void* O, float* LSE, void* stream);
+
+/* Debug form of star_query_prefill ([P2] Phase 2 Steps 3 and 5, one partial
+ * per partition): the same append, O and LSE, computed with exactly one
+ * partial per context segment and one for the query region, and returned:
+ *   Ah  [n+1][B][Hq][lq][D] float32, sh [n+1][B][Hq][lq] float32 (required):
+ *       part h < n is (A_h, s_h) of context segment h, part n that of the
+ *       query region (rows 0..len0+r for row r); s_h is the natural-log LSE
+ *       of the scaled logits, A_h the normalised local output;
+ *   O32 [B][Hq][lq][D] float32 (optional, NULL = none): the merged rows
+ *       before the bf16 rounding of O.
+ * n = star_cache_num_segments(c) - 1.  With lq = 1 this is a generation step
+ * (append, then attend to every row, itself included) on the bf16 cache.
+ * Slower than star_query_prefill (one CTA per segment); for tests and
+ * inspection.  Errors as star_query_prefill, plus STAR_EINVAL for a NULL Ah
+ * or sh. */
+STAR_API int star_query_prefill_partials(star_cache* c, int lq, const void* Q, const void* K,
+                                         const void* V, void* O, float* LSE, float* Ah, float* sh,
+                                         float* O32, void* stream);
 
 /* Phase 2 -- one generation step ([P2] Phase 2 Step 7).  Appends k, v
  * [B][Hkv][1][D] to the query region, then q [B][Hq][1][D] attends to every

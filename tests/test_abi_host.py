@@ -59,6 +59,11 @@ def test_argument_errors_are_caught_on_the_host(lib):
         assert lib.star_last_error()
     p = _abi.StarParams(1, 4, 2, 96, 1024, 256, 256, 8, 0.0)     # D = 96
     assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
+    p = _abi.StarParams(1, 4, 2, 64, 192 * 64, 64, 64, 8, 0.0)   # 192 blocks: beyond the chunk table
+    assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
+    assert b"192 blocks" in lib.star_last_error()
+    p = _abi.StarParams(1, 4, 2, 64, 191 * 64 + 1, 64, 64, 8, 0.0)  # 192 blocks, the last one ragged
+    assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
     assert lib.star_cache_create(None, ctypes.byref(out)) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(0, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(1, 4, 2000, None, None, None, None, None) == _abi.STAR_EINVAL
@@ -66,6 +71,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.star_ctx_encode(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_decode_step(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_query_prefill(None, 4, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_query_prefill_partials(None, 4, *([None] * 9)) == _abi.STAR_EINVAL
     assert lib.star_cache_segment_fp8(None, 0, None, None, None, None) == _abi.STAR_EINVAL
     p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 1)  # the no-alloc path is bf16 only
     assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *([None] * 10)) == _abi.STAR_EINVAL

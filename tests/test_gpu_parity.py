@@ -95,6 +95,7 @@ TINY_VARIANTS = {
     "batch2": dict(B=2, L=700, b=256, b_a=200, lq=9, T=4),
     "g16": dict(Hq=16, Hkv=1, L=400, b=128, b_a=128, lq=3, T=2),
     "tiny-blocks": dict(L=200, b=40, b_a=40, lq=70, T=3),
+    "max-blocks": dict(L=191 * 48 - 5, b=48, b_a=41, lq=3, T=2),  # 191 blocks, the last one ragged
 }
 
 

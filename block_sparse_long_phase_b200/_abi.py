@@ -23,7 +23,7 @@ EXPORTS = (
     "star_cache_segment", "star_cache_segment_fp8", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_query_prefill_partials", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
-    "star_rope", "star_anchor_keys", "star_ctx_encode_anchored",
+    "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
 )
 
 
@@ -65,6 +65,7 @@ def load(path: str = LIB_PATH):
     lib.star_cache_reset_query.argtypes = [vp]
     lib.star_ctx_encode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_query_prefill.argtypes = [vp, i, vp, vp, vp, vp, vp, vp]
+    lib.star_ctx_encode_host.argtypes = [vp] + [vp] * 10 + [vp]
     lib.star_query_prefill_partials.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_lse_merge.argtypes = [i, ll, i, vp, vp, vp, vp, vp]

@@ -159,6 +159,40 @@ class StarCache:
                                                      _ptr(LSE), _stream(Q.device)))
         return O, LSE
 
+    def star_ctx_encode_host(self, hQ, hK, hV, hO=None, hLSE=None, staging=None):
+        """Phase 1 from host tensors: the copies in and out overlap the encoding.
+
+        ``hQ``, ``hK``, ``hV``: CPU bf16 tensors (pinned for overlap) shaped as
+        for :meth:`star_ctx_encode`; ``hO``, ``hLSE``: CPU outputs (pinned ones
+        are allocated if None).  ``staging``: optional dict of device tensors
+        ``Q, K, V, O, LSE`` reused between calls (allocated if None).
+        Returns ``(hO, hLSE, staging)``; the host outputs are complete once the
+        current stream reaches this point.
+        """
+        B, Hq, Hkv, D, L = self.B, self.Hq, self.Hkv, self.D, self.L
+        shapes = {"Q": (B, Hq, L, D), "K": (B, Hkv, L, D), "V": (B, Hkv, L, D),
+                  "O": (B, Hq, L, D), "LSE": (B, Hq, L)}
+        for name, t in (("hQ", hQ), ("hK", hK), ("hV", hV)):
+            if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 \
+                    or tuple(t.shape) != shapes[name[1:]] or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CPU bf16 tensor of shape {shapes[name[1:]]}")
+        if hO is None:
+            hO = torch.empty(shapes["O"], dtype=torch.bfloat16).pin_memory()
+        if hLSE is None:
+            hLSE = torch.empty(shapes["LSE"], dtype=torch.float32).pin_memory()
+        for name, t, dt in (("hO", hO, torch.bfloat16), ("hLSE", hLSE, torch.float32)):
+            if t.is_cuda or t.dtype != dt or tuple(t.shape) != shapes[name[1:]] or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CPU {dt} tensor of shape {shapes[name[1:]]}")
+        if staging is None:
+            staging = {k: torch.empty(v, dtype=torch.float32 if k == "LSE" else torch.bfloat16,
+                                      device=self.device) for k, v in shapes.items()}
+        for k, v in shapes.items():
+            _need(staging[k], v, torch.float32 if k == "LSE" else torch.bfloat16, k)
+        _abi.check(self.lib.star_ctx_encode_host(
+            self.handle, hQ.data_ptr(), hK.data_ptr(), hV.data_ptr(), hO.data_ptr(), hLSE.data_ptr(),
+            *(_ptr(staging[k]) for k in ("Q", "K", "V", "O", "LSE")), _stream(self.device)))
+        return hO, hLSE, staging
+
     def star_anchor_keys(self, K, anchor="first", theta=ROPE_THETA, Ka=None):
         """Anchor keys of blocks 1..n-1 from un-rotated K [B, Hkv, L, D]:
         ``anchor`` = "first" (IDs 0..b_a-1), "previous" (the b_a positions before

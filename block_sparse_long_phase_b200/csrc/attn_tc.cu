@@ -525,6 +525,36 @@ void ctx_tc_fill_work(const CacheView& c, int4* out) {
   for (size_t i = 0; i < items.size(); ++i) out[i] = items[i].v;
 }
 
+void ctx_tc_fill_units(const CacheView& c, int num_sms, std::vector<CtxUnit>& units, int4* out) {
+  const int pairs = (c.G + 1) / 2;
+  const int BG = c.B * c.Hkv;
+  units.clear();
+  int off = 0;
+  for (int blk = 0; blk < c.n_seg; ++blk) {
+    const long long tiles = (seg_len(c, blk) + BM - 1) / BM;
+    // equal units of at least one wave of CTAs each (the units run on two
+    // streams, so one unit's tail overlaps the next unit's start): the largest
+    // divisor of B*Hkv that keeps a unit at num_sms CTAs or more
+    const long long per_bg = tiles * pairs;
+    int parts = 1;
+    for (int d = 1; d <= BG; ++d)
+      if (BG % d == 0 && per_bg * (BG / d) >= num_sms) parts = d;
+    for (int k = 0; k < parts; ++k) {
+      CtxUnit u;
+      u.blk = blk;
+      u.bg0 = (int)((long long)BG * k / parts);
+      u.bg1 = (int)((long long)BG * (k + 1) / parts);
+      u.off = off;
+      // longest tile (last one, most K/V tiles) first
+      for (long long qt = tiles - 1; qt >= 0; --qt)
+        for (int bg = u.bg0; bg < u.bg1; ++bg)
+          for (int hp = 0; hp < pairs; ++hp) out[off++] = make_int4(bg, hp, blk, (int)qt);
+      u.n = off - u.off;
+      units.push_back(u);
+    }
+  }
+}
+
 cudaError_t attn_tc_prepare(int D) {
   cudaError_t e;
   if (D == 128) {

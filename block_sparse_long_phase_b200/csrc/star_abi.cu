@@ -25,6 +25,12 @@ struct star_cache {
   int4* ctx_work;           // phase-1 work list, block by block, longest tile first
   int n_ctx_work;
   star::DecodeMaps dmaps;   // TMA maps of the cache (built once)
+  // star_ctx_encode_host: the same work cut into pipeline units, and the copy
+  // streams and events, created on its first call
+  std::vector<star::CtxUnit> units;
+  int4* unit_work;
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_comp = nullptr;
+  std::vector<cudaEvent_t> events;     // start, end, compute done, then (input ready, output ready) per unit
 };
 
 namespace {
@@ -202,6 +208,8 @@ int star_cache_create(const star_params* p, star_cache** out) {
   std::vector<int4> work(star::ctx_tc_work_count(v));
   star::ctx_tc_fill_work(v, work.data());
   c->n_ctx_work = (int)work.size();
+  std::vector<int4> unit_work(work.size());
+  star::ctx_tc_fill_units(v, c->num_sms, c->units, unit_work.data());
 
   const long long kv_ctx = (long long)p->B * p->Hkv * p->L * p->D;        // elements
   const long long kv_q = (long long)p->B * p->Hkv * p->q_cap * p->D;
@@ -214,6 +222,7 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const size_t o_t = take(n_tickets * 4);
   const size_t o_e = take(sizeof(int));
   const size_t o_w = take(work.size() * sizeof(int4));
+  const size_t o_uw = take(unit_work.size() * sizeof(int4));
   const bool fp8 = p->kv_fp8 != 0;
   const long long ctx_rows = (long long)p->B * p->Hkv * p->L;
   const size_t o_k8 = fp8 ? take(kv_ctx) : 0, o_v8 = fp8 ? take(kv_ctx) : 0;
@@ -242,6 +251,7 @@ int star_cache_create(const star_params* p, star_cache** out) {
   c->scratch.partS_elems = partS;
   c->scratch.n_tickets = (int)n_tickets;
   c->ctx_work = reinterpret_cast<int4*>(base + o_w);
+  c->unit_work = reinterpret_cast<int4*>(base + o_uw);
   v.ctxK8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_k8) : nullptr;
   v.ctxV8 = fp8 ? reinterpret_cast<uint8_t*>(base + o_v8) : nullptr;
   v.ctxKs = fp8 ? reinterpret_cast<float*>(base + o_ks) : nullptr;
@@ -257,6 +267,8 @@ int star_cache_create(const star_params* p, star_cache** out) {
   if (e == cudaSuccess) e = cudaMemset(c->scratch.err, 0, sizeof(int));
   if (e == cudaSuccess)
     e = cudaMemcpy(c->ctx_work, work.data(), work.size() * sizeof(int4), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(c->unit_work, unit_work.data(), unit_work.size() * sizeof(int4), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(c->block);
     delete c;
@@ -283,6 +295,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
 int star_cache_destroy(star_cache* c) {
   if (!c) return STAR_OK;
   cudaError_t e = cudaDeviceSynchronize();
+  for (cudaEvent_t ev : c->events) cudaEventDestroy(ev);
+  if (c->s_in) cudaStreamDestroy(c->s_in);
+  if (c->s_out) cudaStreamDestroy(c->s_out);
+  if (c->s_comp) cudaStreamDestroy(c->s_comp);
   cudaError_t f = cudaFree(c->block);
   delete c;
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
@@ -374,6 +390,83 @@ int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const 
 int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
                     float* LSE, void* stream) {
   return star_ctx_encode_anchored(c, Q, K, V, nullptr, O, LSE, stream);
+}
+
+int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const void* hV, void* hO,
+                         float* hLSE, void* Q, void* K, void* V, void* O, float* LSE, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (!hQ || !hK || !hV || !hO || !hLSE || !Q || !K || !V || !O || !LSE)
+    return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return fail(STAR_EINVAL, "device tensor pointers must be 16-byte aligned");
+  const star::CacheView& w = c->view;
+  cudaError_t e = cudaSuccess;
+  if (!c->s_in) {
+    e = cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking);
+    for (size_t i = 0; e == cudaSuccess && i < 3 + 2 * c->units.size(); ++i) {
+      cudaEvent_t ev;
+      e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+      if (e == cudaSuccess) c->events.push_back(ev);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "copy streams");
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev_start = c->events[0], ev_end = c->events[1], ev_comp = c->events[2];
+  // the device buffers are free once the work before this call on `stream` is done
+  e = cudaEventRecord(ev_start, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->s_in, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->s_out, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->s_comp, ev_start, 0);
+  const size_t row_b = (size_t)w.D * sizeof(bf16), row_l = sizeof(float);
+  // rows [start, start + len) of heads [h0, h1) of batch entry bb of a [B][H][L] tensor of rb-byte rows
+  auto rows2d = [&](void* dst, const void* src, int H, int bb, int h0, int h1, long long start, long long len,
+                    size_t rb, cudaMemcpyKind kind, cudaStream_t s) {
+    const size_t pit = (size_t)w.L * rb;
+    const size_t o = (((size_t)bb * H + h0) * w.L + start) * rb;
+    return cudaMemcpy2DAsync(static_cast<char*>(dst) + o, pit, static_cast<const char*>(src) + o, pit,
+                             (size_t)len * rb, (size_t)(h1 - h0), kind, s);
+  };
+  for (size_t u = 0; u < c->units.size() && e == cudaSuccess; ++u) {
+    const star::CtxUnit& un = c->units[u];
+    const long long start = (long long)un.blk * w.b, len = star::seg_len(w, un.blk);
+    cudaEvent_t ev_in = c->events[3 + 2 * u], ev_out = c->events[4 + 2 * u];
+    const cudaStream_t cs = (u & 1) ? c->s_comp : st;      // units alternate between two compute streams
+    // inputs of the unit, one 2-D copy per batch entry it touches
+    for (int bb = un.bg0 / w.Hkv; bb * w.Hkv < un.bg1 && e == cudaSuccess; ++bb) {
+      const int g0 = std::max(un.bg0, bb * w.Hkv) - bb * w.Hkv, g1 = std::min(un.bg1, (bb + 1) * w.Hkv) - bb * w.Hkv;
+      e = rows2d(Q, hQ, w.Hq, bb, g0 * w.G, g1 * w.G, start, len, row_b, cudaMemcpyHostToDevice, c->s_in);
+      if (e == cudaSuccess) e = rows2d(K, hK, w.Hkv, bb, g0, g1, start, len, row_b, cudaMemcpyHostToDevice, c->s_in);
+      if (e == cudaSuccess) e = rows2d(V, hV, w.Hkv, bb, g0, g1, start, len, row_b, cudaMemcpyHostToDevice, c->s_in);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in, c->s_in);
+    // the unit's tiles (their anchor rows came with block 0's units, earlier on the same copy stream)
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ev_in, 0);
+    if (e == cudaSuccess)
+      e = star::launch_ctx_encode_tc(w, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+                                     static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE,
+                                     c->unit_work + un.off, un.n, c->scratch.err, cs, nullptr);
+    if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out, cs);
+    // outputs of the unit
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->s_out, ev_out, 0);
+    for (int bb = un.bg0 / w.Hkv; bb * w.Hkv < un.bg1 && e == cudaSuccess; ++bb) {
+      const int g0 = std::max(un.bg0, bb * w.Hkv) - bb * w.Hkv, g1 = std::min(un.bg1, (bb + 1) * w.Hkv) - bb * w.Hkv;
+      e = rows2d(hO, O, w.Hq, bb, g0 * w.G, g1 * w.G, start, len, row_b, cudaMemcpyDeviceToHost, c->s_out);
+      if (e == cudaSuccess)
+        e = rows2d(hLSE, LSE, w.Hq, bb, g0 * w.G, g1 * w.G, start, len, row_l, cudaMemcpyDeviceToHost, c->s_out);
+    }
+  }
+  // the caller's stream takes over once every unit's tiles are done
+  if (e == cudaSuccess) e = cudaEventRecord(ev_comp, c->s_comp);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_comp, 0);
+  if (e == cudaSuccess && w.ctxK8) e = star::launch_quantize_ctx_fp8(w, st);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_end, c->s_out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_end, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode_host");
+  c->q_len = 0;
+  return STAR_OK;
 }
 
 int star_rope(int B, int H, long long L, int D, double theta, const int* pos, long long pos0, const void* x,

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 namespace star {
 
 typedef __nv_bfloat16 bf16;
@@ -76,6 +78,14 @@ struct Scratch {
 size_t ctx_tc_work_count(const CacheView& c);
 // phase-1 work list (b*Hkv + g, head pair, block, q tile), block by block
 void ctx_tc_fill_work(const CacheView& c, int4* out);
+// Phase-1 work cut into pipeline units for copies overlapped with compute: a
+// unit is (block, batch x kv head range [bg0, bg1)), its items a contiguous
+// run [off, off + n) of the list, longest tile first; units run block 0 first.
+struct CtxUnit {
+  int blk, bg0, bg1;
+  int off, n;
+};
+void ctx_tc_fill_units(const CacheView& c, int num_sms, std::vector<CtxUnit>& units, int4* out);
 // Ka (may be null): anchor keys of blocks 1..n-1 as [n-1][B][Hkv][b_a][D];
 // block i >= 1 then reads its anchor keys from Ka[i-1] instead of K rows 0..b_a-1.
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,

@@ -140,6 +140,29 @@ STAR_API int star_ctx_encode(star_cache* c, const void* Q, const void* K, const 
 STAR_API int star_rope(int B, int H, long long L, int D, double theta, const int* pos,
                        long long pos0, const void* x, void* y, void* stream);
 
+/* Phase 1 from and to HOST memory ([P2] Phase 1 Steps 1-5): star_ctx_encode
+ * with the host->device copies of Q, K, V and the device->host copies of O,
+ * LSE overlapped with the encoding.  The blocks are encoded in order 0..n-1,
+ * each in one or more units of (batch x kv head) ranges; a unit's rows are
+ * copied in on one copy stream while earlier units compute, and its O / LSE
+ * rows are copied out on another while later units compute (block 0's units
+ * come first, since every later block reads its anchor rows).
+ *   hQ, hK, hV   host inputs, same layout as star_ctx_encode's Q, K, V
+ *   hO, hLSE     host outputs, same layout as O, LSE
+ *   Q, K, V, O, LSE  device buffers of the same shapes (caller-owned,
+ *                16-byte aligned): the staging copies, left holding the
+ *                inputs and outputs
+ * Host buffers should be page-locked (cudaHostAlloc, or a pinned tensor):
+ * with pageable memory the copies are still correct but not overlapped.
+ * Results are identical, bit for bit, to star_ctx_encode on the same inputs.
+ * Asynchronous on `stream`: work already on `stream` finishes before the
+ * device buffers are written, and `stream` reaches completion only after the
+ * host outputs are written.  The first call creates two copy streams and
+ * their events (kept until star_cache_destroy). */
+STAR_API int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const void* hV,
+                                  void* hO, float* hLSE, void* Q, void* K, void* V, void* O,
+                                  float* LSE, void* stream);
+
 /* Anchor keys of blocks 1..n-1 under a position-ID variant ("Star
  * Attention", Section 4.1, Table 4): Ka[i-1] = the anchor rows 0..b_a-1 of
  * K (un-rotated, [B][Hkv][L][D] bf16) rotated at the IDs block i gives its

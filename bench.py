@@ -277,6 +277,77 @@ def measure_long_decode(dev, flush, warmup, steps, world, kv_fp8=False):
     return w, t_ms * 1e3
 
 
+CONFIGS = ["tiny", "8b-128k-needle", "70b-128k", "70b-128k-b4", "8b-1m"]
+
+
+def measure_configs(dev, flush, warmup, steps, world, dec_steps=8):
+    """Every other configuration of the metric (8B-32K is the main line): phase 1,
+    the query prefill and the first ``dec_steps`` decode steps, each timed on its
+    own with L2 flushed before it; phase-1 launches are ``steps`` per config after
+    ``warmup`` (the 1M-token launch takes seconds)."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+    pk = peaks()
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    for name in CONFIGS:
+        w = wl.get(name)
+        x = wl.make_inputs(w, dev)
+        cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+        O = torch.empty_like(x["Qc"])
+        LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+        Oq = torch.empty_like(x["Qq"])
+        LSEq = torch.empty((w.B, w.Hq, w.lq), dtype=torch.float32, device=dev)
+        od = torch.empty((w.B, w.Hq, 1, w.D), dtype=torch.bfloat16, device=dev)
+        lsed = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+        T = min(w.T, dec_steps)
+        enc, pre, dec = [], [], []
+        for it in range(warmup + steps):
+            flush.flush(8.0)
+            a, b = ev(), ev()
+            a.record(stream)
+            cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"], O, LSE)
+            b.record(stream)
+            flush.flush(9.0)
+            c, d = ev(), ev()
+            c.record(stream)
+            cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"], Oq, LSEq)
+            d.record(stream)
+            steps_ev = []
+            for t in range(T):
+                flush.flush(10.0)
+                e0, e1 = ev(), ev()
+                e0.record(stream)
+                cache.star_decode_step(x["qd"][t], x["kd"][t], x["vd"][t], od, lsed)
+                e1.record(stream)
+                steps_ev.append((e0, e1))
+            if it >= warmup:
+                enc.append((a, b))
+                pre.append((c, d))
+                dec.extend(steps_ev)
+        torch.cuda.synchronize(dev)
+        t_enc = sum(a.elapsed_time(b) for a, b in enc) / len(enc)
+        t_pre = sum(a.elapsed_time(b) for a, b in pre) / len(pre)
+        t_dec = sum(a.elapsed_time(b) for a, b in dec) / len(dec)
+        t_enc, t_pre, t_dec = max_over_ranks([t_enc, t_pre, t_dec], dev, world)
+        flops, _ = phase1_flops(w)
+        dbytes = sum(decode_bytes(w, t) for t in range(T)) / T
+        tf = flops / (t_enc / 1e3) / 1e12
+        gbs = dbytes / (t_dec / 1e3) / 1e9
+        out[name] = {
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L, "block": w.b, "anchor": w.b_a, "lq": w.lq,
+            "phase1_ms": t_enc, "ctx_tok_s": world * w.B * w.L / (t_enc / 1e3), "tflops": tf,
+            "frac": tf / pk["bf16_tflops"],
+            "frac_sustained": tf / pk["bf16_tflops_sustained"] if pk["bf16_tflops_sustained"] else None,
+            "prefill_ms": t_pre, "decode_steps_timed": T * steps, "decode_us": t_dec * 1e3,
+            "decode_tok_s": world * w.B / (t_dec / 1e3), "decode_gbs": gbs, "decode_frac": gbs / pk["hbm_gbs"]}
+        cache.close()
+        del x, O, LSE, Oq, LSEq
+        torch.cuda.empty_cache()
+    return out
+
+
 PHASE1_VARIANTS = {
     # anchor shorter than the block (the pages' anchor-size sweep), ragged last block, batch 4
     "8b-32k-anchor2k": dict(b_a=2048),
@@ -432,6 +503,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-long-decode", action="store_true",
                     help="skip the decode measurement at 128K context")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip phase 1 / prefill / decode on the other four configurations")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the phase-1 variants (anchor shorter than the block, ragged context, batch 4)")
     args = ap.parse_args()
@@ -544,6 +617,10 @@ def main():
         long_dec = measure_long_decode(dev, flush, args.warmup, args.steps, world)
         settle()
         long_dec_fp8 = measure_long_decode(dev, flush, args.warmup, args.steps, world, kv_fp8=True)
+    configs = None
+    if not args.no_configs:
+        settle()
+        configs = measure_configs(dev, flush, args.warmup, min(args.steps, 3), world)
     rope = variants = None
     if not args.no_variants:
         settle()
@@ -589,6 +666,8 @@ def main():
     if rope:
         rope["rotation_frac"] = rope["rotation_gbs"] / pk["hbm_gbs"]
         line["rope"] = rope
+    if configs:
+        line["configs"] = configs
     if variants:
         for v in variants.values():
             # burst peak for a launch of a few ms; a launch of 10+ ms runs under

@@ -658,7 +658,8 @@ def main():
                      "kernel": "phase-1 context encode", "flops_per_launch": flops,
                      "peak_source": pk["source"] + " burst bf16 dense"},
         "clocks": clk,
-        "gpu_launches": args.steps * (1 + 2 + w.T),
+        # per step: phase 1 (1 launch), prefill (append, tile kernel, merge: 3), one per decode step
+        "gpu_launches": args.steps * (1 + 3 + w.T),
         "wall_s_timed_region": wall,
     }
     if e2e:

@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
 }  // namespace
 
 // Work list for the tensor-core phase-1 kernel: (b*Hkv + g, head pair, block,
-// q tile) for every 128-row tile, longest (most K/V tiles) first.
+// q tile) for every 128-row tile; the order is set by ctx_tc_fill_work below.
 size_t ctx_tc_work_count(const CacheView& c) {
   const int pairs = (c.G + 1) / 2;
   size_t n = 0;

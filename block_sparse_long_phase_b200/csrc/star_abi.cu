@@ -22,7 +22,7 @@ struct star_cache {
   int device;
   int num_sms;
   void* block;              // the one cudaMalloc holding everything below
-  int4* ctx_work;           // phase-1 work list, block by block, longest tile first
+  int4* ctx_work;           // phase-1 work list: L2-sized groups of blocks, longest tile first
   int n_ctx_work;
   star::DecodeMaps dmaps;   // TMA maps of the cache (built once)
   // star_ctx_encode_host: the same work cut into pipeline units, and the copy

@@ -18,11 +18,12 @@
 //              of the kv group are the M rows of a 16x8x16 bf16 MMA (rows G..15
 //              zero), online softmax in base 2, fp32 accumulation.
 // When a span ends a (batch, kv head) piece, the consumer warps combine their
-// states in shared memory into one partial (A, s) of that piece; the CTA that
-// holds the piece's last cached row also folds in the new token (attended
-// from its input k, v, which it appends to the query region).  The last CTA
+// states in shared memory into one partial (A, s) of that piece.  The last CTA
 // of a (batch, kv head) to finish -- an atomic ticket, no CTA ever waits for
-// another -- merges that head's partials and writes o and lse.
+// another -- merges that head's partials together with the new token's own
+// part (score q.k, value v, computed on the spot from the step's inputs) and
+// writes o and lse.  The producer warp appends the token's k, v to the query
+// region (a row no reader of this launch touches) after its last stage.
 #include <cuda_bf16.h>
 #include <stdio.h>
 #include <algorithm>
@@ -293,6 +294,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       if (broke)
         for (int k = 0; k < S::NST; ++k)
           if (last_use[k] >= 0) mbar_wait(smem_u32(&bar_full[k]), last_use[k] & 1);
+    }
+    __syncwarp();
+    // The new token's row of the query region (row len0, which no reader of
+    // this launch touches) and its FP8 copy for the steps after this one,
+    // written by the whole warp once its last stage is issued: off the path
+    // the step's time depends on.
+    if (!aborted()) {
+      for (int bg = blockIdx.x; bg < c.B * c.Hkv; bg += a.ncta) {
+        const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+        const long long qo = q_row_offset(c, bb, g, a.len0);
+        const uint4* kn = reinterpret_cast<const uint4*>(a.k + (long long)bg * D);
+        const uint4* vn = reinterpret_cast<const uint4*>(a.v + (long long)bg * D);
+        if (lane < D / 8) reinterpret_cast<uint4*>(c.qK + qo)[lane] = kn[lane];
+        else if (lane >= 16 && lane < 16 + D / 8) reinterpret_cast<uint4*>(c.qV + qo)[lane - 16] = vn[lane - 16];
+        if (FP8) {
+          const long long qrow = (long long)bg * c.q_cap + a.len0;
+          quantize_row_warp<D>(a.k + (long long)bg * D, c.qK8 + qrow * D, c.qKs + qrow, lane);
+          quantize_row_warp<D>(a.v + (long long)bg * D, c.qV8 + qrow * D, c.qVs + qrow, lane);
+        }
+      }
     }
     return;   // the producer takes part in no named barrier
   }
@@ -566,22 +587,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     }
   };
 
-  // [B*Hkv] rows of each (batch, kv head) folded into parts (the new token
-  // counts as one): the CTA that completes rpb + 1 rows merges
+  // [B*Hkv] cached rows of each (batch, kv head) folded into parts: the CTA
+  // that completes rpb rows merges
   unsigned* const done = a.tickets;
-  const int newslot = a.maxp - 1;                 // the new token's part
 
   // ---- merge of bg's parts: one per CTA whose span holds rows of bg (slots
-  // 0..nspan-1) and the new token (slot maxp-1).  A thread owns one float4
-  // column of one row and every npg-th part: it loads their A_h and s_h
-  // together (one L2 round trip), folds them with a running maximum, and
-  // the npg threads of a column combine through shared memory. -------------
+  // 0..nspan-1), and the new token.  A thread owns one float4 column of one
+  // row and every npg-th part: it loads their A_h and s_h together with its
+  // slices of q, k and v (one round trip), folds the parts with a running
+  // maximum, and the npg threads of a column combine through shared memory.
+  // The row's D/4 consecutive threads (one warp, or half of one at D = 64)
+  // sum q.k by shuffles; the npg == 0 thread folds the new token in. -------
   auto merge_bg = [&](int bg) {
     const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
     const long long R = (long long)c.B * c.Hkv * a.rpb;
     const int nspan = cta_of((long long)bg * a.rpb + a.rpb - 1, R, a.ncta) - cta_of((long long)bg * a.rpb, R, a.ncta) + 1;
-    const int cnt = nspan + 1;
-    auto slot_of = [&](int p) { return p < nspan ? p : newslot; };
+    const int cnt = nspan;
+    const bf16* kn = a.k + (long long)bg * D;
+    const bf16* vn = a.v + (long long)bg * D;
     constexpr int NT = 32 * NCW;
     constexpr int KMAX = 11;
     const int nout = G * (D / 4);
@@ -599,6 +622,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       const long long pstride = (long long)G * D / 4;
       float M = -INFINITY, L = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      // the new token: this thread's 4 elements of q_r . k, and of v
+      uint2 q2 = make_uint2(0u, 0u), k2 = make_uint2(0u, 0u), v2 = make_uint2(0u, 0u);
+      if (active) {
+        q2 = *reinterpret_cast<const uint2*>(a.q + ((long long)bb * c.Hq + (long long)g * G + r) * D + 4 * d4);
+        k2 = *reinterpret_cast<const uint2*>(kn + 4 * d4);
+        v2 = *reinterpret_cast<const uint2*>(vn + 4 * d4);
+      }
       for (int p0 = 0; p0 < cnt; p0 += KMAX * npg) {
         float4 v[KMAX];
         float sp[KMAX];
@@ -606,8 +636,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         for (int k = 0; k < KMAX; ++k) {
           const int p = p0 + pg + k * npg;
           const bool ok = active && p < cnt;
-          v[k] = ok ? __ldcg(pa + slot_of(p) * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
-          sp[k] = ok ? __ldcg(ps + (long long)slot_of(p) * G) : -INFINITY;
+          v[k] = ok ? __ldcg(pa + p * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+          sp[k] = ok ? __ldcg(ps + (long long)p * G) : -INFINITY;
         }
         float Mn = M;
 #pragma unroll
@@ -630,6 +660,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           }
           M = Mn;
         }
+      }
+      // (every thread takes part in the shuffles: the groups of D/4 threads are
+      // wholly active or wholly idle, nb * npg being a multiple of D/4)
+      float qk = __uint_as_float(q2.x << 16) * __uint_as_float(k2.x << 16) +
+                 __uint_as_float(q2.x & 0xffff0000u) * __uint_as_float(k2.x & 0xffff0000u) +
+                 __uint_as_float(q2.y << 16) * __uint_as_float(k2.y << 16) +
+                 __uint_as_float(q2.y & 0xffff0000u) * __uint_as_float(k2.y & 0xffff0000u);
+#pragma unroll
+      for (int off = D / 8; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
+      if (active && pg == 0) {
+        const float sn = qk * a.scale_log2 * kLn2;  // natural-log units, like s_h
+        const float Mn = fmaxf(M, sn);
+        const float al = M == -INFINITY ? 0.f : __expf(M - Mn);
+        const float wk = __expf(sn - Mn);
+        L = L * al + wk;
+        acc.x = acc.x * al + wk * __uint_as_float(v2.x << 16);
+        acc.y = acc.y * al + wk * __uint_as_float(v2.x & 0xffff0000u);
+        acc.z = acc.z * al + wk * __uint_as_float(v2.y << 16);
+        acc.w = acc.w * al + wk * __uint_as_float(v2.y & 0xffff0000u);
+        M = Mn;
       }
       if (active) {
         red[pg * nb + (oi - ob)] = acc;
@@ -671,7 +721,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
   auto complete = [&](int bg, int rows) {
     named_sync(1, 32 * NCW);
     if (ctid == 0)
-      s_last = atom_add_acq_rel_gpu(&done[bg], (unsigned)rows) + (unsigned)rows == (unsigned)a.rpb + 1u;
+      s_last = atom_add_acq_rel_gpu(&done[bg], (unsigned)rows) + (unsigned)rows == (unsigned)a.rpb;
     named_sync(1, 32 * NCW);
     if (s_last) merge_bg(bg);
   };
@@ -738,36 +788,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     cur_bg = -1;
     complete(bg, rows);
   };
-
-  // ---- the new token of bg = this CTA's index (+ k ncta): its own part (score
-  // q.k per head, value v) and its row of the query region (row len0, which
-  // no reader of this launch touches) ------------------------------------------
-  for (int bg = blockIdx.x; bg < c.B * c.Hkv; bg += a.ncta) {
-    const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
-    const bf16* kn = a.k + (long long)bg * D;
-    const bf16* vn = a.v + (long long)bg * D;
-    for (int r = cw; r < G; r += NCW) {
-      const bf16* qr = a.q + (((long long)bb * c.Hq + (long long)g * G + r) * D);
-      float acc = 0.f;
-      for (int d = lane; d < D; d += 32) acc += __bfloat162float(qr[d]) * __bfloat162float(kn[d]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (lane == 0) a.partS[((long long)bg * a.maxp + newslot) * G + r] = acc * a.scale_log2 * kLn2;
-    }
-    for (int i = ctid; i < G * D; i += 32 * NCW)
-      a.partA[(((long long)bg * a.maxp + newslot) * G) * D + i] = __bfloat162float(vn[i % D]);
-    if (ctid < D / 8) {
-      const long long qo = q_row_offset(c, bb, g, a.len0);
-      reinterpret_cast<uint4*>(c.qK + qo)[ctid] = reinterpret_cast<const uint4*>(kn)[ctid];
-      reinterpret_cast<uint4*>(c.qV + qo)[ctid] = reinterpret_cast<const uint4*>(vn)[ctid];
-    }
-    if (FP8 && cw < 2) {                        // its FP8 copy, for the steps after this one
-      const long long qrow = (long long)bg * c.q_cap + a.len0;
-      if (cw == 0) quantize_row_warp<D>(kn, c.qK8 + qrow * D, c.qKs + qrow, lane);
-      else quantize_row_warp<D>(vn, c.qV8 + qrow * D, c.qVs + qrow, lane);
-    }
-    complete(bg, 1);
-  }
 
   for (int st = 0;; ++st) {
     const int slot = st % S::NST, use = st / S::NST;

@@ -84,12 +84,18 @@ struct DecodeArgs {
   int* err;
 };
 
+// Row indices stay below 2^31 (checked when the cache is made), so both
+// quotients below divide a numerator under 2^53 by at most 2^31.  They are
+// taken in double, which is exact there: the rounding error of the quotient
+// is below 1 / divisor, the least distance of a non-integer quotient from an
+// integer, so its floor is the integer quotient.  (A 64-bit integer division
+// costs several times as long, ahead of the first TMA load.)
 __device__ __forceinline__ long long span_start(long long i, long long R, int n) {
-  return i * R / n;
+  return (long long)floor((double)(i * R) / (double)n);
 }
 // CTA whose span holds row x (largest i with span_start(i) <= x).
 __device__ __forceinline__ int cta_of(long long x, long long R, int n) {
-  return (int)(((x + 1) * n - 1) / R);
+  return (int)floor((double)((x + 1) * n - 1) / (double)R);
 }
 
 // Release the partials this CTA wrote (ordered before by the consumer barrier,
@@ -225,12 +231,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         long long n = 0;
         bool ctx = false;
         if (have) {
-          bg = (int)(x / a.rpb);
+          bg = (int)((unsigned)x / (unsigned)a.rpb);
           const long long off = x - (long long)bg * a.rpb;         // key index within bg
           const long long run_end = ((long long)bg + 1) * a.rpb < x1 ? ((long long)bg + 1) * a.rpb : x1;
           long long region_end;
           if (off < c.L) {
-            const int seg = (int)(off / c.b);
+            const int seg = (int)((unsigned)off / (unsigned)c.b);
             const long long len = seg_len(c, seg);
             region_end = (long long)seg * c.b + len;
             row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * len + (off - (long long)seg * c.b));

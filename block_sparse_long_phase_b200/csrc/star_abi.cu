@@ -119,6 +119,8 @@ int validate_params(const star_params* p) {
   if (p->q_cap < 1) return fail(STAR_EINVAL, "q_cap must be >= 1");
   if (p->kv_fp8 != 0 && p->kv_fp8 != 1) return fail(STAR_EINVAL, "kv_fp8 must be 0 or 1");
   if (p->L + p->q_cap + 1 > 0x7fffffffLL) return fail(STAR_EINVAL, "L + q_cap too large");
+  if ((long long)p->B * p->Hkv * (p->L + p->q_cap) >= 0x7fffffffLL)
+    return fail(STAR_EUNSUPPORTED, "B * Hkv * (L + q_cap) cached rows must stay below 2^31");
   if ((p->L + p->block - 1) / p->block > star::kMaxPrefillChunks - 1)
     return fail(STAR_EUNSUPPORTED, "%lld blocks: at most %d", (p->L + p->block - 1) / p->block,
                 star::kMaxPrefillChunks - 1);

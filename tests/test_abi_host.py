@@ -64,6 +64,9 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert b"192 blocks" in lib.star_last_error()
     p = _abi.StarParams(1, 4, 2, 64, 191 * 64 + 1, 64, 64, 8, 0.0)  # 192 blocks, the last one ragged
     assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
+    p = _abi.StarParams(1024, 8, 8, 64, 1 << 18, 1 << 12, 1 << 12, 8, 0.0)  # 2^31 cached rows
+    assert lib.star_cache_create(ctypes.byref(p), ctypes.byref(out)) == _abi.STAR_EUNSUPPORTED
+    assert b"2^31" in lib.star_last_error()
     assert lib.star_cache_create(None, ctypes.byref(out)) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(0, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(1, 4, 2000, None, None, None, None, None) == _abi.STAR_EINVAL

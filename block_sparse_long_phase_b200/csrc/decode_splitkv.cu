@@ -826,7 +826,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
 }  // namespace
 
 int decode_max_partials(const CacheView& c, int ncta) {
-  // spans that touch one (batch, kv head), + the new token's part
+  // spans that can touch one (batch, kv head): ceil(ncta / (B * Hkv)), one
+  // more where a span straddles two of them, and spare slots
   const int bgs = c.B * c.Hkv;
   return (ncta + bgs - 1) / bgs + 3;
 }

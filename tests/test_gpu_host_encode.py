@@ -29,12 +29,12 @@ def bits(t):
     return t.contiguous().view(torch.int16)
 
 
-def encode_both(w, x, pinned=True):
+def encode_both(w, x, pinned=True, kv_fp8=False):
     from block_sparse_long_phase_b200 import StarCache
     cap = w.lq + w.T
-    ref = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, cap, w.scale)
+    ref = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, cap, w.scale, kv_fp8=kv_fp8)
     O, LSE = ref.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
-    host = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, cap, w.scale)
+    host = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, cap, w.scale, kv_fp8=kv_fp8)
     h = {k: x[k].cpu() for k in ("Qc", "Kc", "Vc")}
     if pinned:
         h = {k: v.pin_memory() for k, v in h.items()}
@@ -84,8 +84,23 @@ def test_pageable_host_memory_is_still_correct():
     out[1].close()
 
 
+def test_host_encode_fills_the_fp8_copy():
+    """With an FP8 cache the copy is quantised once every unit is done: codes
+    and scales equal the device entry's."""
+    w = wl.get("tiny").with_(**VARIANTS["d128-gqa8-batch3"])
+    x = {k: v.cuda() for k, v in wl.make_inputs(w, "cpu", with_decode=False).items()}
+    out = encode_both(w, x, kv_fp8=True)
+    check_same(w, *out)
+    ref, host = out[0], out[1]
+    for i in range(ref.num_segments - 1):
+        for a, b in zip(ref.segment_fp8_tensors(i), host.segment_fp8_tensors(i)):
+            assert torch.equal(a, b), f"FP8 segment {i}"
+    ref.close()
+    host.close()
+
+
 def test_full_size_8b_32k_host_encode_is_bit_exact():
-    """The bench's end-to-end call on its own workload: 8 pipeline units."""
+    """The bench's end-to-end call on its own workload: 16 pipeline units."""
     w = wl.get("8b-32k")
     x = wl.make_inputs(w, "cuda", with_decode=False)
     out = encode_both(w, x)

@@ -24,6 +24,7 @@ EXPORTS = (
     "star_query_prefill", "star_query_prefill_partials", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
     "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
+    "star_selftest_wait_timeout",
 )
 
 
@@ -65,6 +66,7 @@ def load(path: str = LIB_PATH):
     lib.star_cache_reset_query.argtypes = [vp]
     lib.star_ctx_encode.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.star_query_prefill.argtypes = [vp, i, vp, vp, vp, vp, vp, vp]
+    lib.star_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.POINTER(ctypes.c_int), vp]
     lib.star_ctx_encode_host.argtypes = [vp] + [vp] * 10 + [vp]
     lib.star_query_prefill_partials.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp]

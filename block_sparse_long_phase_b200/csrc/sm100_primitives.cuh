@@ -64,8 +64,8 @@ SM100_DEV bool mbar_spin(uint32_t bar, uint32_t parity) {
 // Bounded wait: gives up after `limit` polls (each poll may suspend briefly)
 // and returns false, so a broken pipeline ends instead of hanging the GPU.
 constexpr uint32_t kWaitLimit = 1u << 22;
-SM100_DEV bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+SM100_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }

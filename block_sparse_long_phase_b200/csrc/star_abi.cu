@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -235,7 +236,10 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const size_t qscl_bytes = (size_t)((q_rows + 3) / 4) * 16;
   const size_t o_qk8 = fp8 ? take(kv_q) : 0, o_qv8 = fp8 ? take(kv_q) : 0;
   const size_t o_qks = fp8 ? take(qscl_bytes) : 0, o_qvs = fp8 ? take(qscl_bytes) : 0;
-  e = cudaMalloc(&c->block, off);
+  // STAR_FAULT_INJECT=alloc makes this allocation fail (a test hook for the
+  // STAR_ENOMEM path)
+  const char* inject = getenv("STAR_FAULT_INJECT");
+  e = inject && strcmp(inject, "alloc") == 0 ? cudaErrorMemoryAllocation : cudaMalloc(&c->block, off);
   if (e != cudaSuccess) {
     delete c;
     return fail(STAR_ENOMEM, "cudaMalloc(%zu bytes): %s", off, cudaGetErrorString(e));
@@ -552,6 +556,15 @@ int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
       c->scratch, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_decode_step launch");
   c->q_len += 1;
+  return STAR_OK;
+}
+
+int star_selftest_wait_timeout(unsigned polls, int* gave_up, void* stream) {
+  if (!gave_up) return fail(STAR_EINVAL, "gave_up is NULL");
+  if (polls < 1 || polls > (1u << 22)) return fail(STAR_EINVAL, "polls must be in 1..2^22");
+  *gave_up = 0;
+  cudaError_t e = star::run_wait_timeout(polls, gave_up, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_selftest_wait_timeout");
   return STAR_OK;
 }
 

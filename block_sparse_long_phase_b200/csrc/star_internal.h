@@ -109,6 +109,9 @@ struct RopeJob {
 };
 void rope_inv_freq(int D, double base, double* out);
 cudaError_t launch_rope(const RopeJob& j, int D, int B, int groups, cudaStream_t st);
+// one CTA whose bounded wait on a barrier nothing completes must give up
+// (selftest.cu); synchronous, *gave_up = 1 when it did
+cudaError_t run_wait_timeout(unsigned polls, int* gave_up, cudaStream_t st);
 
 struct PrefillChunk {
   int seg;     // context segment, or -1 for the query region

@@ -85,7 +85,9 @@ typedef struct star_cache star_cache;
 /* Allocates the cache for `p` on the current CUDA device (cudaMalloc).
  * Layout in HBM: context segment i holds K (then V) as [B][Hkv][len_i][D]
  * bf16, len_i = min(b, L - i*b), segments back to back; the query region is
- * [B][Hkv][q_cap][D] for K and for V.  *out is NULL on failure. */
+ * [B][Hkv][q_cap][D] for K and for V.  *out is NULL on failure.
+ * STAR_ENOMEM when the allocation fails; with the environment variable
+ * STAR_FAULT_INJECT=alloc it fails on purpose (a test hook for that path). */
 STAR_API int star_cache_create(const star_params* p, star_cache** out);
 
 /* Frees everything the cache owns (synchronises the device first).  NULL is
@@ -227,6 +229,15 @@ STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const
  * R >= 0, 1 <= D <= 1024.  out_* must not alias the inputs. */
 STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const float* s,
                    float* out_A, float* out_s, void* stream);
+
+/* Self-test of the failure path every pipelined kernel here uses: one CTA
+ * waits, with the kernels' bounded mbarrier wait limited to `polls` polls
+ * (1..2^22; the kernels use 2^22), on a barrier nothing completes, so the
+ * wait must run out; the kernel then sets its error word and returns.
+ * Synchronous (waits for `stream`): *gave_up = 1 when the wait gave up, the
+ * expected outcome.  The context stays usable.  STAR_EINVAL for a NULL
+ * gave_up or polls out of range. */
+STAR_API int star_selftest_wait_timeout(unsigned polls, int* gave_up, void* stream);
 
 /* Decode step that allocates nothing (the pages have no counterpart: this is
  * an integration entry point).  For callers that cannot call cudaMalloc on

@@ -76,6 +76,11 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.star_query_prefill(None, 4, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_query_prefill_partials(None, 4, *([None] * 9)) == _abi.STAR_EINVAL
     assert lib.star_ctx_encode_host(*([None] * 12)) == _abi.STAR_EINVAL
+    flag = ctypes.c_int(7)
+    assert lib.star_selftest_wait_timeout(1000, None, None) == _abi.STAR_EINVAL
+    assert lib.star_selftest_wait_timeout(0, ctypes.byref(flag), None) == _abi.STAR_EINVAL
+    assert lib.star_selftest_wait_timeout((1 << 22) + 1, ctypes.byref(flag), None) == _abi.STAR_EINVAL
+    assert flag.value == 7                                     # nothing launched
     assert lib.star_cache_segment_fp8(None, 0, None, None, None, None) == _abi.STAR_EINVAL
     p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 1)  # the no-alloc path is bf16 only
     assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *([None] * 10)) == _abi.STAR_EINVAL

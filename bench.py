@@ -49,6 +49,7 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 TRAFFIC = {
     "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "7e0e6c54edb4d65b", 1395578368),
     "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 145053184),
+    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 544438272),
     "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 287573504),
 }
 
@@ -684,7 +685,7 @@ def main():
             "workload": wl2.name, "value": world * wl2.B / (t_us * 1e-6), "unit": "decode tok/s",
             "us_per_step": t_us,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "frac": gbs / pk["hbm_gbs"], "traffic": traffic("decode 8b-128k"),
                          "bytes_per_step": decode_bytes(wl2, 0)}}
         wl3, t3 = long_dec_fp8
         gbs = decode_bytes_fp8(wl3, 0) / (t3 * 1e-6) / 1e9

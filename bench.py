@@ -80,6 +80,22 @@ def phase1_flops(w):
     return 4 * w.D * w.Hq * w.B * pairs, pairs
 
 
+def prefill_roofline(w, ms, pk):
+    """Query prefill against min(bf16 peak, intensity x HBM): flops 4*D per
+    (query row, visible key) pair -- row r sees the L context keys and query
+    rows 0..r -- and bytes of the cache read once plus the query rows in and
+    the outputs out."""
+    pairs = w.lq * w.L + w.lq * (w.lq + 1) // 2
+    flops = 4 * w.D * w.Hq * w.B * pairs
+    nbytes = (w.B * w.Hkv * (w.L + w.lq) * w.D * 2 * 2            # K, V of the cache
+              + w.B * w.Hq * w.lq * w.D * 2 * 2 + w.B * w.Hq * w.lq * 4)   # Q in, O out, LSE out
+    peak_tf = min(pk["bf16_tflops"], flops / nbytes * pk["hbm_gbs"] / 1e3)
+    tf = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor" if peak_tf == pk["bf16_tflops"] else "hbm", "achieved": tf, "peak": peak_tf,
+            "unit": "TFLOP/s", "frac": tf / peak_tf, "flops": flops, "bytes": nbytes,
+            "intensity_flops_per_byte": flops / nbytes}
+
+
 def decode_bytes(w, t):
     """Algorithmic bytes of decode step t: the K and V of every cached row."""
     return w.B * w.Hkv * (w.L + w.lq + t + 1) * w.D * 2 * 2
@@ -341,7 +357,8 @@ def measure_configs(dev, flush, warmup, steps, world, dec_steps=8):
             "phase1_ms": t_enc, "ctx_tok_s": world * w.B * w.L / (t_enc / 1e3), "tflops": tf,
             "frac": tf / pk["bf16_tflops"],
             "frac_sustained": tf / pk["bf16_tflops_sustained"] if pk["bf16_tflops_sustained"] else None,
-            "prefill_ms": t_pre, "decode_steps_timed": T * steps, "decode_us": t_dec * 1e3,
+            "prefill_ms": t_pre, "prefill_frac": prefill_roofline(w, t_pre, pk)["frac"],
+            "decode_steps_timed": T * steps, "decode_us": t_dec * 1e3,
             "decode_tok_s": world * w.B / (t_dec / 1e3), "decode_gbs": gbs, "decode_frac": gbs / pk["hbm_gbs"]}
         cache.close()
         del x, O, LSE, Oq, LSEq
@@ -654,6 +671,7 @@ def main():
                                 "traffic": traffic("decode 8b-32k") if w.name == "8b-32k" else None,
                                 "peak_source": pk["source"]}},
         "prefill_ms": sum(pre_ms) / args.steps,
+        "prefill_roofline": prefill_roofline(w, sum(pre_ms) / args.steps, peaks()),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"],
                      "traffic": traffic("phase1 8b-32k") if w.name == "8b-32k" else None,

@@ -623,20 +623,27 @@ __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, 
 }
 
 // Merge the chunks' partials of every packed query row and scatter to O / LSE.
+// One warp per row: lane p holds the s of chunks p, p + 32, ... (one load
+// each, all in flight together), the maximum and the total come from warp
+// reductions, the chunk weights go through shared memory, and the lanes then
+// accumulate their D/32 columns over the chunks, eight chunks' loads at a time.
 // Debug outputs (null in the normal path): O32, the merged rows in float32;
 // Ah / sh, every chunk's partial in [chunk][B][Hq][lq] row order.
+constexpr int kMergeWarps = 4;
+constexpr int kSPerLane = (kMaxPrefillChunks + 31) / 32;
 template <int D>
-__global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq, int n_chunks,
-                                                            const float* __restrict__ partA,
-                                                            const float* __restrict__ partS,
-                                                            bf16* __restrict__ O,
-                                                            float* __restrict__ LSE,
-                                                            float* __restrict__ O32,
-                                                            float* __restrict__ Ah,
-                                                            float* __restrict__ sh) {
+__global__ void __launch_bounds__(32 * kMergeWarps) prefill_merge_kernel(CacheView c, int lq, int n_chunks,
+                                                                        const float* __restrict__ partA,
+                                                                        const float* __restrict__ partS,
+                                                                        bf16* __restrict__ O,
+                                                                        float* __restrict__ LSE,
+                                                                        float* __restrict__ O32,
+                                                                        float* __restrict__ Ah,
+                                                                        float* __restrict__ sh) {
+  __shared__ float wgt[kMergeWarps][kSPerLane * 32];
   const int rows_total = c.G * lq;
-  const long long gw = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long gw = (long long)blockIdx.x * kMergeWarps + wid;
   if (gw >= (long long)c.B * c.Hkv * rows_total) return;
   const long long bg = gw / rows_total;
   const int m = (int)(gw - bg * rows_total);
@@ -644,29 +651,56 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(CacheView c, int lq,
   const int h = g * c.G + m / lq;
   const int rr = m % lq;
   const long long orow_i = ((long long)bb * c.Hq + h) * lq + rr;   // row of O / LSE
+  const long long prow0 = bg * n_chunks * rows_total + m;          // chunk p's row: prow0 + p * rows_total
+  float sv[kSPerLane];
   float mx = -INFINITY;
-  for (int p = 0; p < n_chunks; ++p) mx = fmaxf(mx, partS[(bg * n_chunks + p) * rows_total + m]);
+#pragma unroll
+  for (int k = 0; k < kSPerLane; ++k) {
+    const int p = lane + 32 * k;
+    sv[k] = p < n_chunks ? partS[prow0 + (long long)p * rows_total] : -INFINITY;
+    mx = fmaxf(mx, sv[k]);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   const float base = mx == -INFINITY ? 0.f : mx;
   float tot = 0.f;
-  for (int p = 0; p < n_chunks; ++p) tot += __expf(partS[(bg * n_chunks + p) * rows_total + m] - base);
+#pragma unroll
+  for (int k = 0; k < kSPerLane; ++k) tot += sv[k] == -INFINITY ? 0.f : __expf(sv[k] - base);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
   const float lse = mx == -INFINITY ? -INFINITY : base + __logf(tot);
+  const long long prow_stride = (long long)c.B * c.Hq * lq;        // rows per chunk in Ah / sh
+#pragma unroll
+  for (int k = 0; k < kSPerLane; ++k) {
+    const int p = lane + 32 * k;
+    if (p < n_chunks) {
+      wgt[wid][p] = sv[k] == -INFINITY ? 0.f : __expf(sv[k] - lse);
+      if (sh) sh[p * prow_stride + orow_i] = sv[k];
+    }
+  }
+  __syncwarp();
   constexpr int PER = D / 32;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  const long long prow_stride = (long long)c.B * c.Hq * lq;        // rows per chunk in Ah / sh
-  for (int p = 0; p < n_chunks; ++p) {
-    const long long r = (bg * n_chunks + p) * rows_total + m;
-    const float s = partS[r];
-    if (Ah) {
+  constexpr int U = 8;
+  for (int p0 = 0; p0 < n_chunks; p0 += U) {
+    float v[U][PER];
 #pragma unroll
-      for (int i = 0; i < PER; ++i) Ah[(p * prow_stride + orow_i) * D + lane + 32 * i] = partA[r * D + lane + 32 * i];
-      if (lane == 0) sh[p * prow_stride + orow_i] = s;
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        v[u][i] = p0 + u < n_chunks ? partA[(prow0 + (long long)(p0 + u) * rows_total) * D + lane + 32 * i] : 0.f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (p0 + u >= n_chunks) break;
+      const float w = wgt[wid][p0 + u];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        acc[i] += w * v[u][i];
+        if (Ah) Ah[((p0 + u) * prow_stride + orow_i) * D + lane + 32 * i] = v[u][i];
+      }
     }
-    if (s == -INFINITY) continue;
-    const float w = __expf(s - lse);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] += w * partA[r * D + lane + 32 * i];
   }
   bf16* orow = O + orow_i * D;
 #pragma unroll
@@ -713,11 +747,11 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
   else
     attn_tc_kernel<64, true><<<grid, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
-  const int mgrid = (int)((rows + 3) / 4);
+  const int mgrid = (int)((rows + kMergeWarps - 1) / kMergeWarps);
   if (c.D == 128)
-    prefill_merge_kernel<128><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
+    prefill_merge_kernel<128><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
   else
-    prefill_merge_kernel<64><<<mgrid, 128, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
+    prefill_merge_kernel<64><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
   return cudaGetLastError();
 }
 

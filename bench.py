@@ -47,7 +47,7 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 # ncu captures summarised under profiles/, valid only for the kernel source they
 # were taken on (first 16 hex digits of its sha256); null otherwise.
 TRAFFIC = {
-    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "7e0e6c54edb4d65b", 1395578368),
+    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "1d236e77d71137c2", 1394200320),
     "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 145053184),
     "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 544438272),
     "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 287573504),

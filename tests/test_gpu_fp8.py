@@ -114,6 +114,9 @@ VARIANTS = {
     "batch2": dict(B=2, L=700, b=256, b_a=200, lq=9, T=4),
     "g16": dict(Hq=16, Hkv=1, L=400, b=128, b_a=128, lq=3, T=2),
     "tiny-blocks": dict(L=200, b=40, b_a=40, lq=70, T=3),
+    # 32 (batch, kv head) pairs of about 100 rows on ~6 decode CTAs: every CTA streams
+    # several short runs and flushes at each boundary
+    "many-heads-short": dict(B=4, Hq=16, Hkv=8, D=64, L=96, b=32, b_a=32, lq=5, T=3),
 }
 
 

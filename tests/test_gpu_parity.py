@@ -96,6 +96,9 @@ TINY_VARIANTS = {
     "g16": dict(Hq=16, Hkv=1, L=400, b=128, b_a=128, lq=3, T=2),
     "tiny-blocks": dict(L=200, b=40, b_a=40, lq=70, T=3),
     "max-blocks": dict(L=191 * 48 - 5, b=48, b_a=41, lq=3, T=2),  # 191 blocks, the last one ragged
+    # 32 (batch, kv head) pairs of about 100 rows on ~6 decode CTAs: every CTA streams
+    # several short runs and flushes at each boundary
+    "many-heads-short": dict(B=4, Hq=16, Hkv=8, D=64, L=96, b=32, b_a=32, lq=5, T=3),
 }
 
 

@@ -104,7 +104,12 @@ TINY_VARIANTS = {
 
 @pytest.mark.parametrize("variant", list(TINY_VARIANTS))
 def test_small_cases_every_element(variant):
-    w = wl.get("tiny").with_(**TINY_VARIANTS[variant])
+    check_every_element(wl.get("tiny").with_(**TINY_VARIANTS[variant]), variant)
+
+
+def check_every_element(w, variant):
+    """Phase 1, the cache, the prefill and every decode step of workload w
+    against the oracle, element by element."""
     x = {k: v.cuda() for k, v in wl.make_inputs(w, "cpu").items()}
     cache, O, LSE, Oq, LSEq, dec = run_path(w, x)
     cpu = {k: v.cpu() for k, v in x.items()}

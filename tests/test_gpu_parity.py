@@ -99,6 +99,8 @@ TINY_VARIANTS = {
     # 32 (batch, kv head) pairs of about 100 rows on ~6 decode CTAs: every CTA streams
     # several short runs and flushes at each boundary
     "many-heads-short": dict(B=4, Hq=16, Hkv=8, D=64, L=96, b=32, b_a=32, lq=5, T=3),
+    # 600 query rows: G * lq = 1200 packed rows, five 256-row pairs per kv head in the prefill
+    "long-query": dict(L=512, b=256, b_a=256, lq=600, T=2),
 }
 
 

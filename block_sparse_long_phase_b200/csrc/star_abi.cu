@@ -408,15 +408,25 @@ int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const vo
   const star::CacheView& w = c->view;
   cudaError_t e = cudaSuccess;
   if (!c->s_in) {
-    e = cudaStreamCreateWithFlags(&c->s_in, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->s_out, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking);
+    // created once, all or nothing: a failure leaves the cache as it was
+    cudaStream_t st3[3] = {nullptr, nullptr, nullptr};
+    std::vector<cudaEvent_t> evs;
+    for (int i = 0; e == cudaSuccess && i < 3; ++i) e = cudaStreamCreateWithFlags(&st3[i], cudaStreamNonBlocking);
     for (size_t i = 0; e == cudaSuccess && i < 3 + 2 * c->units.size(); ++i) {
       cudaEvent_t ev;
       e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
-      if (e == cudaSuccess) c->events.push_back(ev);
+      if (e == cudaSuccess) evs.push_back(ev);
     }
-    if (e != cudaSuccess) return cuda_fail(e, "copy streams");
+    if (e != cudaSuccess) {
+      for (cudaEvent_t ev : evs) cudaEventDestroy(ev);
+      for (cudaStream_t x : st3)
+        if (x) cudaStreamDestroy(x);
+      return cuda_fail(e, "copy streams");
+    }
+    c->s_in = st3[0];
+    c->s_out = st3[1];
+    c->s_comp = st3[2];
+    c->events = std::move(evs);
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaEvent_t ev_start = c->events[0], ev_end = c->events[1], ev_comp = c->events[2];
@@ -453,7 +463,6 @@ int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const vo
       e = star::launch_ctx_encode_tc(w, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
                                      static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE,
                                      c->unit_work + un.off, un.n, c->scratch.err, cs, nullptr);
-    if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
     if (e == cudaSuccess) e = cudaEventRecord(ev_out, cs);
     // outputs of the unit
     if (e == cudaSuccess) e = cudaStreamWaitEvent(c->s_out, ev_out, 0);
@@ -470,7 +479,14 @@ int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const vo
   if (e == cudaSuccess && w.ctxK8) e = star::launch_quantize_ctx_fp8(w, st);
   if (e == cudaSuccess) e = cudaEventRecord(ev_end, c->s_out);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_end, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode_host");
+  if (e != cudaSuccess) {
+    // whatever was enqueued on the side streams still ends before `stream` goes on
+    const cudaStream_t side[3] = {c->s_in, c->s_comp, c->s_out};
+    for (cudaStream_t x : side)
+      if (cudaEventRecord(ev_end, x) == cudaSuccess) cudaStreamWaitEvent(st, ev_end, 0);
+    if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
+    return cuda_fail(e, "star_ctx_encode_host");
+  }
   c->q_len = 0;
   return STAR_OK;
 }

@@ -48,9 +48,9 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 # were taken on (first 16 hex digits of its sha256); null otherwise.
 TRAFFIC = {
     "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "1d236e77d71137c2", 1394200320),
-    "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 145053184),
-    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 544438272),
-    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "a9d59e0db7a2c7ee", 287573504),
+    "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 145271552),
+    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 547147264),
+    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 290108928),
 }
 
 

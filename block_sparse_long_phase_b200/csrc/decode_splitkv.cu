@@ -795,6 +795,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     complete(bg, rows);
   };
 
+  // Warm L2 with the step's q, k and v rows of every (batch, kv head) this
+  // CTA's span touches: the flush cleared them out, and whichever CTA merges a
+  // pair reads them right after its last stage, on the step's critical path.
+  {
+    const long long R = (long long)c.B * c.Hkv * a.rpb;
+    const long long x0 = span_start(blockIdx.x, R, a.ncta), x1 = span_start(blockIdx.x + 1, R, a.ncta);
+    if (x1 > x0) {
+      const int bg0 = (int)((unsigned)x0 / (unsigned)a.rpb), bg1 = (int)((unsigned)(x1 - 1) / (unsigned)a.rpb);
+      constexpr int kLine = 128;                       // bytes per L2 prefetch
+      const int q_lines = G * D * 2 / kLine, kv_lines = D * 2 / kLine;
+      const int per_bg = q_lines + 2 * kv_lines;
+      for (int i = ctid; i < (bg1 - bg0 + 1) * per_bg; i += 32 * NCW) {
+        const int bg = bg0 + i / per_bg, l = i % per_bg;
+        const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
+        const char* p = l < q_lines
+                            ? reinterpret_cast<const char*>(a.q + ((long long)bb * c.Hq + (long long)g * G) * D) + l * kLine
+                            : reinterpret_cast<const char*>((l - q_lines < kv_lines ? a.k : a.v) + (long long)bg * D) +
+                                  ((l - q_lines) % kv_lines) * kLine;
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
+      }
+    }
+  }
+
   for (int st = 0;; ++st) {
     const int slot = st % S::NST, use = st / S::NST;
     // every consumer warp takes the same path: a warp whose bounded wait gave

@@ -23,12 +23,16 @@ Sources (page title, then section / step / equation):
   Attention": Phase 1 bullets (segmentation, anchor prefix, non-anchor KV kept)
   and Phase 2 bullets (A_h, s_h, s_global, A_global).
 
-Readings where the pages are silent or garbled (each is listed in the design doc):
+Readings where the pages are silent or garbled (the passage each one settles
+is the [P2] Phase 1 / Phase 2 step named beside it):
 
-* the anchor is the first ``b_a`` context tokens, ``0 <= b_a <= b``;
+* the anchor is the first ``b_a`` context tokens, ``0 <= b_a <= b`` ([P2]
+  Phase 1 Step 2 names the first block as the anchor; its length is left open);
 * block 0 is plain causal attention over its own rows, blocks i >= 1 see the
-  whole anchor plus their own block causally; only block rows are outputs;
-* the last block may be short;
+  whole anchor plus their own block causally; only block rows are outputs
+  ([P2] Phase 1 Steps 2 and 4: causal attention over the augmented block,
+  whose anchor KV Step 5 then discards);
+* the last block may be short ([P2] Phase 1 Step 1);
 * ``s_h`` is carried as a natural-log log-sum-exp over the *scaled* logits;
   the merge is ``s = log sum_h exp(s_h)``, ``A = sum_h exp(s_h - s) A_h``
   (algebraically the README's ``s_h / s_global`` weights); the garbled
@@ -387,7 +391,8 @@ def fp8_dequantize_rows(codes, s):
 # the block's own tokens keep theirs; [P2] ablation of section 4.1 (Table 4):
 # anchor position IDs taken from the first block (proposed), from the block
 # just before block i, or sampled at random from [0, start of block i).
-# Readings (listed in the design doc): rotary embedding in the RoFormer form on
+# Readings (the pages name Llama 3.1 models but give no rotary details):
+# rotary embedding in the RoFormer form on
 # adjacent pairs (2k, 2k+1) with inverse frequencies base^(-2k/D), base
 # 500000 (Llama 3) and no frequency rescaling; "previous" = the b_a positions
 # right before block i; random positions are drawn by the caller; query-region

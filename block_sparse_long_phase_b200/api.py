@@ -361,6 +361,17 @@ def star_decode_step_noalloc(params, q_len, ctx_k, ctx_v, q_k, q_v, q, k, v, o=N
     return o, lse
 
 
+def star_noalloc_device_error(device=None) -> int:
+    """Reads and clears the error word of the no-alloc decode scratch on the
+    current device, after the work queued on the current stream: non-zero if
+    a step since the last read gave up a bounded wait (its outputs are invalid)."""
+    lib = _abi.load()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    f = ctypes.c_int()
+    _abi.check(lib.star_noalloc_device_error(ctypes.byref(f), _stream(dev)))
+    return f.value
+
+
 def _view_from_ptr(ptr: int, n_elems: int, typestr: str, device) -> torch.Tensor:
     """A flat view of ``n_elems`` elements of device memory owned by libstar."""
 

@@ -1080,12 +1080,40 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
   sc.partS_elems = kNoAllocPartS;
   sc.n_tickets = (int)kNoAllocTickets;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // the tickets (and the error word next to them) must start at zero
-  e = cudaMemsetAsync(sc.tickets, 0, (kNoAllocTickets + 1) * sizeof(float), st);
+  // the merge tickets must start at zero (a step that gave up a wait may have
+  // left some behind); the error word next to them is left as it is, so an
+  // abandoned wait stays visible until star_noalloc_device_error reads it
+  e = cudaMemsetAsync(sc.tickets, 0, kNoAllocTickets * sizeof(unsigned), st);
   if (e == cudaSuccess)
     e = launch_decode_step(c, maps, p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->D), (int)q_len,
                            static_cast<const bf16*>(q), static_cast<const bf16*>(k),
                            static_cast<const bf16*>(v), static_cast<bf16*>(o), lse, pl, sc, st);
   if (e != cudaSuccess) return set_error(STAR_ECUDA, cudaGetErrorString(e));
+  return STAR_OK;
+}
+
+// Reads and clears the error word of the static decode scratch on the current
+// device, after the work already queued on `stream`.
+extern "C" STAR_API int star_noalloc_device_error(int* flag, void* stream) {
+  using namespace star;
+  if (!flag) return set_error(STAR_EINVAL, "flag is NULL");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return set_error(STAR_ECUDA, "cudaGetDevice failed");
+  float* base = nullptr;
+  int sms = 0;
+  e = noalloc_setup(dev, &base, &sms);
+  if (e != cudaSuccess) return set_error(STAR_ECUDA, cudaGetErrorString(e));
+  unsigned* tickets = reinterpret_cast<unsigned*>(base + kNoAllocPartA + kNoAllocPartS);
+  int* err = reinterpret_cast<int*>(base + kNoAllocPartA + kNoAllocPartS + kNoAllocTickets);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  e = cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess && h) e = cudaMemsetAsync(err, 0, sizeof(int), st);
+  if (e == cudaSuccess && h) e = cudaMemsetAsync(tickets, 0, kNoAllocTickets * sizeof(unsigned), st);
+  if (e == cudaSuccess && h) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return set_error(STAR_ECUDA, cudaGetErrorString(e));
+  *flag = h;
   return STAR_OK;
 }

@@ -259,11 +259,22 @@ STAR_API int star_selftest_wait_timeout(unsigned polls, int* gave_up, void* stre
  * else STAR_EINVAL.  The first call on a device looks up the array's device
  * address (make it before any stream capture).  Every call shares the one
  * array, so calls that overlap on the GPU (other streams, other threads) race;
- * each call clears the merge tickets it needs. */
+ * each call clears the merge tickets it needs.  A kernel that gives up one of
+ * its bounded pipeline waits sets the array's error word and returns early
+ * (o and lse of that call are then invalid); the word is not cleared by later
+ * calls: read it with star_noalloc_device_error. */
 STAR_API int star_decode_step_noalloc(const star_params* p, long long q_len,
                                       const void* ctx_k, const void* ctx_v, void* q_k, void* q_v,
                                       const void* q, const void* k, const void* v,
                                       void* o, float* lse, void* stream);
+
+/* Error word of star_decode_step_noalloc's static scratch on the current
+ * device (no counterpart in the pages, like the entry point it serves):
+ * waits for the work queued on `stream`, then *flag = non-zero if any
+ * no-alloc decode step since the last read gave up a bounded wait (its o and
+ * lse are invalid).  Clears the word and the merge tickets when it was set.
+ * Allocates nothing.  STAR_EINVAL for a NULL flag. */
+STAR_API int star_noalloc_device_error(int* flag, void* stream);
 
 /* Description of the last error in this thread ("" if none). */
 STAR_API const char* star_last_error(void);

@@ -85,6 +85,15 @@ def test_argument_errors_are_caught_on_the_host(lib):
     p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0, 1)  # the no-alloc path is bf16 only
     assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *([None] * 10)) == _abi.STAR_EINVAL
     assert b"kv_fp8" in lib.star_last_error()
+    # a full query region is refused before anything touches the device (any
+    # non-null, 16-byte aligned pointers will do: none is dereferenced)
+    p = _abi.StarParams(1, 4, 2, 64, 1024, 256, 256, 8, 0.0)
+    fake = [ctypes.c_void_p(4096 * (i + 1)) for i in range(9)]
+    assert lib.star_decode_step_noalloc(ctypes.byref(p), 8, *fake, None) == _abi.STAR_ENOSPC
+    assert lib.star_decode_step_noalloc(ctypes.byref(p), -1, *fake, None) == _abi.STAR_EINVAL
+    misaligned = fake[:4] + [ctypes.c_void_p(4096 + 8)] + fake[5:]
+    assert lib.star_decode_step_noalloc(ctypes.byref(p), 0, *misaligned, None) == _abi.STAR_EINVAL
+    assert lib.star_noalloc_device_error(None, None) == _abi.STAR_EINVAL
     assert lib.star_rope(1, 1, 8, 96, 500000.0, None, 0, None, None, None) == _abi.STAR_EUNSUPPORTED
     assert lib.star_rope(1, 1, 8, 64, 1.0, None, 0, None, None, None) == _abi.STAR_EINVAL     # theta <= 1
     assert lib.star_rope(1, 1, 8, 64, 500000.0, None, -1, None, None, None) == _abi.STAR_EINVAL

@@ -24,7 +24,7 @@ EXPORTS = (
     "star_query_prefill", "star_query_prefill_partials", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
     "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
-    "star_selftest_wait_timeout", "star_noalloc_device_error",
+    "star_selftest_wait_timeout", "star_noalloc_device_error", "star_ctx_encode_fp32",
 )
 
 
@@ -77,6 +77,7 @@ def load(path: str = LIB_PATH):
     lib.star_decode_step_noalloc.argtypes = [ctypes.POINTER(StarParams), ll, vp, vp, vp, vp,
                                              vp, vp, vp, vp, vp, vp]
     lib.star_noalloc_device_error.argtypes = [ctypes.POINTER(i), vp]
+    lib.star_ctx_encode_fp32.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = i
     lib.star_last_error.restype = ctypes.c_char_p

@@ -159,6 +159,26 @@ class StarCache:
                                                      _ptr(LSE), _stream(Q.device)))
         return O, LSE
 
+    def star_ctx_encode_fp32(self, Q, K, V, O=None, LSE=None, O32=None):
+        """Debug form of phase 1: also returns O32 [B, Hq, L, D] float32, the
+        rows before their bf16 rounding.  Returns (O, LSE, O32)."""
+        B, Hq, Hkv, D, L = self.B, self.Hq, self.Hkv, self.D, self.L
+        _need(Q, (B, Hq, L, D), torch.bfloat16, "Q")
+        _need(K, (B, Hkv, L, D), torch.bfloat16, "K")
+        _need(V, (B, Hkv, L, D), torch.bfloat16, "V")
+        if O is None:
+            O = torch.empty((B, Hq, L, D), dtype=torch.bfloat16, device=Q.device)
+        if LSE is None:
+            LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
+        if O32 is None:
+            O32 = torch.empty((B, Hq, L, D), dtype=torch.float32, device=Q.device)
+        _need(O, (B, Hq, L, D), torch.bfloat16, "O")
+        _need(LSE, (B, Hq, L), torch.float32, "LSE")
+        _need(O32, (B, Hq, L, D), torch.float32, "O32")
+        _abi.check(self.lib.star_ctx_encode_fp32(self.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                                 _ptr(O32), _stream(Q.device)))
+        return O, LSE, O32
+
     def star_ctx_encode_host(self, hQ, hK, hV, hO=None, hLSE=None, staging=None):
         """Phase 1 from host tensors: the copies in and out overlap the encoding.
 

@@ -69,6 +69,7 @@ struct CtxTcArgs {
   const bf16* V;
   bf16* O;
   float* LSE;
+  float* O32;         // phase 1, debug: the rows before their bf16 rounding (null: none)
   const int4* work;   // phase 1: (b*Hkv + g, head pair, block, q tile)
   int* err;
   int anchor_keys;    // phase 1: block i >= 1 reads its anchor's K tiles from tkq
@@ -421,20 +422,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       const float lse = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
       if (!PF) {
         const int h = h0 + q;
-        bf16* orow = a.O + (((long long)bb * c.Hq + h) * c.L + pos) * D;
+        const long long orow_i = ((long long)bb * c.Hq + h) * c.L + pos;
+        bf16* orow = a.O + orow_i * D;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
           if (r < n_rows) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv);
             uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               reinterpret_cast<uint4*>(orow + cc * 32)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            if (a.O32) {
+              float4* o32 = reinterpret_cast<float4*>(a.O32 + orow_i * D + cc * 32);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                o32[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                     __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+            }
           }
         }
         if (r < n_rows) a.LSE[((long long)bb * c.Hq + h) * c.L + pos] = lse;
@@ -573,7 +583,7 @@ cudaError_t attn_tc_prepare(int D) {
 
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
-                                 int* err, cudaStream_t st, const bf16* Ka) {
+                                 int* err, cudaStream_t st, const bf16* Ka, float* O32) {
   if (n_work == 0) return cudaSuccess;
   CtxTcArgs a;
   memset(&a, 0, sizeof(a));
@@ -593,6 +603,7 @@ cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q,
   a.V = V;
   a.O = O;
   a.LSE = LSE;
+  a.O32 = O32;
   a.work = work;
   a.err = err;
   if (c.D == 128)

@@ -375,27 +375,46 @@ int star_cache_reset_query(star_cache* c) {
   return STAR_OK;
 }
 
-int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const void* V, const void* Ka,
-                             void* O, float* LSE, void* stream) {
+}  // extern "C"
+
+namespace {
+// star_ctx_encode and its forms: per-block anchor keys (Ka) and the float32
+// debug rows (O32), either may be null.
+int ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, const void* Ka, void* O,
+               float* LSE, float* O32, void* stream) {
   if (!c) return fail(STAR_EINVAL, "cache is NULL");
   if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
-      (Ka && !aligned16(Ka)))
+      (Ka && !aligned16(Ka)) || (O32 && !aligned16(O32)))
     return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
   cudaError_t e = star::launch_ctx_encode_tc(
       c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
       static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work, c->scratch.err,
-      static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka));
+      static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka), O32);
   if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
   if (e == cudaSuccess && c->view.ctxK8) e = star::launch_quantize_ctx_fp8(c->view, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
   c->q_len = 0;
   return STAR_OK;
 }
+}  // namespace
+
+extern "C" {
+
+int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const void* V, const void* Ka,
+                             void* O, float* LSE, void* stream) {
+  return ctx_encode(c, Q, K, V, Ka, O, LSE, nullptr, stream);
+}
 
 int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
                     float* LSE, void* stream) {
-  return star_ctx_encode_anchored(c, Q, K, V, nullptr, O, LSE, stream);
+  return ctx_encode(c, Q, K, V, nullptr, O, LSE, nullptr, stream);
+}
+
+int star_ctx_encode_fp32(star_cache* c, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         float* O32, void* stream) {
+  if (!O32) return fail(STAR_EINVAL, "O32 is NULL");
+  return ctx_encode(c, Q, K, V, nullptr, O, LSE, O32, stream);
 }
 
 int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK, const void* hV, void* hO,

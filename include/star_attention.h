@@ -132,6 +132,16 @@ STAR_API int star_cache_reset_query(star_cache* c);
 STAR_API int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V,
                     void* O, float* LSE, void* stream);
 
+/* Debug form of star_ctx_encode ([P2] Phase 1 Steps 1-5): the same encode,
+ * cache, O and LSE, and also O32 [B][Hq][L][D] float32, every output row
+ * before its bf16 rounding (O is bit for bit the round-to-nearest-even of
+ * O32).  For tests and inspection: with very short blocks or anchors a row
+ * averages a handful of values, and the bf16 rounding of O alone can then be
+ * most of an absolute error bar.  Errors as star_ctx_encode, plus STAR_EINVAL
+ * for a NULL O32. */
+STAR_API int star_ctx_encode_fp32(star_cache* c, const void* Q, const void* K, const void* V,
+                                  void* O, float* LSE, float* O32, void* stream);
+
 /* RoPE front end ("Star Attention", Phase 1 Step 2: every token keeps its
  * position ID; anchor tokens keep theirs).  Rotary embedding of
  * x [B][H][L][D] bf16 into y (y == x allowed): each adjacent pair

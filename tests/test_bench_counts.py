@@ -59,3 +59,19 @@ def test_decode_bytes_count_every_row_the_token_sees():
         assert bench.decode_bytes(w, t) == w.B * w.Hkv * seen * w.D * 2 * 2
         # FP8: codes + a float32 scale per row for K and V, the token's own row in bf16
         assert bench.decode_bytes_fp8(w, t) == w.B * w.Hkv * ((seen - 1) * (w.D + 4) * 2 + w.D * 4)
+
+
+@pytest.mark.parametrize("L,b,b_a", [(1024, 256, 256), (1000, 256, 100), (300, 512, 512)])
+def test_cpu_baseline_sample_pairs_equal_the_star_mask(L, b, b_a):
+    """The CPU baseline extrapolates by visible pairs: the sampled rows' count
+    must equal the explicit Star mask's row sums, and the sample must hold
+    every block's first and last rows."""
+    w = wl.get("tiny").with_(L=L, b=b, b_a=b_a)
+    data = bench.oracle_sample_inputs(w)
+    rows = np.concatenate(data["blocks"])
+    assert bench.sample_pairs(w, data["blocks"]) == int(so.star_mask_rows(L, b, b_a, rows).sum()) * w.G
+    for (s, n), blk in zip(so.block_table(L, b), data["blocks"]):
+        assert blk[0] == s and blk[-1] == s + n - 1
+    again = bench.oracle_sample_inputs(w)
+    assert all(np.array_equal(x, y) for x, y in zip(data["blocks"], again["blocks"]))
+    assert np.array_equal(data["K"], again["K"])

@@ -25,6 +25,8 @@ EXPORTS = (
     "star_decode_step_noalloc", "star_last_error", "star_version",
     "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
     "star_selftest_wait_timeout", "star_noalloc_device_error", "star_ctx_encode_fp32",
+    "star_decode_step_partials", "star_partial_attend",
+    "star_lse_merge_bf16",
 )
 
 
@@ -78,6 +80,10 @@ def load(path: str = LIB_PATH):
                                              vp, vp, vp, vp, vp, vp]
     lib.star_noalloc_device_error.argtypes = [ctypes.POINTER(i), vp]
     lib.star_ctx_encode_fp32.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.star_lse_merge_bf16.argtypes = [i, ll, i, vp, vp, vp, vp, vp]
+    lib.star_partial_attend.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp, vp]
+    lib.star_decode_step_partials.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ll), i,
+                                              ctypes.POINTER(i), vp]
     for name in EXPORTS:
         getattr(lib, name).restype = i
     lib.star_last_error.restype = ctypes.c_char_p

@@ -314,6 +314,51 @@ class StarCache:
         return o, lse
 
 
+    def star_partial_attend(self, Q, first_seg, n_seg, K=None, V=None):
+        """Phase-2 partial of rows Q [B, Hq, lq, D] over context segments
+        [first_seg, first_seg + n_seg) and, when K and V are given, the query
+        region after appending them.  Returns (A [B, Hq, lq, D], s [B, Hq, lq])
+        float32."""
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        lq = Q.shape[2]
+        _need(Q, (B, Hq, lq, D), torch.bfloat16, "Q")
+        with_query = K is not None
+        if with_query:
+            _need(K, (B, Hkv, lq, D), torch.bfloat16, "K")
+            _need(V, (B, Hkv, lq, D), torch.bfloat16, "V")
+        A = torch.empty((B, Hq, lq, D), dtype=torch.float32, device=Q.device)
+        s = torch.empty((B, Hq, lq), dtype=torch.float32, device=Q.device)
+        _abi.check(self.lib.star_partial_attend(
+            self.handle, int(first_seg), int(n_seg), int(with_query), lq, _ptr(Q),
+            _ptr(K) if with_query else None, _ptr(V) if with_query else None, _ptr(A), _ptr(s),
+            _stream(Q.device)))
+        return A, s
+
+    def star_decode_step_partials(self, q, k, v):
+        """Debug form of :meth:`star_decode_step` that also returns the decode
+        kernel's own partials: ``(o, lse, Ah [P, G, D], sh [P, G], spans)``,
+        ``spans`` an int64 array [P, 3] of (b*Hkv + kv head, first row, end
+        row) over that kv head's cached rows (context, then query region)."""
+        import numpy as np
+        B, Hq, Hkv, D = self.B, self.Hq, self.Hkv, self.D
+        _need(q, (B, Hq, 1, D), torch.bfloat16, "q")
+        _need(k, (B, Hkv, 1, D), torch.bfloat16, "k")
+        _need(v, (B, Hkv, 1, D), torch.bfloat16, "v")
+        G = Hq // Hkv
+        o = torch.empty((B, Hq, 1, D), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        n = ctypes.c_int(0)
+        cap = 4 * B * Hkv + 4 * torch.cuda.get_device_properties(q.device).multi_processor_count
+        Ah = torch.empty((cap, G, D), dtype=torch.float32, device=q.device)
+        sh = torch.empty((cap, G), dtype=torch.float32, device=q.device)
+        spans = np.zeros((cap, 3), dtype=np.int64)
+        _abi.check(self.lib.star_decode_step_partials(
+            self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(Ah), _ptr(sh),
+            spans.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), cap, ctypes.byref(n), _stream(q.device)))
+        P = n.value
+        return o, lse, Ah[:P], sh[:P], spans[:P]
+
+
 def star_rope(x: torch.Tensor, positions=None, pos0=0, theta=ROPE_THETA, out=None):
     """Rotary embedding of x [B, H, L, D] bf16 (CUDA) at positions
     ``positions`` (int32 CUDA tensor [L]) or pos0 + t; ``out`` may be ``x``."""
@@ -379,6 +424,22 @@ def star_decode_step_noalloc(params, q_len, ctx_k, ctx_v, q_k, q_v, q, k, v, o=N
                                             _ptr(q_k), _ptr(q_v), _ptr(q), _ptr(k), _ptr(v),
                                             _ptr(o), _ptr(lse), _stream(q.device)))
     return o, lse
+
+
+def star_lse_merge_bf16(A: torch.Tensor, s: torch.Tensor, out_O=None, out_s=None):
+    """Merge partials A [P, R, D], s [P, R] (float32, CUDA) -> (O [R, D] bf16, s [R])."""
+    lib = _abi.load()
+    P, R, D = A.shape
+    _need(A, (P, R, D), torch.float32, "A")
+    _need(s, (P, R), torch.float32, "s")
+    if out_O is None:
+        out_O = torch.empty((R, D), dtype=torch.bfloat16, device=A.device)
+    if out_s is None:
+        out_s = torch.empty((R,), dtype=torch.float32, device=A.device)
+    _need(out_O, (R, D), torch.bfloat16, "out_O")
+    _need(out_s, (R,), torch.float32, "out_s")
+    _abi.check(lib.star_lse_merge_bf16(P, R, D, _ptr(A), _ptr(s), _ptr(out_O), _ptr(out_s), _stream(A.device)))
+    return out_O, out_s
 
 
 def star_noalloc_device_error(device=None) -> int:

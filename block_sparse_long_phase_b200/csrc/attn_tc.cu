@@ -639,7 +639,8 @@ __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, 
 // reductions, the chunk weights go through shared memory, and the lanes then
 // accumulate their D/32 columns over the chunks, eight chunks' loads at a time.
 // Debug outputs (null in the normal path): O32, the merged rows in float32;
-// Ah / sh, every chunk's partial in [chunk][B][Hq][lq] row order.
+// Ah / sh, every chunk's partial in [chunk][B][Hq][lq] row order.  O may be
+// null when only the float32 rows are wanted (a partial over part of the cache).
 constexpr int kMergeWarps = 4;
 constexpr int kSPerLane = (kMaxPrefillChunks + 31) / 32;
 template <int D>
@@ -713,9 +714,11 @@ __global__ void __launch_bounds__(32 * kMergeWarps) prefill_merge_kernel(CacheVi
       }
     }
   }
-  bf16* orow = O + orow_i * D;
+  if (O) {
+    bf16* orow = O + orow_i * D;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
+    for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
+  }
   if (O32) {
 #pragma unroll
     for (int i = 0; i < PER; ++i) O32[orow_i * D + lane + 32 * i] = acc[i];
@@ -730,7 +733,7 @@ int prefill_row_pairs(const CacheView& c, int lq) { return (c.G * lq + 2 * BM - 
 cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, float scale, int lq,
                                     int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
-                                    cudaStream_t st, float* O32, float* Ah, float* sh) {
+                                    cudaStream_t st, float* O32, float* Ah, float* sh, bool append) {
   CtxTcArgs a;
   memset(&a, 0, sizeof(a));
   const unsigned long long qrows = (unsigned long long)c.B * c.Hq * lq;
@@ -748,15 +751,19 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
   a.partA = s.partA;
   a.partS = s.partS;
   a.plan = plan;
-  const long long n16 = (long long)c.B * c.Hkv * lq * (c.D / 8);
-  const int agrid = (int)((n16 + 255) / 256 < 1024 ? (n16 + 255) / 256 : 1024);
-  query_append_kernel<<<agrid, 256, 0, st>>>(c, lq, len0, reinterpret_cast<const uint4*>(Kq),
-                                             reinterpret_cast<const uint4*>(Vq));
+  if (append) {
+    const long long n16 = (long long)c.B * c.Hkv * lq * (c.D / 8);
+    const int agrid = (int)((n16 + 255) / 256 < 1024 ? (n16 + 255) / 256 : 1024);
+    query_append_kernel<<<agrid, 256, 0, st>>>(c, lq, len0, reinterpret_cast<const uint4*>(Kq),
+                                               reinterpret_cast<const uint4*>(Vq));
+  }
   const int grid = c.B * c.Hkv * a.row_pairs * plan.n_chunks;
-  if (c.D == 128)
-    attn_tc_kernel<128, true><<<grid, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
-  else
-    attn_tc_kernel<64, true><<<grid, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+  if (grid > 0) {
+    if (c.D == 128)
+      attn_tc_kernel<128, true><<<grid, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
+    else
+      attn_tc_kernel<64, true><<<grid, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+  }
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
   const int mgrid = (int)((rows + kMergeWarps - 1) / kMergeWarps);
   if (c.D == 128)

@@ -84,19 +84,6 @@ struct DecodeArgs {
   int* err;
 };
 
-// Row indices stay below 2^31 (checked when the cache is made), so both
-// quotients below divide a numerator under 2^53 by at most 2^31.  They are
-// taken in double, which is exact there: the rounding error of the quotient
-// is below 1 / divisor, the least distance of a non-integer quotient from an
-// integer, so its floor is the integer quotient.  (A 64-bit integer division
-// costs several times as long, ahead of the first TMA load.)
-__device__ __forceinline__ long long span_start(long long i, long long R, int n) {
-  return (long long)floor((double)(i * R) / (double)n);
-}
-// CTA whose span holds row x (largest i with span_start(i) <= x).
-__device__ __forceinline__ int cta_of(long long x, long long R, int n) {
-  return (int)floor((double)((x + 1) * n - 1) / (double)R);
-}
 
 // Release the partials this CTA wrote (ordered before by the consumer barrier,
 // cumulatively) and acquire every other CTA's, in one atomic.
@@ -847,6 +834,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
 }
 
 }  // namespace
+
+void decode_parts(const CacheView& c, long long len0, const DecodePlan& pl, std::vector<DecodePart>& out) {
+  out.clear();
+  const long long rpb = c.L + len0;
+  const long long R = (long long)c.B * c.Hkv * rpb;
+  for (int bg = 0; bg < c.B * c.Hkv; ++bg) {
+    const long long lo = (long long)bg * rpb, hi = lo + rpb;
+    const int c0 = cta_of(lo, R, pl.ncta), c1 = cta_of(hi - 1, R, pl.ncta);
+    for (int i = c0; i <= c1; ++i) {
+      const long long x0 = std::max(lo, span_start(i, R, pl.ncta));
+      const long long x1 = std::min(hi, span_start(i + 1, R, pl.ncta));
+      out.push_back({bg, i - c0, x0 - lo, x1 - lo});
+    }
+  }
+}
 
 int decode_max_partials(const CacheView& c, int ncta) {
   // spans that can touch one (batch, kv head): ceil(ncta / (B * Hkv)), one

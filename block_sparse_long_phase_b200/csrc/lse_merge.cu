@@ -16,10 +16,11 @@ namespace {
 
 constexpr int ROWS_PER_CTA = 8;
 
+// outA (float32) and outB (bf16, rounded to nearest even once) may each be null.
 __global__ void __launch_bounds__(32 * ROWS_PER_CTA)
     lse_merge_kernel(int P, long long R, int D, const float* __restrict__ A,
                      const float* __restrict__ S, float* __restrict__ outA,
-                     float* __restrict__ outS) {
+                     bf16* __restrict__ outB, float* __restrict__ outS) {
   const long long r = (long long)blockIdx.x * ROWS_PER_CTA + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= R) return;
@@ -62,7 +63,8 @@ __global__ void __launch_bounds__(32 * ROWS_PER_CTA)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int d = d0 + lane + 32 * i;
-      if (d < D) outA[r * D + d] = acc[i];
+      if (d < D && outA) outA[r * D + d] = acc[i];
+      if (d < D && outB) outB[r * D + d] = __float2bfloat16_rn(acc[i]);
     }
   }
   if (lane == 0) outS[r] = lse;
@@ -71,10 +73,10 @@ __global__ void __launch_bounds__(32 * ROWS_PER_CTA)
 }  // namespace
 
 cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,
-                             float* outA, float* outS, cudaStream_t st) {
+                             float* outA, float* outS, cudaStream_t st, bf16* outB) {
   if (R == 0) return cudaSuccess;
   const long long grid = (R + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
-  lse_merge_kernel<<<(unsigned)grid, 32 * ROWS_PER_CTA, 0, st>>>(P, R, D, A, S, outA, outS);
+  lse_merge_kernel<<<(unsigned)grid, 32 * ROWS_PER_CTA, 0, st>>>(P, R, D, A, S, outA, outB, outS);
   return cudaGetLastError();
 }
 

@@ -60,21 +60,26 @@ constexpr int kTileRows = 64;
 // Prefill chunks: each context segment is cut into equal pieces (multiples of
 // 128 keys) so that (batch x kv head) x (256-row pairs) x chunks is about one
 // CTA per SM; the query region is one more chunk.
-star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
+// Context segments [s0, s1) are chunked; the query region is one more chunk
+// when `query` is set.
+star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0, int s0 = 0, int s1 = -1,
+                               bool query = true) {
   const star::CacheView& v = c->view;
+  if (s1 < 0) s1 = v.n_seg;
   star::PrefillPlan pl{};
+  const int nseg = s1 - s0;
   const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
   const long long want = std::max(1LL, (long long)c->num_sms / bgp);
-  const long long per_seg = std::max(1LL, (want - 1) / v.n_seg);
+  const long long per_seg = nseg > 0 ? std::max(1LL, (want - (query ? 1 : 0)) / nseg) : 1;
   long long chunk_len = round_up((v.b + per_seg - 1) / per_seg, 128);
   for (;;) {
     int n = 0;
-    for (int s = 0; s < v.n_seg; ++s) n += (int)((star::seg_len(v, s) + chunk_len - 1) / chunk_len);
+    for (int s = s0; s < s1; ++s) n += (int)((star::seg_len(v, s) + chunk_len - 1) / chunk_len);
     if (n + 1 <= star::kMaxPrefillChunks) break;
     chunk_len *= 2;
   }
   int n = 0;
-  for (int s = 0; s < v.n_seg; ++s) {
+  for (int s = s0; s < s1; ++s) {
     const long long len = star::seg_len(v, s);
     for (long long st = 0; st < len; st += chunk_len) {
       pl.chunk[n].seg = s;
@@ -83,10 +88,13 @@ star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0) {
       ++n;
     }
   }
-  pl.chunk[n].seg = -1;
-  pl.chunk[n].start = 0;
-  pl.chunk[n].len = (int)(len0 + lq);
-  pl.n_chunks = n + 1;
+  if (query) {
+    pl.chunk[n].seg = -1;
+    pl.chunk[n].start = 0;
+    pl.chunk[n].len = (int)(len0 + lq);
+    ++n;
+  }
+  pl.n_chunks = n;
   return pl;
 }
 
@@ -198,8 +206,12 @@ int star_cache_create(const star_params* p, star_cache** out) {
   // admits, and the decode plan at the fullest query region.
   long long partA = 0, partS = 0;
   for (int lq = 1; lq <= p->q_cap; ++lq) {
+    // a plan over any range of segments (star_partial_attend) has at most
+    // max(n_seg, CTAs wanted) + 1 chunks; the full plan is one of them
     star::PrefillPlan pl = plan_prefill(c, lq, 0);
-    const long long rows = (long long)v.B * v.Hkv * pl.n_chunks * v.G * lq;
+    const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
+    const long long nmax = std::max<long long>(pl.n_chunks, std::max<long long>(v.n_seg, c->num_sms / bgp) + 1);
+    const long long rows = (long long)v.B * v.Hkv * std::min<long long>(nmax, star::kMaxPrefillChunks) * v.G * lq;
     partA = std::max(partA, rows * v.D);
     partS = std::max(partS, rows);
   }
@@ -594,12 +606,90 @@ int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
   return STAR_OK;
 }
 
+int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query, int lq, const void* Q,
+                        const void* K, const void* V, float* A, float* s, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  const star::CacheView& w = c->view;
+  if (lq < 1) return fail(STAR_EINVAL, "lq must be >= 1");
+  if (first_seg < 0 || n_seg < 0 || first_seg + n_seg > w.n_seg)
+    return fail(STAR_EINVAL, "segments [%d, %d) outside 0..%d", first_seg, first_seg + n_seg, w.n_seg);
+  if (with_query != 0 && with_query != 1) return fail(STAR_EINVAL, "with_query must be 0 or 1");
+  if (!Q || !A || !s || (with_query && (!K || !V))) return fail(STAR_EINVAL, "NULL tensor pointer");
+  if (!aligned16(Q) || !aligned16(A) || !aligned16(s) || (with_query && (!aligned16(K) || !aligned16(V))))
+    return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (with_query && c->q_len + lq > w.q_cap)
+    return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, w.q_cap);
+  if (lq > w.q_cap) return fail(STAR_EINVAL, "lq %d beyond q_cap %d (the scratch is sized by it)", lq, w.q_cap);
+  const star::PrefillPlan pl = plan_prefill(c, lq, c->q_len, first_seg, first_seg + n_seg, with_query != 0);
+  cudaError_t e = star::launch_query_prefill_tc(
+      w, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+      static_cast<const bf16*>(V), nullptr, s, pl, c->scratch, static_cast<cudaStream_t>(stream), A, nullptr,
+      nullptr, with_query != 0);
+  if (e == cudaSuccess && with_query && w.qK8)
+    e = star::launch_quantize_qregion_fp8(w, static_cast<const bf16*>(K), static_cast<const bf16*>(V),
+                                          (int)c->q_len, lq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "star_partial_attend launch");
+  if (with_query) c->q_len += lq;
+  return STAR_OK;
+}
+
+int star_decode_step_partials(star_cache* c, const void* q, const void* k, const void* v, void* o, float* lse,
+                              float* Ah, float* sh, long long* spans, int max_parts, int* n_parts, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (!Ah || !sh || !spans || !n_parts) return fail(STAR_EINVAL, "NULL partials pointer");
+  const star::CacheView& w = c->view;
+  if (c->q_len + 1 > w.q_cap)
+    return fail(STAR_ENOSPC, "query region full: %lld rows, q_cap %d", c->q_len, w.q_cap);
+  const star::DecodePlan pl = plan_decode(c, c->q_len);
+  std::vector<star::DecodePart> parts;
+  star::decode_parts(w, c->q_len, pl, parts);
+  *n_parts = (int)parts.size();
+  if ((int)parts.size() > max_parts)
+    return fail(STAR_EINVAL, "%d parts do not fit max_parts = %d", (int)parts.size(), max_parts);
+  const int rc = star_decode_step(c, q, k, v, o, lse, stream);
+  if (rc) return rc;
+  // the step left every part in the cache's scratch: [B*Hkv][maxp][G][D] and [B*Hkv][maxp][G]
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rowA = (size_t)w.G * w.D, rowS = (size_t)w.G;
+  cudaError_t e = cudaSuccess;
+  size_t i = 0;
+  while (i < parts.size() && e == cudaSuccess) {
+    size_t j = i;                                    // the parts of one bg are consecutive slots
+    while (j < parts.size() && parts[j].bg == parts[i].bg) ++j;
+    const size_t src = (size_t)parts[i].bg * pl.maxp;
+    e = cudaMemcpyAsync(Ah + i * rowA, c->scratch.partA + src * rowA, (j - i) * rowA * sizeof(float),
+                        cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(sh + i * rowS, c->scratch.partS + src * rowS, (j - i) * rowS * sizeof(float),
+                          cudaMemcpyDeviceToDevice, st);
+    i = j;
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "star_decode_step_partials copies");
+  for (size_t p = 0; p < parts.size(); ++p) {
+    spans[3 * p] = parts[p].bg;
+    spans[3 * p + 1] = parts[p].first;
+    spans[3 * p + 2] = parts[p].end;
+  }
+  return STAR_OK;
+}
+
 int star_selftest_wait_timeout(unsigned polls, int* gave_up, void* stream) {
   if (!gave_up) return fail(STAR_EINVAL, "gave_up is NULL");
   if (polls < 1 || polls > (1u << 22)) return fail(STAR_EINVAL, "polls must be in 1..2^22");
   *gave_up = 0;
   cudaError_t e = star::run_wait_timeout(polls, gave_up, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_selftest_wait_timeout");
+  return STAR_OK;
+}
+
+int star_lse_merge_bf16(int P, long long R, int D, const float* A, const float* s, void* out_O,
+                        float* out_s, void* stream) {
+  if (P < 1 || R < 0 || D < 1 || D > 1024) return fail(STAR_EINVAL, "need P >= 1, R >= 0, 1 <= D <= 1024");
+  if (R == 0) return STAR_OK;
+  if (!A || !s || !out_O || !out_s) return fail(STAR_EINVAL, "NULL tensor pointer");
+  cudaError_t e = star::launch_lse_merge(P, R, D, A, s, nullptr, out_s, static_cast<cudaStream_t>(stream),
+                                         static_cast<bf16*>(out_O));
+  if (e != cudaSuccess) return cuda_fail(e, "star_lse_merge_bf16 launch");
   return STAR_OK;
 }
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <vector>
@@ -140,6 +141,32 @@ struct DecodePlan {
 int decode_max_partials(const CacheView& c, int ncta);
 DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms);
 
+// Span of CTA i: rows [span_start(i), span_start(i + 1)) of the R cached rows
+// of all (batch, kv head) pairs laid end to end.  Row indices stay below 2^31
+// (checked when the cache is made), so both quotients below divide a
+// numerator under 2^53 by at most 2^31.  They are taken in double, which is
+// exact there: the rounding error of the quotient is below 1 / divisor, the
+// least distance of a non-integer quotient from an integer, so its floor is
+// the integer quotient.  (A 64-bit integer division costs several times as
+// long on the device, ahead of the first TMA load.)  Host and device share
+// these two functions, so the host's list of parts is the kernel's.
+__host__ __device__ __forceinline__ long long span_start(long long i, long long R, int n) {
+  return (long long)floor((double)(i * R) / (double)n);
+}
+// CTA whose span holds row x (largest i with span_start(i) <= x).
+__host__ __device__ __forceinline__ int cta_of(long long x, long long R, int n) {
+  return (int)floor((double)((x + 1) * n - 1) / (double)R);
+}
+
+// One part of a decode step: the run of (batch, kv head) bg's cached rows
+// [first, end) (context rows, then query-region rows from L on) that one CTA
+// folds into part slot `slot` of bg.
+struct DecodePart {
+  int bg, slot;
+  long long first, end;
+};
+void decode_parts(const CacheView& c, long long len0, const DecodePlan& pl, std::vector<DecodePart>& out);
+
 // TMA maps of the cache, built once per cache.
 struct DecodeMaps {
   CUtensorMap k_ctx, v_ctx, k_q, v_q;
@@ -164,9 +191,10 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
                                     int len0, const bf16* Q, const bf16* Kq, const bf16* Vq, bf16* O,
                                     float* LSE, const PrefillPlan& plan, const Scratch& s,
                                     cudaStream_t st, float* O32 = nullptr, float* Ah = nullptr,
-                                    float* sh = nullptr);
+                                    float* sh = nullptr, bool append = true);
 
+// outA (float32) or outB (bf16) may be null
 cudaError_t launch_lse_merge(int P, long long R, int D, const float* A, const float* S,
-                             float* outA, float* outS, cudaStream_t st);
+                             float* outA, float* outS, cudaStream_t st, bf16* outB = nullptr);
 
 }  // namespace star

@@ -232,6 +232,40 @@ STAR_API int star_query_prefill_partials(star_cache* c, int lq, const void* Q, c
 STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const void* v,
                      void* o, float* lse, void* stream);
 
+/* Phase-2 partial over part of the cache ([P2] Phase 2 Steps 2-4: every host
+ * attends the broadcast query to its own blocks and returns its local A_h
+ * and s_h), for a caller that spreads the context blocks over several GPUs
+ * and merges the hosts' partials itself (star_lse_merge).  Rows Q
+ * [B][Hq][lq][D] bf16 attend to the context segments [first_seg, first_seg +
+ * n_seg) and, when with_query = 1, to the query region after K, V
+ * [B][Hkv][lq][D] are appended to it (causal, as star_query_prefill; lq = 1
+ * is a generation step).  With with_query = 0 the query region is neither
+ * read nor written and K, V may be NULL.  Outputs, float32: A [B][Hq][lq][D]
+ * the normalised local attention output, s [B][Hq][lq] its natural-log LSE
+ * of the scaled logits (A = 0, s = -inf for a row that sees no key).
+ * 1 <= lq <= q_cap.  STAR_ENOSPC if with_query and the region is full. */
+STAR_API int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query, int lq,
+                                 const void* Q, const void* K, const void* V, float* A, float* s,
+                                 void* stream);
+
+/* Debug form of star_decode_step ([P2] Phase 2 Steps 3 and 5): the same
+ * step, append, o and lse, and the decode kernel's own partials.  The cached
+ * rows of every (batch, kv head) -- context tokens 0..L-1, then query-region
+ * rows at L + r -- are split over the kernel's CTAs; each piece one CTA folds
+ * is one part:
+ *   Ah [P][G][D], sh [P][G] float32: the part's local output A_h (normalised)
+ *       and s_h (natural-log LSE of the scaled logits) for the G q heads of
+ *       its kv head;
+ *   spans [P][3]: (b*Hkv + kv head, first row, end row) of the part, host
+ *       memory, written before the call returns.
+ * The step's own new token is one more part the kernel folds in at the merge
+ * (s = scale * q.k, A = v); it is not listed.  P is written to *n_parts;
+ * STAR_EINVAL (nothing launched) when P > max_parts.  For tests and
+ * inspection: slower than star_decode_step by the copies. */
+STAR_API int star_decode_step_partials(star_cache* c, const void* q, const void* k, const void* v,
+                                       void* o, float* lse, float* Ah, float* sh, long long* spans,
+                                       int max_parts, int* n_parts, void* stream);
+
 /* Phase 2 merge of P partials ([P2] Phase 2 Step 5; [P3] s_global, A_global):
  * A [P][R][D], s [P][R] float32 (s_h as natural-log LSE, -inf = empty part)
  * -> out_A [R][D] = sum_h exp(s_h - s) A_h, out_s [R] = s = log sum_h
@@ -239,6 +273,12 @@ STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const
  * R >= 0, 1 <= D <= 1024.  out_* must not alias the inputs. */
 STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const float* s,
                    float* out_A, float* out_s, void* stream);
+
+/* The same merge with the output rounded once to bf16 (nearest even): out_O
+ * [R][D] bf16, out_s [R] float32 -- the last step on the query host when the
+ * partials come from several GPUs ([P2] Phase 2 Steps 4-5). */
+STAR_API int star_lse_merge_bf16(int P, long long R, int D, const float* A, const float* s,
+                                 void* out_O, float* out_s, void* stream);
 
 /* Self-test of the failure path every pipelined kernel here uses: one CTA
  * waits, with the kernels' bounded mbarrier wait limited to `polls` polls

@@ -71,8 +71,13 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.star_lse_merge(0, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(1, 4, 2000, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_lse_merge(1, 0, 8, None, None, None, None, None) == _abi.STAR_OK
+    assert lib.star_lse_merge_bf16(0, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_lse_merge_bf16(1, 4, 8, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_ctx_encode(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_ctx_encode_fp32(None, *([None] * 7)) == _abi.STAR_EINVAL
+    assert lib.star_partial_attend(None, 0, 1, 0, 1, *([None] * 6)) == _abi.STAR_EINVAL
+    n = ctypes.c_int(-1)
+    assert lib.star_decode_step_partials(None, *([None] * 8), 0, ctypes.byref(n), None) == _abi.STAR_EINVAL
     assert lib.star_decode_step(None, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_query_prefill(None, 4, None, None, None, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_query_prefill_partials(None, 4, *([None] * 9)) == _abi.STAR_EINVAL

@@ -113,3 +113,86 @@ def test_partials_form_agrees_with_the_fast_path():
     assert (O1 - O2).abs().max().item() <= MAX_ABS and (L1 - L2).abs().max().item() <= LSE_ABS
     assert torch.equal(k1.view(torch.int16), k2.view(torch.int16))
     assert torch.equal(v1.view(torch.int16), v2.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# The decode kernel's own partials: one per piece of cached rows a CTA folds.
+# ---------------------------------------------------------------------------
+DECODE_VARIANTS = {
+    "tiny": {},
+    "ragged-anchor-shorter": dict(L=1000, b=256, b_a=100, lq=11, T=2),
+    # 32 (batch, kv head) pairs of about 100 rows on a few CTAs: spans cross pairs
+    "many-heads-short": dict(B=4, Hq=16, Hkv=8, D=64, L=96, b=32, b_a=32, lq=5, T=2),
+    "8b-32k": None,
+}
+
+
+def check_decode_parts(parts, x_cpu, t, segs, qk, qv, w, what):
+    """Every listed part against the oracle's local partial over its rows; the
+    parts of each (batch, kv head) tile its cached rows exactly; their merge,
+    with the step's own token as one more part, gives o and lse."""
+    o, lse, Ah, sh, spans = parts
+    G = w.Hq // w.Hkv
+    rpb = w.L + w.lq + t                         # rows cached before the step
+    A = Ah.double().cpu().numpy()
+    S = sh.double().cpu().numpy()
+    q = x_cpu["qd"][t].double().numpy()
+    for bg in range(w.B * w.Hkv):
+        bi, g = divmod(bg, w.Hkv)
+        idx = np.nonzero(spans[:, 0] == bg)[0]
+        assert len(idx) >= 1, f"{what}: no part for pair {bg}"
+        rng_ = spans[idx, 1:]
+        assert rng_[0, 0] == 0 and rng_[-1, 1] == rpb and np.all(rng_[1:, 0] == rng_[:-1, 1]), \
+            f"{what}: parts of pair {bg} do not tile its {rpb} rows"
+        kc = np.concatenate([so._f64(s[2][bi, g]) for s in segs] + [qk[bi, g, :w.lq + t]], axis=0)
+        vc = np.concatenate([so._f64(s[3][bi, g]) for s in segs] + [qv[bi, g, :w.lq + t]], axis=0)
+        qh = q[bi, g * G:(g + 1) * G, 0]
+        parts_a, parts_s = [], []
+        for p, (x0, x1) in zip(idx, rng_):
+            a_ref, s_ref = so.local_partial(qh, kc[x0:x1], vc[x0:x1], w.scale)
+            err = np.abs(A[p] - a_ref)
+            assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, f"{what}: part {p} A_h max {err.max():.3e}"
+            assert np.abs(S[p] - s_ref).max() <= LSE_ABS, f"{what}: part {p} s_h"
+            parts_a.append(A[p])
+            parts_s.append(S[p])
+        # the token itself: s = scale q.k_new, A = v_new
+        kn, vn = qk[bi, g, w.lq + t], qv[bi, g, w.lq + t]
+        parts_a.append(np.repeat(vn[None], G, axis=0))
+        parts_s.append(w.scale * (qh @ kn))
+        m_a, m_s = so.lse_merge(np.stack(parts_a), np.stack(parts_s))
+        og = o[bi, g * G:(g + 1) * G, 0].double().cpu().numpy()
+        assert np.abs(og - m_a).max() <= MAX_ABS, f"{what}: merge of the parts != o"
+        assert np.abs(lse[bi, g * G:(g + 1) * G].double().cpu().numpy() - m_s).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("variant", list(DECODE_VARIANTS))
+def test_decode_kernel_partials_match_the_oracle(variant):
+    from block_sparse_long_phase_b200 import StarCache
+    if DECODE_VARIANTS[variant] is None:
+        w = wl.get(variant).with_(T=2)
+        x = wl.make_inputs(w, "cuda")
+        cpu = {k: v.cpu() for k, v in x.items() if k != "Qc"}
+    else:
+        w = wl.get("tiny").with_(**DECODE_VARIANTS[variant])
+        cpu = wl.make_inputs(w, "cpu")
+        x = {k: v.cuda() for k, v in cpu.items()}
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+    cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
+    cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
+    got = []
+    for t in range(w.T):
+        got.append(cache.star_decode_step_partials(x["qd"][t], x["kd"][t], x["vd"][t]))
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    segs = so.cache_segments(cpu["Kc"], cpu["Vc"], w.b)
+    qk = np.zeros((w.B, w.Hkv, w.lq + w.T, w.D))
+    qv = np.zeros_like(qk)
+    qk[:, :, :w.lq] = cpu["Kq"].double().numpy()
+    qv[:, :, :w.lq] = cpu["Vq"].double().numpy()
+    for t in range(w.T):
+        qk[:, :, w.lq + t] = cpu["kd"][t][:, :, 0].double().numpy()
+        qv[:, :, w.lq + t] = cpu["vd"][t][:, :, 0].double().numpy()
+        check_decode_parts(got[t], cpu, t, segs, qk, qv, w, f"{variant} step {t}")
+        if variant == "8b-32k":
+            assert len(got[t][4]) > 2 * w.B * w.Hkv          # several CTAs per (batch, kv head)
+    cache.close()

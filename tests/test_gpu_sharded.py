@@ -1,0 +1,104 @@
+"""The block-sharded layer's kernels on one GPU, its ranks run one after another.
+
+Every run here gets one GPU, so the ranks of the multi-GPU layer
+(block_sparse_long_phase_b200/sharded.py) are emulated in one process: each
+rank's cache, its phase 1 on the local [anchor | zeros | own blocks] layout,
+and its phase-2 partial (star_partial_attend) run on the GPU in turn; the
+partials are stacked as all_gather would leave them and merged with
+star_lse_merge_bf16.  No collective is issued and no kernel waits for
+another.  Against the single-device fp64 oracle, at the parity bar.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_phase_b200 import workloads as wl
+from block_sparse_long_phase_b200.sharded import ShardedStarCache
+from oracle import star_oracle as so
+
+from test_gpu_parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (2, dict(L=1024, b=256, b_a=256, lq=5, T=2)),
+    (3, dict(L=1000, b=256, b_a=100, lq=4, T=2)),
+    (4, dict(L=700, b=128, b_a=64, B=2, Hq=8, Hkv=2, D=128, lq=3, T=2)),
+    (3, dict(L=300, b=256, b_a=256, lq=3, T=1)),       # a rank without blocks
+    (8, dict(L=4096, b=512, b_a=512, Hq=16, Hkv=4, D=128, lq=16, T=3)),
+]
+
+
+@pytest.mark.parametrize("world,shape", CASES)
+def test_sharded_kernels_match_the_oracle(world, shape):
+    w = wl.get("tiny").with_(**shape)
+    cpu = wl.make_inputs(w, "cpu")
+    x = {k: v.cuda() for k, v in cpu.items()}
+    ranks = [ShardedStarCache(r, world, w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+             for r in range(world)]
+    # phase 1, rank by rank
+    O = torch.empty_like(x["Qc"])
+    LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device="cuda")
+    for sc in ranks:
+        lay = sc.layout
+        r0, r1 = lay.rows0, lay.rows0 + lay.rows
+        o, l = sc.encode(x["Qc"][:, :, r0:r1].contiguous(), x["Kc"][:, :, r0:r1].contiguous(),
+                         x["Vc"][:, :, r0:r1].contiguous(), x["Kc"][:, :, :w.b_a].contiguous(),
+                         x["Vc"][:, :, :w.b_a].contiguous())
+        O[:, :, r0:r1] = o
+        LSE[:, :, r0:r1] = l
+    torch.cuda.synchronize()
+    Oref, Lref = so.ctx_encode(cpu["Qc"], cpu["Kc"], cpu["Vc"], w.b, w.b_a, w.scale)
+    assert_close(O, Oref, LSE, Lref, f"sharded x{world} phase 1")
+    # each rank's cache holds exactly its own blocks' rows
+    for sc in ranks:
+        lay = sc.layout
+        for j in range(lay.n_blocks):
+            k, v, seg = sc.cache.segment_tensors(lay.first_seg + j)
+            s0 = (lay.first_block + j) * w.b
+            assert torch.equal(k.view(torch.int16), x["Kc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
+            assert torch.equal(v.view(torch.int16), x["Vc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
+
+    def step(Q, K, V):
+        parts = [sc.local_partial(Q, K, V) for sc in ranks]
+        A = torch.stack([p[0] for p in parts])
+        s = torch.stack([p[1] for p in parts])
+        return ranks[-1].merge(A, s)
+
+    Oq, Lq = step(x["Qq"], x["Kq"], x["Vq"])
+    dec = [step(x["qd"][t], x["kd"][t], x["vd"][t]) for t in range(w.T)]
+    torch.cuda.synchronize()
+    segs = so.cache_segments(cpu["Kc"], cpu["Vc"], w.b)
+    region = np.zeros((w.B, w.Hkv, w.lq + w.T, w.D))
+    ref, lref, qk, qv = so.query_prefill(cpu["Qq"], cpu["Kq"], cpu["Vq"], segs, region, region, 0, w.scale)
+    assert_close(Oq, ref, Lq, lref, f"sharded x{world} prefill")
+    for t in range(w.T):
+        ref, lref, qk, qv = so.decode_step(cpu["qd"][t], cpu["kd"][t], cpu["vd"][t], segs, qk, qv, w.lq + t, w.scale)
+        assert_close(dec[t][0], ref, dec[t][1], lref, f"sharded x{world} decode {t}")
+    assert [sc.cache.q_len for sc in ranks] == [0] * (world - 1) + [w.lq + w.T]
+    for sc in ranks:
+        assert sc.cache.device_error() == 0
+        sc.close()
+
+
+def test_partial_attend_over_every_segment_equals_the_prefill():
+    """star_partial_attend over all segments with the query region gives the
+    prefill's rows (float32 before the rounding), and over no segment and no
+    query region it gives empty rows (A = 0, s = -inf)."""
+    from block_sparse_long_phase_b200 import StarCache
+    w = wl.get("tiny").with_(L=1000, b=256, b_a=100, lq=6, T=0)
+    x = {k: v.cuda() for k, v in wl.make_inputs(w, "cpu").items()}
+    a = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq, w.scale)
+    b = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq, w.scale)
+    a.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
+    b.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
+    O, L = a.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
+    A, s = b.star_partial_attend(x["Qq"], 0, b.num_segments - 1, x["Kq"], x["Vq"])
+    A0, s0 = b.star_partial_attend(x["Qq"], 0, 0)
+    torch.cuda.synchronize()
+    assert (O.double() - A.double()).abs().max().item() <= 1e-2
+    assert (L - s).abs().max().item() <= 1e-3
+    assert (A0 == 0).all() and torch.isinf(s0).all() and (s0 < 0).all()
+    a.close()
+    b.close()

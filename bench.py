@@ -556,6 +556,37 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def profile_case(args):
+    """Launches of one kernel for an ncu capture (no bench line): ``phase1``
+    runs star_ctx_encode ``steps`` times, ``decode`` runs phase 1 and the query
+    prefill once and then ``steps`` decode steps.  ``--blocks N`` keeps the
+    first N blocks of the workload (a capture small enough to replay)."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+    torch.cuda.set_device(0)
+    w = wl.get(args.workload)
+    if args.blocks:
+        w = w.with_(L=min(w.L, args.blocks * w.b))
+    if args.profile == "decode":
+        w = w.with_(T=max(w.T, args.steps))
+    x = wl.make_inputs(w, "cuda")
+    cache = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale, kv_fp8=args.kv_fp8)
+    O = torch.empty_like(x["Qc"])
+    LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device="cuda")
+    n = args.steps if args.profile == "phase1" else 1
+    for _ in range(n):
+        cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"], O, LSE)
+    if args.profile == "decode":
+        cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
+        for t in range(args.steps):
+            cache.star_decode_step(x["qd"][t], x["kd"][t], x["vd"][t])
+    torch.cuda.synchronize()
+    if cache.device_error():
+        raise SystemExit("a kernel gave up a bounded wait")
+    cache.close()
+    print(f"profile case {args.profile}: {w.name} L={w.L} kv_fp8={args.kv_fp8} launches={args.steps}")
+
+
 def host_buffers(x, O, LSE):
     """Host copies of the phase-1 inputs and room for its outputs, page-locked
     in place (cudaHostRegister of exactly their bytes); pageable if the host
@@ -598,9 +629,15 @@ def main():
                     help="skip phase 1 / prefill / decode on the other configurations")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the phase-1 variants (anchor shorter than the block, ragged context, batch 4)")
+    ap.add_argument("--profile", choices=["phase1", "decode"],
+                    help="only launch this kernel `steps` times for an ncu capture (no bench line)")
+    ap.add_argument("--blocks", type=int, default=0, help="--profile: keep the first N blocks")
+    ap.add_argument("--kv-fp8", action="store_true", help="--profile decode: stream the FP8 cache")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return profile_case(args)
 
     import torch
     from block_sparse_long_phase_b200 import StarCache, workloads as wl

@@ -8,7 +8,9 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libstar.so")
+# STAR_LIB=checked selects the bounds-checked build (lib/libstar_checked.so)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                        "libstar_checked.so" if os.environ.get("STAR_LIB") == "checked" else "libstar.so")
 
 STAR_OK = 0
 STAR_EINVAL = -1
@@ -26,7 +28,7 @@ EXPORTS = (
     "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
     "star_selftest_wait_timeout", "star_noalloc_device_error", "star_ctx_encode_fp32",
     "star_decode_step_partials", "star_partial_attend",
-    "star_lse_merge_bf16",
+    "star_lse_merge_bf16", "star_cache_check_guards",
 )
 
 
@@ -80,6 +82,7 @@ def load(path: str = LIB_PATH):
                                              vp, vp, vp, vp, vp, vp]
     lib.star_noalloc_device_error.argtypes = [ctypes.POINTER(i), vp]
     lib.star_ctx_encode_fp32.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.star_cache_check_guards.argtypes = [vp, ctypes.POINTER(i)]
     lib.star_lse_merge_bf16.argtypes = [i, ll, i, vp, vp, vp, vp, vp]
     lib.star_partial_attend.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step_partials.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ll), i,

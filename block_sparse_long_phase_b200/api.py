@@ -132,6 +132,13 @@ class StarCache:
         _abi.check(self.lib.star_cache_device_error(self.handle, ctypes.byref(f)))
         return f.value
 
+    def check_guards(self):
+        """(-1, "") if every canary guard of the cache is intact, else (index of
+        the first overwritten guard, which part it follows)."""
+        f = ctypes.c_int()
+        _abi.check(self.lib.star_cache_check_guards(self.handle, ctypes.byref(f)))
+        return f.value, (self.lib.star_last_error().decode() if f.value >= 0 else "")
+
     @property
     def q_len(self) -> int:
         return self.segment(self.num_segments - 1).len

@@ -52,7 +52,8 @@ using namespace sm100;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 128;          // keys per K/V tile
-constexpr int NBUF = 4;          // K/V ring slots
+constexpr int NBUF = 4;          // K/V ring slots, phase 1
+constexpr int NBUF_PF = 5;       // prefill: its tiles stream from HBM, one more in flight
 constexpr int NTHREADS = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
@@ -77,6 +78,7 @@ struct CtxTcArgs {
   int lq, len0, row_pairs;
   float* partA;
   float* partS;
+  long long part_rows;   // rows the scratch holds (partS elements)
   PrefillPlan plan;
 };
 static_assert(sizeof(CtxTcArgs) <= 4096, "kernel parameters beyond 4 KB");
@@ -107,19 +109,78 @@ SM100_DEV float fmax3(float a, float b, float c) {
   return d;
 }
 
-template <int D>
+template <int D, int NB>
 struct Smem {
   static constexpr int TILE = BM * D * 2;           // one Q or K/V tile, bytes
   static constexpr int HALF = BM * 128;             // one 64-column (128 B) half
   static constexpr int Q0 = 0;
   static constexpr int Q1 = TILE;
   static constexpr int RING = 2 * TILE;
-  static constexpr int BYTES = RING + NBUF * TILE;  // + barriers in static smem
+  static constexpr int BYTES = RING + NB * TILE;    // + barriers in static smem
 };
+static_assert(Smem<128, NBUF_PF>::BYTES + 1024 <= 227 * 1024, "prefill ring beyond shared memory");
+
+// The 128-key tiles of one prefill span [x, x1) of a (batch, kv head)'s key
+// rows, numbered over the context (0..L-1) and then the query region (L..).
+// A tile never crosses the end of a context segment or of the context; for
+// each one: its first row in the TMA map it is read through (the context
+// cache, or the query region from row L on), its key count, and for the query
+// region the region row of its first key.  The producer and every softmax
+// thread walk the same sequence.
+struct TileWalk {
+  long long x, x1, seg_end;
+  int seg;                                          // -1 once in the query region
+  __device__ __forceinline__ void start(long long x0, long long xe, const CacheView& c) {
+    x = x0;
+    x1 = xe;
+    seg = x0 < c.L ? (int)(x0 / c.b) : -1;
+    seg_end = seg >= 0 ? min((long long)(seg + 1) * c.b, c.L) : xe;
+  }
+  __device__ __forceinline__ int next(const CacheView& c, int bg, int& row, bool& region, int& r0) {
+    if (seg >= 0 && x >= seg_end) {
+      if (x < c.L) {
+        ++seg;
+        seg_end = min((long long)(seg + 1) * c.b, c.L);
+      } else {
+        seg = -1;
+        seg_end = x1;
+      }
+    }
+    const long long end = seg_end < x1 ? seg_end : x1;
+    const int n = (int)(end - x < BN ? end - x : BN);
+    if (seg >= 0) {
+      row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * seg_len(c, seg) + (x - (long long)seg * c.b));
+      region = false;
+      r0 = 0;
+    } else {
+      r0 = (int)(x - c.L);
+      row = (int)((long long)bg * c.q_cap + r0);
+      region = true;
+    }
+    x += n;
+    return n;
+  }
+};
+
+// Tiles of span [x0, x1): one term per segment it overlaps, then the region.
+__device__ __forceinline__ int span_tiles(long long x0, long long x1, const CacheView& c) {
+  int n = 0;
+  long long x = x0;
+  while (x < x1 && x < c.L) {
+    const int seg = (int)(x / c.b);
+    long long e = min((long long)(seg + 1) * c.b, c.L);
+    if (e > x1) e = x1;
+    n += (int)((e - x + BN - 1) / BN);
+    x = e;
+  }
+  if (x < x1) n += (int)((x1 - x + BN - 1) / BN);
+  return n;
+}
 
 template <int D, bool PF>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_constant__ CtxTcArgs a) {
-  using S = Smem<D>;
+  constexpr int NBUF = PF ? NBUF_PF : ::star::NBUF;
+  using S = Smem<D, NBUF>;
   constexpr int NH = D / 64;                          // 128-byte halves per row
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -168,10 +229,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
     n_rows0 = rows_total - r0 < BM ? rows_total - r0 : BM;
     n_rows1 = rows_total - r0 - BM < BM ? rows_total - r0 - BM : BM;
     t0 = r0;                                                // packed row of Q0's first row
-    n_kv = (a.plan.chunk[chunk].len + BN - 1) / BN;
-    const PrefillChunk ch = a.plan.chunk[chunk];
-    kv_row0 = ch.seg >= 0 ? (long long)ch.seg * c.B * c.Hkv * c.b + (long long)bg * seg_len(c, ch.seg) + ch.start
-                          : (long long)bg * c.q_cap;
+    n_kv = span_tiles(a.plan.span[chunk].x0, a.plan.span[chunk].x1, c);
+    kv_row0 = 0;
     qrow0 = ((long long)bb * c.Hq + (long long)g * c.G) * a.lq + r0;   // Q1 is 128 rows later
   }
 
@@ -205,12 +264,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
   if (warp == 0) {
     // ------------------------------ TMA producer -----------------------------
     if (elect_one()) {
-      const bool qregion = PF && a.plan.chunk[chunk].seg < 0;
-      const CUtensorMap* mk = qregion ? &a.tkq : &a.tk;
-      const CUtensorMap* mv = qregion ? &a.tvq : &a.tv;
+      const CUtensorMap* mk = &a.tk;
+      const CUtensorMap* mv = &a.tv;
       prefetch_tmap(&a.tq);
       prefetch_tmap(mk);
       prefetch_tmap(mv);
+      TileWalk walk;
+      if (PF) {
+        walk.start(a.plan.span[chunk].x0, a.plan.span[chunk].x1, c);
+        if (a.plan.span[chunk].x1 > c.L) {
+          prefetch_tmap(&a.tkq);
+          prefetch_tmap(&a.tvq);
+        }
+      }
+      int pf_row = 0;
+      bool pf_region = false;
       const bool own_anchor = !PF && a.anchor_keys && blk > 0;   // per-block anchor keys
       if (own_anchor) prefetch_tmap(&a.tkq);
       const uint32_t qb = smem_u32(&bar_q_full);
@@ -227,10 +295,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         const int j = i >> 1, slot = i % NBUF, use = i / NBUF;
         if (use > 0 && !mbar_wait(smem_u32(&bar_kv_empty[slot]), (use - 1) & 1)) { fail(); break; }
         if (*(volatile int*)&abort_s) break;
-        const long long tok = PF ? (long long)j * BN
-                                 : (j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN);
+        const long long tok = PF ? 0 : (j < n_anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN);
         int row = (int)(kv_row0 + tok);
         const CUtensorMap* m = (i & 1) ? mv : mk;
+        if (PF) {
+          if (!(i & 1)) {                                  // K comes first: step to the next tile
+            int r0u;
+            walk.next(c, bg, pf_row, pf_region, r0u);
+          }
+          row = pf_row;
+          if (pf_region) m = (i & 1) ? &a.tvq : &a.tkq;
+        }
         if (own_anchor && !(i & 1) && j < n_anchor) {
           // K of block blk's anchor: rows of Ka[blk - 1] for this (batch, kv head)
           m = &a.tkq;
@@ -315,8 +390,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
                               ((long long)bg * len + (t0 - bstart)) * D;
       const long long gbase = (kv_row0 + t0) * D;
       constexpr int CPR = D / 8;
+      const long long kv_elems = (long long)c.B * c.Hkv * c.L * D;
       for (int i = tid - 64; i < n_rows * CPR; i += 64) {
         const int r = i / CPR, ch = i - (i / CPR) * CPR;
+        if (!STAR_STORE_OK(sbase + (long long)r * D + ch * 8 + 7, kv_elems, a.err) ||
+            !STAR_STORE_OK(gbase + (long long)r * D + ch * 8 + 7, kv_elems, a.err))
+          continue;
         const uint4 kv = *reinterpret_cast<const uint4*>(a.K + gbase + (long long)r * D + ch * 8);
         const uint4 vv = *reinterpret_cast<const uint4*>(a.V + gbase + (long long)r * D + ch * 8);
         *reinterpret_cast<uint4*>(c.ctxK + sbase + (long long)r * D + ch * 8) = kv;
@@ -333,11 +412,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       const uint32_t tO = tmem + lane_off + 256 + q * D;
       const long long pos = t0 + (PF ? q * BM : 0) + r;  // token (phase 1) / packed row (prefill)
       const int n_rows = q ? (n_rows1 > 0 ? n_rows1 : 0) : n_rows0;
-      // prefill: keys visible to this row in the chunk are [0, lim_pf)
-      long long lim_pf = 0;
+      // prefill: this row sees query-region rows 0..len0 + (its query index)
+      TileWalk walk;
+      long long q_lim = 0;
       if (PF) {
-        const PrefillChunk ch = a.plan.chunk[chunk];
-        lim_pf = ch.seg >= 0 ? ch.len : a.len0 + (pos % a.lq) + 1;
+        walk.start(a.plan.span[chunk].x0, a.plan.span[chunk].x1, c);
+        q_lim = a.len0 + (pos % a.lq) + 1;
       }
       float m_used = -INFINITY, l = 0.f;
       const float sl2 = a.scale_log2;
@@ -351,8 +431,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         // mask: phase 1 -- anchor tail (keys >= b_a) and the causal diagonal;
         // prefill -- chunk tail, or the causal query region
         const bool anchor = !PF && j < n_anchor;
-        const long long k0 = (PF || anchor) ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
-        const long long lim = PF ? lim_pf : (anchor ? (long long)c.b_a : pos + 1);   // keys < lim visible
+        long long k0 = anchor ? (long long)j * BN : bstart + (long long)(j - n_anchor) * BN;
+        long long lim = anchor ? (long long)c.b_a : pos + 1;     // keys < lim visible
+        if (PF) {
+          // the tile's keys are [0, n) of the walk; in the query region only
+          // those up to this row's own position
+          int row_u, r0;
+          bool region;
+          const int n = walk.next(c, bg, row_u, region, r0);
+          k0 = 0;
+          lim = region ? (q_lim - r0 < n ? q_lim - r0 : n) : n;
+        }
         if (k0 + BN > lim) {
           const int nvis = (int)(lim - k0 < 0 ? 0 : lim - k0);   // visible columns: [0, nvis)
 #pragma unroll
@@ -423,13 +512,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       if (!PF) {
         const int h = h0 + q;
         const long long orow_i = ((long long)bb * c.Hq + h) * c.L + pos;
+        const bool row_ok = r >= n_rows || STAR_STORE_OK(orow_i, (long long)c.B * c.Hq * c.L, a.err);
         bf16* orow = a.O + orow_i * D;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
-          if (r < n_rows) {
+          if (r < n_rows && row_ok) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv);
             uint32_t pk[16];
@@ -447,16 +537,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
             }
           }
         }
-        if (r < n_rows) a.LSE[((long long)bb * c.Hq + h) * c.L + pos] = lse;
+        if (r < n_rows && row_ok) a.LSE[orow_i] = lse;
       } else {
-        const long long prow = ((long long)bg * a.plan.n_chunks + chunk) * (c.G * a.lq) + pos;
+        const long long prow = ((long long)bg * a.plan.n_spans + chunk) * (c.G * a.lq) + pos;
+        const bool row_ok = r >= n_rows || STAR_STORE_OK(prow, a.part_rows, a.err);
         float* arow = a.partA + prow * D;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tO + cc * 32, o);
           tmem_wait_ld();
-          if (r < n_rows) {
+          if (r < n_rows && row_ok) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               reinterpret_cast<float4*>(arow + cc * 32)[v] =
@@ -464,7 +555,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
                               __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
           }
         }
-        if (r < n_rows) a.partS[prow] = lse;
+        if (r < n_rows && row_ok) a.partS[prow] = lse;
       }
     }
   }
@@ -565,18 +656,25 @@ void ctx_tc_fill_units(const CacheView& c, int num_sms, std::vector<CtxUnit>& un
   }
 }
 
+template <int D, bool PF>
+constexpr int smem_bytes() {
+  return Smem<D, PF ? NBUF_PF : NBUF>::BYTES + 1024;
+}
+
 cudaError_t attn_tc_prepare(int D) {
   cudaError_t e;
   if (D == 128) {
-    const int smem = Smem<128>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes<128, false>());
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem_bytes<128, true>());
   } else {
-    const int smem = Smem<64>::BYTES + 1024;
-    e = cudaFuncSetAttribute(attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem_bytes<64, false>());
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem_bytes<64, true>());
   }
   return e;
 }
@@ -607,9 +705,9 @@ cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q,
   a.work = work;
   a.err = err;
   if (c.D == 128)
-    attn_tc_kernel<128, false><<<n_work, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
+    attn_tc_kernel<128, false><<<n_work, NTHREADS, smem_bytes<128, false>(), st>>>(a);
   else
-    attn_tc_kernel<64, false><<<n_work, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+    attn_tc_kernel<64, false><<<n_work, NTHREADS, smem_bytes<64, false>(), st>>>(a);
   return cudaGetLastError();
 }
 
@@ -628,6 +726,7 @@ __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, 
     const int ch = (int)(i - row * cpr);
     const int bg = (int)(row / lq), t = (int)(row - (long long)bg * lq);
     const long long dst = (((long long)bg * c.q_cap) + len0 + t) * cpr + ch;
+    if (!STAR_STORE_OK(dst, (long long)c.B * c.Hkv * c.q_cap * cpr, c.err)) continue;
     reinterpret_cast<uint4*>(c.qK)[dst] = K[i];
     reinterpret_cast<uint4*>(c.qV)[dst] = V[i];
   }
@@ -642,9 +741,10 @@ __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, 
 // Ah / sh, every chunk's partial in [chunk][B][Hq][lq] row order.  O may be
 // null when only the float32 rows are wanted (a partial over part of the cache).
 constexpr int kMergeWarps = 4;
-constexpr int kSPerLane = (kMaxPrefillChunks + 31) / 32;
+constexpr int kSPerLane = (kMaxPrefillSpans + 31) / 32;
 template <int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) prefill_merge_kernel(CacheView c, int lq, int n_chunks,
+                                                                        long long part_rows,
                                                                         const float* __restrict__ partA,
                                                                         const float* __restrict__ partS,
                                                                         bf16* __restrict__ O,
@@ -664,6 +764,9 @@ __global__ void __launch_bounds__(32 * kMergeWarps) prefill_merge_kernel(CacheVi
   const int rr = m % lq;
   const long long orow_i = ((long long)bb * c.Hq + h) * lq + rr;   // row of O / LSE
   const long long prow0 = bg * n_chunks * rows_total + m;          // chunk p's row: prow0 + p * rows_total
+  if (!STAR_STORE_OK(orow_i, (long long)c.B * c.Hq * lq, c.err) ||
+      (n_chunks > 0 && !STAR_STORE_OK(prow0 + (long long)(n_chunks - 1) * rows_total, part_rows, c.err)))
+    return;
   float sv[kSPerLane];
   float mx = -INFINITY;
 #pragma unroll
@@ -750,6 +853,7 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
   a.row_pairs = prefill_row_pairs(c, lq);
   a.partA = s.partA;
   a.partS = s.partS;
+  a.part_rows = s.partS_elems;
   a.plan = plan;
   if (append) {
     const long long n16 = (long long)c.B * c.Hkv * lq * (c.D / 8);
@@ -757,19 +861,19 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
     query_append_kernel<<<agrid, 256, 0, st>>>(c, lq, len0, reinterpret_cast<const uint4*>(Kq),
                                                reinterpret_cast<const uint4*>(Vq));
   }
-  const int grid = c.B * c.Hkv * a.row_pairs * plan.n_chunks;
+  const int grid = c.B * c.Hkv * a.row_pairs * plan.n_spans;
   if (grid > 0) {
     if (c.D == 128)
-      attn_tc_kernel<128, true><<<grid, NTHREADS, Smem<128>::BYTES + 1024, st>>>(a);
+      attn_tc_kernel<128, true><<<grid, NTHREADS, smem_bytes<128, true>(), st>>>(a);
     else
-      attn_tc_kernel<64, true><<<grid, NTHREADS, Smem<64>::BYTES + 1024, st>>>(a);
+      attn_tc_kernel<64, true><<<grid, NTHREADS, smem_bytes<64, true>(), st>>>(a);
   }
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
   const int mgrid = (int)((rows + kMergeWarps - 1) / kMergeWarps);
   if (c.D == 128)
-    prefill_merge_kernel<128><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
+    prefill_merge_kernel<128><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_spans, s.partS_elems, s.partA, s.partS, O, LSE, O32, Ah, sh);
   else
-    prefill_merge_kernel<64><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_chunks, s.partA, s.partS, O, LSE, O32, Ah, sh);
+    prefill_merge_kernel<64><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_spans, s.partS_elems, s.partA, s.partS, O, LSE, O32, Ah, sh);
   return cudaGetLastError();
 }
 

@@ -80,6 +80,7 @@ struct DecodeArgs {
   float* lse;                   // [B][Hq]
   float* partA;                 // [B*Hkv][maxp][G][D]
   float* partS;                 // [B*Hkv][maxp][G]
+  long long part_rows;          // rows the scratch holds (partS elements)
   unsigned* tickets;            // [B*Hkv] rows folded into parts (kept at 0 between steps)
   int* err;
 };
@@ -299,6 +300,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         const long long qo = q_row_offset(c, bb, g, a.len0);
         const uint4* kn = reinterpret_cast<const uint4*>(a.k + (long long)bg * D);
         const uint4* vn = reinterpret_cast<const uint4*>(a.v + (long long)bg * D);
+        if (!STAR_STORE_OK(qo + D - 1, (long long)c.B * c.Hkv * c.q_cap * D, a.err)) continue;
         if (lane < D / 8) reinterpret_cast<uint4*>(c.qK + qo)[lane] = kn[lane];
         else if (lane >= 16 && lane < 16 + D / 8) reinterpret_cast<uint4*>(c.qV + qo)[lane - 16] = vn[lane - 16];
         if (FP8) {
@@ -697,11 +699,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         }
         const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
         const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
-        uint2 pk;
-        pk.x = pack_bf16(at.x * inv, at.y * inv);
-        pk.y = pack_bf16(at.z * inv, at.w * inv);
-        *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
-        if (d4 == 0) a.lse[orow] = Lt > 0.f ? Mt + __logf(Lt) : -INFINITY;
+        // (no early exit here: every consumer thread must reach the barrier below)
+        if (STAR_STORE_OK(orow, (long long)c.B * c.Hq, a.err)) {
+          uint2 pk;
+          pk.x = pack_bf16(at.x * inv, at.y * inv);
+          pk.y = pack_bf16(at.z * inv, at.w * inv);
+          *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+          if (d4 == 0) a.lse[orow] = Lt > 0.f ? Mt + __logf(Lt) : -INFINITY;
+        }
       }
       named_sync(1, NT);
     }
@@ -772,6 +777,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
           acc += f * comb[(w * 4 + r) * D + d];
         }
         const long long pr = ((long long)bg * a.maxp + pslot) * G + rr;
+        if (!STAR_STORE_OK(pr, a.part_rows, a.err) || !STAR_STORE_OK(pslot, a.maxp, a.err)) continue;
         a.partA[pr * D + d] = Ls > 0.f ? acc / Ls : 0.f;
         if (d == 0) a.partS[pr] = Ls > 0.f ? (base + log2f(Ls)) * kLn2 : -INFINITY;
       }
@@ -952,6 +958,7 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.lse = lse;
   a.partA = s.partA;
   a.partS = s.partS;
+  a.part_rows = s.partS_elems;
   a.tickets = s.tickets;
   a.err = s.err;
   const bool fp8 = c.ctxK8 != nullptr;
@@ -1060,6 +1067,7 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
   c.qV8 = nullptr;
   c.qKs = nullptr;
   c.qVs = nullptr;
+  c.err = nullptr;
 
   const DecodePlan pl = decode_plan(c, q_len, sms);
   const long long rows = (long long)c.B * c.Hkv * pl.maxp * c.G;
@@ -1074,6 +1082,7 @@ extern "C" STAR_API int star_decode_step_noalloc(const star_params* p, long long
     return set_error(STAR_EINVAL, msg);
   }
   Scratch sc;
+  c.err = reinterpret_cast<int*>(base + kNoAllocPartA + kNoAllocPartS + kNoAllocTickets);
   sc.partA = base;
   sc.partS = base + kNoAllocPartA;
   sc.tickets = reinterpret_cast<unsigned*>(base + kNoAllocPartA + kNoAllocPartS);

@@ -32,11 +32,12 @@ template <int D>
 __global__ void __launch_bounds__(256) quantize_qrows_kernel(const bf16* __restrict__ src,
                                                              uint8_t* __restrict__ dst,
                                                              float* __restrict__ scale, int bgs, int lq,
-                                                             int q_cap, int len0) {
+                                                             int q_cap, int len0, int* err) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= (long long)bgs * lq) return;
   const long long bg = row / lq, r = row - bg * lq;
   const long long out = bg * q_cap + len0 + r;
+  if (!STAR_STORE_OK(out, (long long)bgs * q_cap, err)) return;
   quantize_row_warp<D>(src + row * D, dst + out * D, scale + out, threadIdx.x & 31);
 }
 
@@ -61,11 +62,11 @@ cudaError_t launch_quantize_qregion_fp8(const CacheView& c, const bf16* K, const
   const unsigned grid = (unsigned)(((long long)bgs * lq + 7) / 8);
   if (grid == 0) return cudaSuccess;
   if (c.D == 128) {
-    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0);
-    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0);
+    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0, c.err);
+    quantize_qrows_kernel<128><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0, c.err);
   } else {
-    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0);
-    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0);
+    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(K, c.qK8, c.qKs, bgs, lq, c.q_cap, len0, c.err);
+    quantize_qrows_kernel<64><<<grid, 256, 0, st>>>(V, c.qV8, c.qVs, bgs, lq, c.q_cap, len0, c.err);
   }
   return cudaGetLastError();
 }

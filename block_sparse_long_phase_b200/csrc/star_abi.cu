@@ -32,6 +32,12 @@ struct star_cache {
   int4* unit_work;
   cudaStream_t s_in = nullptr, s_out = nullptr, s_comp = nullptr;
   std::vector<cudaEvent_t> events;     // start, end, compute done, then (input ready, output ready) per unit
+  // canary guard regions, one after each part of the allocation
+  struct Guard {
+    size_t off;
+    const char* after;
+  };
+  std::vector<Guard> guards;
 };
 
 namespace {
@@ -54,58 +60,66 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 long long round_up(long long x, long long m) { return (x + m - 1) / m * m; }
 
-constexpr int kTileRows = 64;
+// Canary guard after each part of a cache's allocation.
+constexpr size_t kGuardBytes = 4096;
+constexpr int kCanary = 0xA5;
 
 // ---- phase-2 plans --------------------------------------------------------
-// Prefill chunks: each context segment is cut into equal pieces (multiples of
-// 128 keys) so that (batch x kv head) x (256-row pairs) x chunks is about one
-// CTA per SM; the query region is one more chunk.
-// Context segments [s0, s1) are chunked; the query region is one more chunk
-// when `query` is set.
+// Prefill spans.  The call attends to the context rows [R0, R1) (R0 = s0 * b,
+// R1 = min(s1 * b, L)) and, with the query, to the query region's len0 + lq
+// rows, numbered from L on.  Those rows are cut into m spans of about equal
+// length, boundaries at multiples of 128 rows from R0 (tiles stay full inside
+// a segment), so that (batch x kv head) x (256-row pairs) x m is about one CTA
+// per SM.  A span never holds rows the call does not attend to: when the
+// context part stops short of L and the query region is attended, the region
+// is a span of its own.
 star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0, int s0 = 0, int s1 = -1,
                                bool query = true) {
   const star::CacheView& v = c->view;
   if (s1 < 0) s1 = v.n_seg;
   star::PrefillPlan pl{};
-  const int nseg = s1 - s0;
+  const long long R0 = (long long)s0 * v.b, R1 = std::min((long long)s1 * v.b, v.L);
+  const long long ctx = std::max(0LL, R1 - R0), nq = query ? len0 + lq : 0;
   const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
-  const long long want = std::max(1LL, (long long)c->num_sms / bgp);
-  const long long per_seg = nseg > 0 ? std::max(1LL, (want - (query ? 1 : 0)) / nseg) : 1;
-  long long chunk_len = round_up((v.b + per_seg - 1) / per_seg, 128);
-  for (;;) {
-    int n = 0;
-    for (int s = s0; s < s1; ++s) n += (int)((star::seg_len(v, s) + chunk_len - 1) / chunk_len);
-    if (n + 1 <= star::kMaxPrefillChunks) break;
-    chunk_len *= 2;
-  }
-  int n = 0;
-  for (int s = s0; s < s1; ++s) {
-    const long long len = star::seg_len(v, s);
-    for (long long st = 0; st < len; st += chunk_len) {
-      pl.chunk[n].seg = s;
-      pl.chunk[n].start = (int)st;
-      pl.chunk[n].len = (int)std::min(chunk_len, len - st);
-      ++n;
+  long long m = std::max(1LL, (long long)c->num_sms / bgp);
+  m = std::min<long long>(m, star::kMaxPrefillSpans);
+  auto cut = [&](long long lo, long long n, long long parts) {   // rows [lo, lo + n) into parts spans
+    parts = std::max(1LL, std::min(parts, n / 128));
+    long long prev = 0;
+    for (long long k = 1; k <= parts; ++k) {
+      const long long e = k == parts ? n : (k * n / parts) / 128 * 128;
+      pl.span[pl.n_spans++] = {(int)(lo + prev), (int)(lo + e)};
+      prev = e;
     }
+  };
+  if (ctx > 0 && nq > 0 && R1 < v.L) {
+    cut(R0, ctx, std::max(1LL, m - 1));
+    cut(v.L, nq, 1);
+  } else if (ctx > 0 && nq > 0) {
+    // [R0, L) and the region are contiguous rows: one range
+    const long long n = ctx + nq;
+    long long parts = std::max(1LL, std::min(m, n / 128)), prev = 0;
+    for (long long k = 1; k <= parts; ++k) {
+      const long long e = k == parts ? n : (k * n / parts) / 128 * 128;
+      pl.span[pl.n_spans++] = {(int)(R0 + prev), (int)(R0 + e)};
+      prev = e;
+    }
+  } else if (ctx > 0) {
+    cut(R0, ctx, m);
+  } else if (nq > 0) {
+    cut(v.L, nq, m);
   }
-  if (query) {
-    pl.chunk[n].seg = -1;
-    pl.chunk[n].start = 0;
-    pl.chunk[n].len = (int)(len0 + lq);
-    ++n;
-  }
-  pl.n_chunks = n;
   return pl;
 }
 
-// One chunk per context segment and one for the query region: the partials
+// One span per context segment and one for the query region: the partials
 // are then exactly the per-segment (A_h, s_h) of the method.
 star::PrefillPlan plan_prefill_per_segment(const star_cache* c, int lq, long long len0) {
   const star::CacheView& v = c->view;
   star::PrefillPlan pl{};
-  for (int s = 0; s < v.n_seg; ++s) pl.chunk[s] = {s, 0, (int)star::seg_len(v, s)};
-  pl.chunk[v.n_seg] = {-1, 0, (int)(len0 + lq)};
-  pl.n_chunks = v.n_seg + 1;
+  for (int s = 0; s < v.n_seg; ++s) pl.span[s] = {(int)((long long)s * v.b), (int)((long long)s * v.b + star::seg_len(v, s))};
+  pl.span[v.n_seg] = {(int)v.L, (int)(v.L + len0 + lq)};
+  pl.n_spans = v.n_seg + 1;
   return pl;
 }
 
@@ -130,9 +144,9 @@ int validate_params(const star_params* p) {
   if (p->L + p->q_cap + 1 > 0x7fffffffLL) return fail(STAR_EINVAL, "L + q_cap too large");
   if ((long long)p->B * p->Hkv * (p->L + p->q_cap) >= 0x7fffffffLL)
     return fail(STAR_EUNSUPPORTED, "B * Hkv * (L + q_cap) cached rows must stay below 2^31");
-  if ((p->L + p->block - 1) / p->block > star::kMaxPrefillChunks - 1)
+  if ((p->L + p->block - 1) / p->block > star::kMaxPrefillSpans - 1)
     return fail(STAR_EUNSUPPORTED, "%lld blocks: at most %d", (p->L + p->block - 1) / p->block,
-                star::kMaxPrefillChunks - 1);
+                star::kMaxPrefillSpans - 1);
   return STAR_OK;
 }
 
@@ -206,12 +220,11 @@ int star_cache_create(const star_params* p, star_cache** out) {
   // admits, and the decode plan at the fullest query region.
   long long partA = 0, partS = 0;
   for (int lq = 1; lq <= p->q_cap; ++lq) {
-    // a plan over any range of segments (star_partial_attend) has at most
-    // max(n_seg, CTAs wanted) + 1 chunks; the full plan is one of them
-    star::PrefillPlan pl = plan_prefill(c, lq, 0);
+    // every plan has at most max(n_seg + 1, SMs / (B*Hkv*pairs) + 1) spans
+    // (per segment and region; or the balanced cut plus a region span)
     const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
-    const long long nmax = std::max<long long>(pl.n_chunks, std::max<long long>(v.n_seg, c->num_sms / bgp) + 1);
-    const long long rows = (long long)v.B * v.Hkv * std::min<long long>(nmax, star::kMaxPrefillChunks) * v.G * lq;
+    const long long nmax = std::max<long long>(v.n_seg + 1, std::max(1LL, (long long)c->num_sms / bgp) + 1);
+    const long long rows = (long long)v.B * v.Hkv * std::min<long long>(nmax, star::kMaxPrefillSpans) * v.G * lq;
     partA = std::max(partA, rows * v.D);
     partS = std::max(partS, rows);
   }
@@ -230,24 +243,34 @@ int star_cache_create(const star_params* p, star_cache** out) {
   const long long kv_q = (long long)p->B * p->Hkv * p->q_cap * p->D;
   const long long n_tickets = (long long)p->B * p->Hkv;
   size_t off = 0;
-  auto take = [&](size_t bytes) { size_t o = off; off = (off + bytes + 255) & ~size_t(255); return o; };
-  const size_t o_ck = take(kv_ctx * 2), o_cv = take(kv_ctx * 2);
-  const size_t o_qk = take(kv_q * 2), o_qv = take(kv_q * 2);
-  const size_t o_pa = take(partA * 4), o_ps = take(partS * 4);
-  const size_t o_t = take(n_tickets * 4);
-  const size_t o_e = take(sizeof(int));
-  const size_t o_w = take(work.size() * sizeof(int4));
-  const size_t o_uw = take(unit_work.size() * sizeof(int4));
+  // every part is followed by a canary guard (star_cache_check_guards): a
+  // kernel writing past the end of one part lands in its guard first
+  auto take = [&](size_t bytes, const char* what) {
+    size_t o = off;
+    off = (off + bytes + 255) & ~size_t(255);
+    c->guards.push_back({off, what});
+    off += kGuardBytes;
+    return o;
+  };
+  const size_t o_ck = take(kv_ctx * 2, "context K"), o_cv = take(kv_ctx * 2, "context V");
+  const size_t o_qk = take(kv_q * 2, "query-region K"), o_qv = take(kv_q * 2, "query-region V");
+  const size_t o_pa = take(partA * 4, "partials A"), o_ps = take(partS * 4, "partials s");
+  const size_t o_t = take(n_tickets * 4, "merge tickets");
+  const size_t o_e = take(sizeof(int), "error word");
+  const size_t o_w = take(work.size() * sizeof(int4), "phase-1 work list");
+  const size_t o_uw = take(unit_work.size() * sizeof(int4), "phase-1 units");
   const bool fp8 = p->kv_fp8 != 0;
   const long long ctx_rows = (long long)p->B * p->Hkv * p->L;
-  const size_t o_k8 = fp8 ? take(kv_ctx) : 0, o_v8 = fp8 ? take(kv_ctx) : 0;
+  const size_t o_k8 = fp8 ? take(kv_ctx, "FP8 context K") : 0, o_v8 = fp8 ? take(kv_ctx, "FP8 context V") : 0;
   // scales padded to whole groups of 4 rows (zeroed below): decode loads them 4 rows at a time
   const size_t scl_bytes = (size_t)((ctx_rows + 3) / 4) * 16;
-  const size_t o_ks = fp8 ? take(scl_bytes) : 0, o_vs = fp8 ? take(scl_bytes) : 0;
+  const size_t o_ks = fp8 ? take(scl_bytes, "FP8 context K scales") : 0;
+  const size_t o_vs = fp8 ? take(scl_bytes, "FP8 context V scales") : 0;
   const long long q_rows = (long long)p->B * p->Hkv * p->q_cap;
   const size_t qscl_bytes = (size_t)((q_rows + 3) / 4) * 16;
-  const size_t o_qk8 = fp8 ? take(kv_q) : 0, o_qv8 = fp8 ? take(kv_q) : 0;
-  const size_t o_qks = fp8 ? take(qscl_bytes) : 0, o_qvs = fp8 ? take(qscl_bytes) : 0;
+  const size_t o_qk8 = fp8 ? take(kv_q, "FP8 query-region K") : 0, o_qv8 = fp8 ? take(kv_q, "FP8 query-region V") : 0;
+  const size_t o_qks = fp8 ? take(qscl_bytes, "FP8 query-region K scales") : 0;
+  const size_t o_qvs = fp8 ? take(qscl_bytes, "FP8 query-region V scales") : 0;
   // STAR_FAULT_INJECT=alloc makes this allocation fail (a test hook for the
   // STAR_ENOMEM path)
   const char* inject = getenv("STAR_FAULT_INJECT");
@@ -265,6 +288,7 @@ int star_cache_create(const star_params* p, star_cache** out) {
   c->scratch.partS = reinterpret_cast<float*>(base + o_ps);
   c->scratch.tickets = reinterpret_cast<unsigned*>(base + o_t);
   c->scratch.err = reinterpret_cast<int*>(base + o_e);
+  v.err = c->scratch.err;
   c->scratch.partA_elems = partA;
   c->scratch.partS_elems = partS;
   c->scratch.n_tickets = (int)n_tickets;
@@ -281,6 +305,8 @@ int star_cache_create(const star_params* p, star_cache** out) {
   // Zero everything once: decode streams whole 128-row boxes and masks the
   // rows past the end, which must hold finite values.
   e = cudaMemset(c->block, 0, off);
+  for (size_t g = 0; e == cudaSuccess && g < c->guards.size(); ++g)
+    e = cudaMemset(base + c->guards[g].off, kCanary, kGuardBytes);
   if (e == cudaSuccess) e = cudaMemset(c->scratch.tickets, 0, n_tickets * 4);
   if (e == cudaSuccess) e = cudaMemset(c->scratch.err, 0, sizeof(int));
   if (e == cudaSuccess)
@@ -333,6 +359,23 @@ int star_cache_device_error(star_cache* c, int* flag) {
   if (e == cudaSuccess && h) e = cudaMemset(c->scratch.tickets, 0, (size_t)c->scratch.n_tickets * 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flag = h;
+  return STAR_OK;
+}
+
+int star_cache_check_guards(star_cache* c, int* first_bad) {
+  if (!c || !first_bad) return fail(STAR_EINVAL, "NULL argument");
+  std::vector<unsigned char> h(kGuardBytes);
+  *first_bad = -1;
+  for (size_t g = 0; g < c->guards.size(); ++g) {
+    cudaError_t e = cudaMemcpy(h.data(), static_cast<char*>(c->block) + c->guards[g].off, kGuardBytes,
+                               cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the cache's guard regions");
+    for (size_t i = 0; i < kGuardBytes; ++i)
+      if (h[i] != (unsigned char)kCanary) {
+        *first_bad = (int)g;
+        return fail(STAR_OK, "guard %zu (after %s) overwritten at byte %zu", g, c->guards[g].after, i);
+      }
+  }
   return STAR_OK;
 }
 

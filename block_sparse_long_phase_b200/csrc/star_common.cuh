@@ -12,6 +12,22 @@ namespace star {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Bounds-checked build (nvcc -DSTAR_CHECK_BOUNDS, lib/libstar_checked.so): a
+// kernel checks each global index it computes for a store (and for the cache
+// rows phase 1 copies) against the size of the buffer; a bad index sets the
+// cache's error word to 2 and the access is skipped.  The normal build
+// compiles the checks away.
+STAR_DEVICE bool store_ok(long long idx, long long n, int* err) {
+  if (idx >= 0 && idx < n) return true;
+  if (err) atomicExch(err, 2);
+  return false;
+}
+#ifdef STAR_CHECK_BOUNDS
+#define STAR_STORE_OK(idx, n, err) ::star::store_ok((long long)(idx), (long long)(n), (err))
+#else
+#define STAR_STORE_OK(idx, n, err) true
+#endif
+
 STAR_DEVICE uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -39,6 +39,7 @@ struct CacheView {
   uint8_t* qV8;
   float* qKs;
   float* qVs;
+  int* err;      // the cache's device error word (bounds-checked builds report into it)
 };
 
 __host__ __device__ inline long long seg_len(const CacheView& c, int seg) {
@@ -116,19 +117,23 @@ cudaError_t launch_rope(const RopeJob& j, int D, int B, int groups, cudaStream_t
 // (selftest.cu); synchronous, *gave_up = 1 when it did
 cudaError_t run_wait_timeout(unsigned polls, int* gave_up, cudaStream_t st);
 
-struct PrefillChunk {
-  int seg;     // context segment, or -1 for the query region
-  int start;   // first row inside the segment
-  int len;     // rows
+// Prefill work split: spans [x0, x1) of a (batch, kv head)'s key rows, which
+// are numbered over the context (0..L-1) and then the query region (L..L+n-1,
+// n = rows in use once the call's rows are appended).  One CTA per (span,
+// batch x kv head, 256-row pair of packed query rows); a span may cross
+// context segments (its tiles split at their ends) and run on into the
+// query region.
+struct PrefillSpan {
+  int x0, x1;
 };
-// Chunk table size of a prefill launch (kernel parameter): every context
-// segment takes at least one chunk, so a cache has at most kMaxPrefillChunks - 1
-// segments.
-constexpr int kMaxPrefillChunks = 192;
+// Span table size of a prefill launch (kernel parameter): the per-segment
+// debug plan needs one span per context segment and one for the query
+// region, so a cache has at most kMaxPrefillSpans - 1 segments.
+constexpr int kMaxPrefillSpans = 192;
 
 struct PrefillPlan {
-  int n_chunks;
-  PrefillChunk chunk[kMaxPrefillChunks];
+  int n_spans;
+  PrefillSpan span[kMaxPrefillSpans];
 };
 
 // Decode work split: the cached rows of all (batch, kv head) pairs, laid end

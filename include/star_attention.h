@@ -108,6 +108,15 @@ STAR_API int star_cache_segment_fp8(const star_cache* c, int seg, void** k8, voi
  * call -- outputs of that call are then invalid.  Kernels never trap. */
 STAR_API int star_cache_device_error(star_cache* c, int* flag);
 
+/* Canary check (a stand-in for a memory checker, which this pool does not
+ * run): the cache's one allocation holds, after each of its parts (context
+ * K, context V, query-region K and V, partials, tickets, error word, work
+ * lists, the FP8 copies), a 4 KB guard filled with 0xA5 bytes when the cache
+ * is made.  Synchronous: waits for the device, then *first_bad = -1 if every
+ * guard is intact, else the index of the first overwritten one (in the order
+ * above); star_last_error() then names the part it follows. */
+STAR_API int star_cache_check_guards(star_cache* c, int* first_bad);
+
 /* Number of segments: n context segments followed by the query region. */
 STAR_API int star_cache_num_segments(const star_cache* c);
 

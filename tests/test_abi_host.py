@@ -107,6 +107,7 @@ def test_argument_errors_are_caught_on_the_host(lib):
     assert lib.star_rope(1, 1, 0, 64, 500000.0, None, 0, None, None, None) == _abi.STAR_OK      # nothing to do
     assert lib.star_anchor_keys(None, 0, None, 500000.0, None, None, None) == _abi.STAR_EINVAL
     assert lib.star_ctx_encode_anchored(None, None, None, None, None, None, None, None) == _abi.STAR_EINVAL
+    assert lib.star_cache_check_guards(None, None) == _abi.STAR_EINVAL
     assert lib.star_cache_destroy(None) == _abi.STAR_OK
     assert lib.star_cache_num_segments(None) == 0
 

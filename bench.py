@@ -33,7 +33,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -558,7 +557,8 @@ def run_reference(args):
 
 def profile_case(args):
     """Launches of one kernel for an ncu capture (no bench line): ``phase1``
-    runs star_ctx_encode ``steps`` times, ``decode`` runs phase 1 and the query
+    runs star_ctx_encode ``steps`` times; ``prefill`` runs phase 1 once and the
+    query prefill ``steps`` times; ``decode`` runs phase 1 and the query
     prefill once and then ``steps`` decode steps.  ``--blocks N`` keeps the
     first N blocks of the workload (a capture small enough to replay)."""
     import torch
@@ -576,6 +576,10 @@ def profile_case(args):
     n = args.steps if args.profile == "phase1" else 1
     for _ in range(n):
         cache.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"], O, LSE)
+    if args.profile == "prefill":
+        for _ in range(args.steps):
+            cache.reset_query()
+            cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
     if args.profile == "decode":
         cache.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
         for t in range(args.steps):
@@ -585,6 +589,60 @@ def profile_case(args):
         raise SystemExit("a kernel gave up a bounded wait")
     cache.close()
     print(f"profile case {args.profile}: {w.name} L={w.L} kv_fp8={args.kv_fp8} launches={args.steps}")
+
+
+def measure_e2e(args, w, x, O, LSE, cache, flush, dev, world):
+    """Phase 1 through star_ctx_encode_host with page-locked host Q, K, V in and
+    O, LSE out, copies inside the timed region.  Every rank of a node holds its
+    own host copies; if they would take more than half of the host memory
+    available, the leg runs on the 8B-128K workload instead (named in the
+    result)."""
+    import torch
+    from block_sparse_long_phase_b200 import StarCache, workloads as wl
+    need = sum(t.numel() * t.element_size() for t in (x["Qc"], x["Kc"], x["Vc"], O, LSE))
+    local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    own = None
+    if avail is not None and need * local_world > avail // 2:
+        w = wl.get("8b-128k-needle")
+        x = wl.make_inputs(w, dev, with_decode=False)
+        own = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)
+        cache = own
+        O = torch.empty_like(x["Qc"])
+        LSE = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    h, locked = host_buffers(x, O, LSE)
+    # the device tensors double as the call's staging buffers (same shapes)
+    staging = {"Q": x["Qc"], "K": x["Kc"], "V": x["Vc"], "O": O, "LSE": LSE}
+    stream = torch.cuda.current_stream(dev)
+    e2e_ms = []
+    for it in range(args.warmup + args.steps):
+        flush.flush(4.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cache.star_ctx_encode_host(h["Q"], h["K"], h["V"], h["O"], h["LSE"], staging)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    (e2e_total,) = max_over_ranks([sum(e2e_ms)], dev, world)
+    h2d = sum(h[k].numel() * h[k].element_size() for k in ("Q", "K", "V"))
+    d2h = h["O"].numel() * 2 + h["LSE"].numel() * 4
+    out = {"value": world * w.B * w.L * args.steps / (e2e_total / 1e3), "unit": "ctx tok/s",
+           "ms_per_step": e2e_total / args.steps, "workload": w.name,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "host_memory": "page-locked (cudaHostRegister)" if locked else "pageable (page-locking refused)",
+           "what": "star_ctx_encode_host: host Q,K,V in, O,LSE out, copies overlapped with the "
+                   "encoding block by block, all inside the timed region"}
+    cudart = torch.cuda.cudart()
+    for t in locked:
+        cudart.cudaHostUnregister(t.data_ptr())
+    if own is not None:
+        own.close()
+    return out
 
 
 def host_buffers(x, O, LSE):
@@ -629,7 +687,7 @@ def main():
                     help="skip phase 1 / prefill / decode on the other configurations")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the phase-1 variants (anchor shorter than the block, ragged context, batch 4)")
-    ap.add_argument("--profile", choices=["phase1", "decode"],
+    ap.add_argument("--profile", choices=["phase1", "prefill", "decode"],
                     help="only launch this kernel `steps` times for an ncu capture (no bench line)")
     ap.add_argument("--blocks", type=int, default=0, help="--profile: keep the first N blocks")
     ap.add_argument("--kv-fp8", action="store_true", help="--profile decode: stream the FP8 cache")
@@ -715,32 +773,7 @@ def main():
     e2e = None
     if not args.no_e2e:
         torch.cuda.synchronize(dev)
-        h, locked = host_buffers(x, O, LSE)
-        # the device tensors double as the call's staging buffers (same shapes)
-        staging = {"Q": x["Qc"], "K": x["Kc"], "V": x["Vc"], "O": O, "LSE": LSE}
-        e2e_ms = []
-        for it in range(args.warmup + args.steps):
-            flush.flush(4.0)
-            a, b = ev(), ev()
-            a.record(stream)
-            cache.star_ctx_encode_host(h["Q"], h["K"], h["V"], h["O"], h["LSE"], staging)
-            b.record(stream)
-            torch.cuda.synchronize(dev)
-            if it >= args.warmup:
-                e2e_ms.append(a.elapsed_time(b))
-        (e2e_total,) = max_over_ranks([sum(e2e_ms)], dev, world)
-        h2d = sum(h[k].numel() * h[k].element_size() for k in ("Q", "K", "V"))
-        d2h = h["O"].numel() * 2 + h["LSE"].numel() * 4
-        e2e = {"value": world * w.B * w.L * args.steps / (e2e_total / 1e3), "unit": "ctx tok/s",
-               "ms_per_step": e2e_total / args.steps,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "host_memory": "page-locked (cudaHostRegister)" if locked else "pageable (page-locking refused)",
-               "what": "star_ctx_encode_host: host Q,K,V in, O,LSE out, copies overlapped with the "
-                       "encoding block by block, all inside the timed region"}
-        cudart = torch.cuda.cudart()
-        for t in locked:
-            cudart.cudaHostUnregister(t.data_ptr())
-        del h, locked, staging
+        e2e = measure_e2e(args, w, x, O, LSE, cache, flush, dev, world)
 
     # the main workload's buffers are no longer needed
     cache.close()

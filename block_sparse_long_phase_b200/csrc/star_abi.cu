@@ -366,6 +366,9 @@ int star_cache_check_guards(star_cache* c, int* first_bad) {
   if (!c || !first_bad) return fail(STAR_EINVAL, "NULL argument");
   std::vector<unsigned char> h(kGuardBytes);
   *first_bad = -1;
+  // every stream's work first: a plain copy orders only after the legacy stream
+  cudaError_t es = cudaDeviceSynchronize();
+  if (es != cudaSuccess) return cuda_fail(es, "cudaDeviceSynchronize");
   for (size_t g = 0; g < c->guards.size(); ++g) {
     cudaError_t e = cudaMemcpy(h.data(), static_cast<char*>(c->block) + c->guards[g].off, kGuardBytes,
                                cudaMemcpyDeviceToHost);

@@ -112,7 +112,8 @@ STAR_API int star_cache_device_error(star_cache* c, int* flag);
  * run): the cache's one allocation holds, after each of its parts (context
  * K, context V, query-region K and V, partials, tickets, error word, work
  * lists, the FP8 copies), a 4 KB guard filled with 0xA5 bytes when the cache
- * is made.  Synchronous: waits for the device, then *first_bad = -1 if every
+ * is made.  Synchronous: waits for all work on the device (every stream),
+ * then *first_bad = -1 if every
  * guard is intact, else the index of the first overwritten one (in the order
  * above); star_last_error() then names the part it follows. */
 STAR_API int star_cache_check_guards(star_cache* c, int* first_bad);

@@ -15,7 +15,6 @@ import os
 import subprocess
 import sys
 
-import numpy as np
 import pytest
 import torch
 

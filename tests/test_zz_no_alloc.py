@@ -12,7 +12,6 @@ last so a failure here leaves every other test already run.
 """
 
 import ctypes
-import math
 
 import numpy as np
 import pytest

@@ -50,11 +50,12 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 # ncu captures summarised under profiles/, valid only for the kernel source they
 # were taken on (first 16 hex digits of its sha256); null otherwise.
 TRAFFIC = {
-    "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "", 0),
-    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "1d236e77d71137c2", 1394200320),
-    "decode 8b-32k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 145271552),
-    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 547147264),
-    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "ec260a0065a9bfbf", 290108928),
+    # the 1M launch scaled from captures at L = b and L = 3b (block 0, then two
+    # anchored blocks: each anchored 64K-row block is an L2 group of its own)
+    "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0ea7f91dde1c55f4", 56853444992),
+    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0ea7f91dde1c55f4", 1409251328),
+    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "b36c09b7fa823fac", 543239168),
+    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "b36c09b7fa823fac", 290013696),
 }
 
 

@@ -28,7 +28,7 @@ EXPORTS = (
     "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
     "star_selftest_wait_timeout", "star_noalloc_device_error", "star_ctx_encode_fp32",
     "star_decode_step_partials", "star_partial_attend",
-    "star_lse_merge_bf16", "star_cache_check_guards",
+    "star_lse_merge_bf16", "star_cache_check_guards", "star_plan_prefill", "star_prefill_span_tiles",
 )
 
 
@@ -83,6 +83,9 @@ def load(path: str = LIB_PATH):
     lib.star_noalloc_device_error.argtypes = [ctypes.POINTER(i), vp]
     lib.star_ctx_encode_fp32.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
     lib.star_cache_check_guards.argtypes = [vp, ctypes.POINTER(i)]
+    ip = ctypes.POINTER(i)
+    lib.star_plan_prefill.argtypes = [ctypes.POINTER(StarParams), i, i, ll, i, i, i, i, i, ip, ip]
+    lib.star_prefill_span_tiles.argtypes = [ctypes.POINTER(StarParams), ll, ll, i, i, ip, ip]
     lib.star_lse_merge_bf16.argtypes = [i, ll, i, vp, vp, vp, vp, vp]
     lib.star_partial_attend.argtypes = [vp, i, i, i, i, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step_partials.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(ll), i,

@@ -52,6 +52,7 @@ using namespace sm100;
 
 constexpr int BM = 128;          // query rows per tile
 constexpr int BN = 128;          // keys per K/V tile
+static_assert(BN == kPrefillTileKeys, "the prefill tile walk uses the kernel's tile length");
 constexpr int NBUF = 4;          // K/V ring slots, phase 1
 constexpr int NBUF_PF = 5;       // prefill: its tiles stream from HBM, one more in flight
 constexpr int NTHREADS = 384;
@@ -119,63 +120,6 @@ struct Smem {
   static constexpr int BYTES = RING + NB * TILE;    // + barriers in static smem
 };
 static_assert(Smem<128, NBUF_PF>::BYTES + 1024 <= 227 * 1024, "prefill ring beyond shared memory");
-
-// The 128-key tiles of one prefill span [x, x1) of a (batch, kv head)'s key
-// rows, numbered over the context (0..L-1) and then the query region (L..).
-// A tile never crosses the end of a context segment or of the context; for
-// each one: its first row in the TMA map it is read through (the context
-// cache, or the query region from row L on), its key count, and for the query
-// region the region row of its first key.  The producer and every softmax
-// thread walk the same sequence.
-struct TileWalk {
-  long long x, x1, seg_end;
-  int seg;                                          // -1 once in the query region
-  __device__ __forceinline__ void start(long long x0, long long xe, const CacheView& c) {
-    x = x0;
-    x1 = xe;
-    seg = x0 < c.L ? (int)(x0 / c.b) : -1;
-    seg_end = seg >= 0 ? min((long long)(seg + 1) * c.b, c.L) : xe;
-  }
-  __device__ __forceinline__ int next(const CacheView& c, int bg, int& row, bool& region, int& r0) {
-    if (seg >= 0 && x >= seg_end) {
-      if (x < c.L) {
-        ++seg;
-        seg_end = min((long long)(seg + 1) * c.b, c.L);
-      } else {
-        seg = -1;
-        seg_end = x1;
-      }
-    }
-    const long long end = seg_end < x1 ? seg_end : x1;
-    const int n = (int)(end - x < BN ? end - x : BN);
-    if (seg >= 0) {
-      row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * seg_len(c, seg) + (x - (long long)seg * c.b));
-      region = false;
-      r0 = 0;
-    } else {
-      r0 = (int)(x - c.L);
-      row = (int)((long long)bg * c.q_cap + r0);
-      region = true;
-    }
-    x += n;
-    return n;
-  }
-};
-
-// Tiles of span [x0, x1): one term per segment it overlaps, then the region.
-__device__ __forceinline__ int span_tiles(long long x0, long long x1, const CacheView& c) {
-  int n = 0;
-  long long x = x0;
-  while (x < x1 && x < c.L) {
-    const int seg = (int)(x / c.b);
-    long long e = min((long long)(seg + 1) * c.b, c.L);
-    if (e > x1) e = x1;
-    n += (int)((e - x + BN - 1) / BN);
-    x = e;
-  }
-  if (x < x1) n += (int)((x1 - x + BN - 1) / BN);
-  return n;
-}
 
 template <int D, bool PF>
 __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_constant__ CtxTcArgs a) {

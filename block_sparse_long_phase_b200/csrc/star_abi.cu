@@ -73,15 +73,16 @@ constexpr int kCanary = 0xA5;
 // per SM.  A span never holds rows the call does not attend to: when the
 // context part stops short of L and the query region is attended, the region
 // is a span of its own.
-star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0, int s0 = 0, int s1 = -1,
-                               bool query = true) {
-  const star::CacheView& v = c->view;
+}  // namespace
+
+star::PrefillPlan star::plan_prefill(const star::CacheView& v, int num_sms, int lq, long long len0, int s0, int s1,
+                                     bool query) {
   if (s1 < 0) s1 = v.n_seg;
   star::PrefillPlan pl{};
   const long long R0 = (long long)s0 * v.b, R1 = std::min((long long)s1 * v.b, v.L);
   const long long ctx = std::max(0LL, R1 - R0), nq = query ? len0 + lq : 0;
   const long long bgp = (long long)v.B * v.Hkv * star::prefill_row_pairs(v, lq);
-  long long m = std::max(1LL, (long long)c->num_sms / bgp);
+  long long m = std::max(1LL, (long long)num_sms / bgp);
   m = std::min<long long>(m, star::kMaxPrefillSpans);
   auto cut = [&](long long lo, long long n, long long parts) {   // rows [lo, lo + n) into parts spans
     parts = std::max(1LL, std::min(parts, n / 128));
@@ -114,14 +115,15 @@ star::PrefillPlan plan_prefill(const star_cache* c, int lq, long long len0, int 
 
 // One span per context segment and one for the query region: the partials
 // are then exactly the per-segment (A_h, s_h) of the method.
-star::PrefillPlan plan_prefill_per_segment(const star_cache* c, int lq, long long len0) {
-  const star::CacheView& v = c->view;
+star::PrefillPlan star::plan_prefill_per_segment(const star::CacheView& v, int lq, long long len0) {
   star::PrefillPlan pl{};
   for (int s = 0; s < v.n_seg; ++s) pl.span[s] = {(int)((long long)s * v.b), (int)((long long)s * v.b + star::seg_len(v, s))};
   pl.span[v.n_seg] = {(int)v.L, (int)(v.L + len0 + lq)};
   pl.n_spans = v.n_seg + 1;
   return pl;
 }
+
+namespace {
 
 star::DecodePlan plan_decode(const star_cache* c, long long len0) {
   star::DecodePlan pl;
@@ -150,6 +152,16 @@ int validate_params(const star_params* p) {
   return STAR_OK;
 }
 
+// The cache geometry of `p` without device memory (host-side planning only).
+star::CacheView host_view(const star_params* p) {
+  star::CacheView v{};
+  v.B = p->B; v.Hq = p->Hq; v.Hkv = p->Hkv; v.D = p->D; v.G = p->Hq / p->Hkv;
+  v.L = p->L; v.b = p->block; v.b_a = p->anchor;
+  v.n_seg = (int)((p->L + p->block - 1) / p->block);
+  v.q_cap = p->q_cap;
+  return v;
+}
+
 }  // namespace
 
 namespace star {
@@ -173,7 +185,8 @@ int query_prefill(star_cache* c, int lq, const void* Q, const void* K, const voi
   if (c->q_len + lq > c->view.q_cap)
     return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, c->view.q_cap);
   const star::PrefillPlan pl =
-      per_segment ? plan_prefill_per_segment(c, lq, c->q_len) : plan_prefill(c, lq, c->q_len);
+      per_segment ? star::plan_prefill_per_segment(c->view, lq, c->q_len)
+                  : star::plan_prefill(c->view, c->num_sms, lq, c->q_len);
   cudaError_t e = star::launch_query_prefill_tc(
       c->view, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q),
       static_cast<const bf16*>(K), static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, pl,
@@ -666,7 +679,8 @@ int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query,
   if (with_query && c->q_len + lq > w.q_cap)
     return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, w.q_cap);
   if (lq > w.q_cap) return fail(STAR_EINVAL, "lq %d beyond q_cap %d (the scratch is sized by it)", lq, w.q_cap);
-  const star::PrefillPlan pl = plan_prefill(c, lq, c->q_len, first_seg, first_seg + n_seg, with_query != 0);
+  const star::PrefillPlan pl =
+      star::plan_prefill(w, c->num_sms, lq, c->q_len, first_seg, first_seg + n_seg, with_query != 0);
   cudaError_t e = star::launch_query_prefill_tc(
       w, c->dmaps, c->p.scale, lq, (int)c->q_len, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
       static_cast<const bf16*>(V), nullptr, s, pl, c->scratch, static_cast<cudaStream_t>(stream), A, nullptr,
@@ -716,6 +730,52 @@ int star_decode_step_partials(star_cache* c, const void* q, const void* k, const
     spans[3 * p + 1] = parts[p].first;
     spans[3 * p + 2] = parts[p].end;
   }
+  return STAR_OK;
+}
+
+int star_plan_prefill(const star_params* p, int num_sms, int lq, long long len0, int first_seg, int n_seg,
+                      int with_query, int per_segment, int max_spans, int* n_spans, int* spans) {
+  int rc = validate_params(p);
+  if (rc) return rc;
+  if (!n_spans || !spans) return fail(STAR_EINVAL, "NULL output pointer");
+  if (num_sms < 1 || lq < 1 || len0 < 0 || len0 + lq > p->q_cap) return fail(STAR_EINVAL, "bad num_sms, lq or len0");
+  const star::CacheView v = host_view(p);
+  if (first_seg < 0 || n_seg < 0 || first_seg + n_seg > v.n_seg) return fail(STAR_EINVAL, "segment range");
+  const star::PrefillPlan pl = per_segment ? star::plan_prefill_per_segment(v, lq, len0)
+                                           : star::plan_prefill(v, num_sms, lq, len0, first_seg, first_seg + n_seg,
+                                                                with_query != 0);
+  *n_spans = pl.n_spans;
+  if (pl.n_spans > max_spans) return fail(STAR_EINVAL, "%d spans do not fit max_spans = %d", pl.n_spans, max_spans);
+  for (int k = 0; k < pl.n_spans; ++k) {
+    spans[2 * k] = pl.span[k].x0;
+    spans[2 * k + 1] = pl.span[k].x1;
+  }
+  return STAR_OK;
+}
+
+int star_prefill_span_tiles(const star_params* p, long long x0, long long x1, int bg, int max_tiles, int* n_tiles,
+                            int* tiles) {
+  int rc = validate_params(p);
+  if (rc) return rc;
+  if (!n_tiles || !tiles) return fail(STAR_EINVAL, "NULL output pointer");
+  const star::CacheView v = host_view(p);
+  if (x0 < 0 || x1 <= x0 || x1 > v.L + v.q_cap || bg < 0 || bg >= v.B * v.Hkv)
+    return fail(STAR_EINVAL, "span or (batch, kv head) out of range");
+  const int n = star::span_tiles(x0, x1, v);
+  *n_tiles = n;
+  if (n > max_tiles) return fail(STAR_EINVAL, "%d tiles do not fit max_tiles = %d", n, max_tiles);
+  star::TileWalk walk;
+  walk.start(x0, x1, v);
+  for (int t = 0; t < n; ++t) {
+    int row, r0;
+    bool region;
+    const int k = walk.next(v, bg, row, region, r0);
+    tiles[4 * t] = row;
+    tiles[4 * t + 1] = region ? 1 : 0;
+    tiles[4 * t + 2] = k;
+    tiles[4 * t + 3] = r0;
+  }
+  if (walk.x != x1) return fail(STAR_EINVAL, "the walk did not end at the span's end");
   return STAR_OK;
 }
 

@@ -136,6 +136,67 @@ struct PrefillPlan {
   PrefillSpan span[kMaxPrefillSpans];
 };
 
+// Keys per prefill tile (the tile kernel's BN).
+constexpr int kPrefillTileKeys = 128;
+
+// The 128-key tiles of one prefill span [x, x1) of a (batch, kv head)'s key
+// rows, numbered over the context (0..L-1) and then the query region (L..).
+// A tile never crosses the end of a context segment or of the context; for
+// each one: its first row in the TMA map it is read through (the context
+// cache, or the query region from row L on), its key count, and for the query
+// region the region row of its first key.  The producer and every softmax
+// thread walk the same sequence.
+struct TileWalk {
+  long long x, x1, seg_end;
+  int seg;                                          // -1 once in the query region
+  __host__ __device__ __forceinline__ void start(long long x0, long long xe, const CacheView& c) {
+    x = x0;
+    x1 = xe;
+    seg = x0 < c.L ? (int)(x0 / c.b) : -1;
+    seg_end = seg >= 0 ? ((long long)(seg + 1) * c.b < c.L ? (long long)(seg + 1) * c.b : c.L) : xe;
+  }
+  __host__ __device__ __forceinline__ int next(const CacheView& c, int bg, int& row, bool& region, int& r0) {
+    if (seg >= 0 && x >= seg_end) {
+      if (x < c.L) {
+        ++seg;
+        seg_end = ((long long)(seg + 1) * c.b < c.L ? (long long)(seg + 1) * c.b : c.L);
+      } else {
+        seg = -1;
+        seg_end = x1;
+      }
+    }
+    const long long end = seg_end < x1 ? seg_end : x1;
+    const int n = (int)(end - x < kPrefillTileKeys ? end - x : kPrefillTileKeys);
+    if (seg >= 0) {
+      row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * seg_len(c, seg) + (x - (long long)seg * c.b));
+      region = false;
+      r0 = 0;
+    } else {
+      r0 = (int)(x - c.L);
+      row = (int)((long long)bg * c.q_cap + r0);
+      region = true;
+    }
+    x += n;
+    return n;
+  }
+};
+
+// Tiles of span [x0, x1): one term per segment it overlaps, then the region.
+__host__ __device__ __forceinline__ int span_tiles(long long x0, long long x1, const CacheView& c) {
+  int n = 0;
+  long long x = x0;
+  while (x < x1 && x < c.L) {
+    const int seg = (int)(x / c.b);
+    long long e = (long long)(seg + 1) * c.b < c.L ? (long long)(seg + 1) * c.b : c.L;
+    if (e > x1) e = x1;
+    n += (int)((e - x + kPrefillTileKeys - 1) / kPrefillTileKeys);
+    x = e;
+  }
+  if (x < x1) n += (int)((x1 - x + kPrefillTileKeys - 1) / kPrefillTileKeys);
+  return n;
+}
+
+
 // Decode work split: the cached rows of all (batch, kv head) pairs, laid end
 // to end, are cut into one balanced span per CTA; each span leaves one part
 // per (batch, kv head) it touches, and the new token one more.
@@ -171,6 +232,13 @@ struct DecodePart {
   long long first, end;
 };
 void decode_parts(const CacheView& c, long long len0, const DecodePlan& pl, std::vector<DecodePart>& out);
+
+// Prefill plans (star_abi.cu): spans of about equal length over the context
+// segments [s0, s1) and, with `query`, the query region's len0 + lq rows; or
+// one span per segment and one for the region.
+PrefillPlan plan_prefill(const CacheView& v, int num_sms, int lq, long long len0, int s0 = 0, int s1 = -1,
+                         bool query = true);
+PrefillPlan plan_prefill_per_segment(const CacheView& v, int lq, long long len0);
 
 // TMA maps of the cache, built once per cache.
 struct DecodeMaps {

@@ -290,6 +290,29 @@ STAR_API int star_lse_merge(int P, long long R, int D, const float* A, const flo
 STAR_API int star_lse_merge_bf16(int P, long long R, int D, const float* A, const float* s,
                                  void* out_O, float* out_s, void* stream);
 
+/* Host-only introspection of the query prefill's work split (no device is
+ * touched; for tests and capacity planning).  The prefill cuts the key rows of
+ * each (batch, kv head) -- context tokens 0..L-1, then query-region rows from
+ * L on -- into spans, one CTA per (span, batch x kv head, 256-row pair of
+ * packed query rows):
+ *   star_plan_prefill: the spans a call with `lq` query rows on a region of
+ *     len0 rows would use on a GPU of `num_sms` SMs -- context segments
+ *     [first_seg, first_seg + n_seg) and, with with_query, the region (as
+ *     star_partial_attend; star_query_prefill is the full range with the
+ *     region), or with per_segment the debug form's one span per segment and
+ *     one for the region.  spans[2k], spans[2k+1] = [x0, x1) of span k;
+ *     *n_spans = their count (STAR_EINVAL if it exceeds max_spans).
+ *   star_prefill_span_tiles: the 128-key tiles of span [x0, x1) of (batch x
+ *     kv head) bg: tiles[4t..4t+3] = (first row in the TMA map read, 1 if
+ *     that map is the query region's, keys in the tile, the region row of its
+ *     first key); tiles never cross a context segment's end.
+ * Arguments as star_cache_create's params otherwise. */
+STAR_API int star_plan_prefill(const star_params* p, int num_sms, int lq, long long len0, int first_seg,
+                               int n_seg, int with_query, int per_segment, int max_spans, int* n_spans,
+                               int* spans);
+STAR_API int star_prefill_span_tiles(const star_params* p, long long x0, long long x1, int bg, int max_tiles,
+                                     int* n_tiles, int* tiles);
+
 /* Self-test of the failure path every pipelined kernel here uses: one CTA
  * waits, with the kernels' bounded mbarrier wait limited to `polls` polls
  * (1..2^22; the kernels use 2^22), on a barrier nothing completes, so the

@@ -203,7 +203,7 @@ int query_prefill(star_cache* c, int lq, const void* Q, const void* K, const voi
 extern "C" {
 
 const char* star_last_error(void) { return g_err; }
-const char* star_version(void) { return "libstar 0.1 (sm_100a)"; }
+const char* star_version(void) { return "libstar 0.2 (sm_100a)"; }
 
 int star_cache_create(const star_params* p, star_cache** out) {
   if (!out) return fail(STAR_EINVAL, "out is NULL");

@@ -80,6 +80,7 @@ struct CtxTcArgs {
   float* partA;
   float* partS;
   long long part_rows;   // rows the scratch holds (partS elements)
+  int wait_first;        // prefill without the append kernel: wait for the previous kernel before any load
   PrefillPlan plan;
 };
 static_assert(sizeof(CtxTcArgs) <= 4096, "kernel parameters beyond 4 KB");
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (PF) griddep_launch();
   const uint32_t tmem = tmem_base_s;
   auto fail = [&]() {
     abort_s = 1;
@@ -222,9 +224,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         }
       }
       int pf_row = 0;
-      bool pf_region = false;
+      bool pf_region = false, region_ready = false;
       const bool own_anchor = !PF && a.anchor_keys && blk > 0;   // per-block anchor keys
       if (own_anchor) prefetch_tmap(&a.tkq);
+      if (PF && a.wait_first) {
+        griddep_wait();                                 // inputs written by the kernel before this one
+        region_ready = true;
+      }
       const uint32_t qb = smem_u32(&bar_q_full);
       mbar_arrive_expect_tx(qb, nq * S::TILE);
       for (int q = 0; q < nq; ++q) {
@@ -248,7 +254,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
             walk.next(c, bg, pf_row, pf_region, r0u);
           }
           row = pf_row;
-          if (pf_region) m = (i & 1) ? &a.tvq : &a.tkq;
+          if (pf_region) {
+            m = (i & 1) ? &a.tvq : &a.tkq;
+            if (!region_ready) {
+              griddep_wait();                           // the append kernel's rows are written
+              region_ready = true;
+            }
+          }
         }
         if (own_anchor && !(i & 1) && j < n_anchor) {
           // K of block blk's anchor: rows of Ka[blk - 1] for this (batch, kv head)
@@ -662,6 +674,7 @@ namespace {
 __global__ void __launch_bounds__(256) query_append_kernel(CacheView c, int lq, int len0,
                                                            const uint4* __restrict__ K,
                                                            const uint4* __restrict__ V) {
+  griddep_launch();                                           // the tile kernel waits for these rows itself
   const int cpr = c.D / 8;                                    // 16-byte chunks per row
   const long long n = (long long)c.B * c.Hkv * lq * cpr;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -697,6 +710,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) prefill_merge_kernel(CacheVi
                                                                         float* __restrict__ Ah,
                                                                         float* __restrict__ sh) {
   __shared__ float wgt[kMergeWarps][kSPerLane * 32];
+  griddep_wait();                                    // the tile kernel's partials are complete
   const int rows_total = c.G * lq;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long gw = (long long)blockIdx.x * kMergeWarps + wid;
@@ -799,25 +813,44 @@ cudaError_t launch_query_prefill_tc(const CacheView& c, const DecodeMaps& maps, 
   a.partS = s.partS;
   a.part_rows = s.partS_elems;
   a.plan = plan;
+  a.wait_first = append ? 0 : 1;
   if (append) {
     const long long n16 = (long long)c.B * c.Hkv * lq * (c.D / 8);
     const int agrid = (int)((n16 + 255) / 256 < 1024 ? (n16 + 255) / 256 : 1024);
     query_append_kernel<<<agrid, 256, 0, st>>>(c, lq, len0, reinterpret_cast<const uint4*>(Kq),
                                                reinterpret_cast<const uint4*>(Vq));
   }
+  // The tile kernel and the merge are launched as programmatic dependents of
+  // the kernel before them: each starts while that one drains and waits for
+  // its results where it reads them (griddep_wait).
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
   const int grid = c.B * c.Hkv * a.row_pairs * plan.n_spans;
   if (grid > 0) {
-    if (c.D == 128)
-      attn_tc_kernel<128, true><<<grid, NTHREADS, smem_bytes<128, true>(), st>>>(a);
-    else
-      attn_tc_kernel<64, true><<<grid, NTHREADS, smem_bytes<64, true>(), st>>>(a);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = c.D == 128 ? smem_bytes<128, true>() : smem_bytes<64, true>();
+    e = c.D == 128 ? cudaLaunchKernelEx(&cfg, attn_tc_kernel<128, true>, a)
+                   : cudaLaunchKernelEx(&cfg, attn_tc_kernel<64, true>, a);
+    if (e != cudaSuccess) return e;
   }
   const long long rows = (long long)c.B * c.Hkv * c.G * lq;
-  const int mgrid = (int)((rows + kMergeWarps - 1) / kMergeWarps);
-  if (c.D == 128)
-    prefill_merge_kernel<128><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_spans, s.partS_elems, s.partA, s.partS, O, LSE, O32, Ah, sh);
-  else
-    prefill_merge_kernel<64><<<mgrid, 32 * kMergeWarps, 0, st>>>(c, lq, plan.n_spans, s.partS_elems, s.partA, s.partS, O, LSE, O32, Ah, sh);
+  cfg.gridDim = dim3((unsigned)((rows + kMergeWarps - 1) / kMergeWarps));
+  cfg.blockDim = dim3(32 * kMergeWarps);
+  cfg.dynamicSmemBytes = 0;
+  const int n_spans = plan.n_spans;
+  const long long part_rows = s.partS_elems;
+  const float* pA = s.partA;
+  const float* pS = s.partS;
+  e = c.D == 128 ? cudaLaunchKernelEx(&cfg, prefill_merge_kernel<128>, c, lq, n_spans, part_rows, pA, pS, O, LSE, O32, Ah, sh)
+                 : cudaLaunchKernelEx(&cfg, prefill_merge_kernel<64>, c, lq, n_spans, part_rows, pA, pS, O, LSE, O32, Ah, sh);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -70,6 +70,15 @@ SM100_DEV bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = kWaitLi
   return false;
 }
 
+// ---- programmatic dependent launch ---------------------------------------------
+// A kernel launched with programmatic stream serialisation may start before the
+// kernel ahead of it in the stream has finished; griddep_wait blocks the
+// calling thread until that kernel has completed and its writes are visible
+// (a no-op for a kernel launched without the attribute).  griddep_launch lets
+// the next such kernel be scheduled once every CTA of this grid has issued it.
+SM100_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+SM100_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- TMA ------------------------------------------------------------------------
 SM100_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");

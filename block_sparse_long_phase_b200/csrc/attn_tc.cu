@@ -56,6 +56,17 @@ static_assert(BN == kPrefillTileKeys, "the prefill tile walk uses the kernel's t
 constexpr int NBUF = 4;          // K/V ring slots, phase 1
 constexpr int NBUF_PF = 5;       // prefill: its tiles stream from HBM, one more in flight
 constexpr int NTHREADS = 384;
+// Register split between the warpgroups (setmaxnreg): warpgroup 0 (producer,
+// MMA issuer, cache copy) drops to kRegsWG0 per thread and the two softmax
+// warpgroups rise to kRegsSoftmax.  The pool is what the CTA was launched
+// with (NTHREADS x the kernel's register count, 168 under these launch
+// bounds): attn_tc_prepare refuses a build whose count is below kRegsPool,
+// since an increase the pool cannot grant would never return.
+constexpr int kRegsWG0 = 120;
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsPool = 4 * 32 * kRegsWG0 + 8 * 32 * kRegsSoftmax;
+static_assert(kRegsPool == NTHREADS * 168, "register split must add up to the launch's registers");
+static_assert(kRegsWG0 % 8 == 0 && kRegsSoftmax % 8 == 0, "setmaxnreg takes multiples of 8");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct CtxTcArgs {
@@ -207,6 +218,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
     atomicExch(a.err, 1);
   };
 
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegsWG0));
   if (warp == 0) {
     // ------------------------------ TMA producer -----------------------------
     if (elect_one()) {
@@ -358,7 +371,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
         *reinterpret_cast<uint4*>(c.ctxV + sbase + (long long)r * D + ch * 8) = vv;
       }
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegsSoftmax));
     // ------------------------------ softmax ----------------------------------
     const int q = (warp - 4) >> 2;                    // head 0 or 1 of the pair
     if (q < nq) {
@@ -617,8 +632,18 @@ constexpr int smem_bytes() {
   return Smem<D, PF ? NBUF_PF : NBUF>::BYTES + 1024;
 }
 
+template <int D, bool PF>
+cudaError_t check_reg_pool() {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<D, PF>);
+  if (e != cudaSuccess) return e;
+  return fa.numRegs * NTHREADS >= kRegsPool ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 cudaError_t attn_tc_prepare(int D) {
-  cudaError_t e;
+  cudaError_t e = D == 128 ? check_reg_pool<128, false>() : check_reg_pool<64, false>();
+  if (e == cudaSuccess) e = D == 128 ? check_reg_pool<128, true>() : check_reg_pool<64, true>();
+  if (e != cudaSuccess) return e;
   if (D == 128) {
     e = cudaFuncSetAttribute(attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes<128, false>());

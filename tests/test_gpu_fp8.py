@@ -172,7 +172,7 @@ def test_fp8_zero_rows_and_wide_range():
     cache.close()
 
 
-@pytest.mark.parametrize("name", ["8b-128k-needle", "70b-128k-b4"])
+@pytest.mark.parametrize("name", ["8b-128k-needle", "70b-128k-b4", "8b-1m"])
 def test_fp8_full_size_sampled(name):
     """Full-size workload in the launch configuration the benchmark times:
     sampled FP8 rows bit-exact, sampled decode steps of two kv groups (first

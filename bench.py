@@ -338,6 +338,89 @@ def measure_long_decode(dev, flush, warmup, steps, world, kv_fp8=False, name="8b
     return w, t_ms * 1e3
 
 
+def measure_sharded(dev, flush, w, ranks=8, steps=8):
+    """The block-sharded layer's per-rank work on one GPU, its ranks run one
+    after another: each rank's phase 1 on its local [anchor | zeros | own
+    blocks] context (input assembly included), its phase-2 partial of the query
+    rows and of ``steps`` decode tokens (star_partial_attend), each timed alone
+    after an L2 flush, and the merge of the gathered partials.  The all_gather
+    between ranks is not run (one GPU); its bytes are reported."""
+    import torch
+    from block_sparse_long_phase_b200 import workloads as wl
+    from block_sparse_long_phase_b200.api import star_lse_merge_bf16
+    from block_sparse_long_phase_b200.sharded import ShardedStarCache
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n = -(-w.L // w.b)
+    R = max(1, min(ranks, n))
+    T = min(w.T, steps + 1)
+    x = wl.make_inputs(w, dev)
+    Ka, Va = x["Kc"][:, :, :w.b_a].contiguous(), x["Vc"][:, :, :w.b_a].contiguous()
+    enc, pre, dec, dec_bytes = [], [], [], []
+    parts = []
+    for r in range(R):
+        sc = ShardedStarCache(r, R, w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale, device=dev)
+        lay = sc.layout
+        r0, r1 = lay.rows0, lay.rows0 + lay.rows
+        own = [x[k][:, :, r0:r1].contiguous() for k in ("Qc", "Kc", "Vc")]
+        flush.flush(11.0)
+        a, b = ev(), ev()
+        a.record(stream)
+        sc.encode(*own, Ka, Va)
+        b.record(stream)
+        del own
+        qkv = (x["Qq"], x["Kq"], x["Vq"]) if sc.is_query_rank else (x["Qq"],)
+        flush.flush(12.0)
+        c, d = ev(), ev()
+        c.record(stream)
+        sc.local_partial(*qkv)
+        d.record(stream)
+        steps_ev = []
+        for t in range(T):
+            qkv = (x["qd"][t], x["kd"][t], x["vd"][t]) if sc.is_query_rank else (x["qd"][t],)
+            flush.flush(13.0)
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            A, s_ = sc.local_partial(*qkv)
+            e1.record(stream)
+            steps_ev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        assert sc.cache.device_error() == 0, "a kernel gave up a bounded pipeline wait"
+        enc.append(a.elapsed_time(b))
+        pre.append(c.elapsed_time(d))
+        dec.append(sum(e0.elapsed_time(e1) for e0, e1 in steps_ev[1:]) / max(1, len(steps_ev) - 1) * 1e3)
+        rows = lay.rows + ((w.lq + T) if sc.is_query_rank else 0)
+        dec_bytes.append(w.B * w.Hkv * rows * w.D * 2 * 2)
+        parts.append((A, s_))
+        sc.close()
+    A = torch.stack([p_[0] for p_ in parts]).reshape(R, w.B * w.Hq, w.D).contiguous()
+    S = torch.stack([p_[1] for p_ in parts]).reshape(R, w.B * w.Hq).contiguous()
+    m = []
+    for _ in range(5):
+        flush.flush(14.0)
+        a, b = ev(), ev()
+        a.record(stream)
+        star_lse_merge_bf16(A, S)
+        b.record(stream)
+        m.append((a, b))
+    torch.cuda.synchronize(dev)
+    merge_us = sum(a.elapsed_time(b) for a, b in m[1:]) / (len(m) - 1) * 1e3
+    del x, Ka, Va, parts, A, S
+    torch.cuda.empty_cache()
+    pk = peaks()
+    gbs = [by / (us * 1e-6) / 1e9 for by, us in zip(dec_bytes, dec)]
+    return {
+        "workload": w.name, "ranks": R, "how": "ranks run one after another on one GPU; the all_gather "
+        "of the partials between them is not run",
+        "phase1_ms_per_rank": enc, "phase1_ms_max": max(enc),
+        "ctx_tok_s_if_ranks_run_at_once": w.B * w.L / (max(enc) / 1e3),
+        "prefill_partial_ms_per_rank": pre,
+        "decode_partial_us_per_rank": dec, "decode_partial_us_max": max(dec),
+        "decode_partial_frac_per_rank": [g / pk["hbm_gbs"] for g in gbs],
+        "merge_us": merge_us,
+        "gather_bytes_per_rank_per_step": w.B * w.Hq * (w.D + 1) * 4}
+
+
 CONFIGS = ["tiny", "8b-32k", "8b-128k-needle", "70b-128k", "70b-128k-b4"]
 DATASHEET_HBM_GBS = 7700.0   # B200 HBM3e, HGX figure: context for the decode fractions
 
@@ -688,6 +771,8 @@ def main():
                     help="skip phase 1 / prefill / decode on the other configurations")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the phase-1 variants (anchor shorter than the block, ragged context, batch 4)")
+    ap.add_argument("--no-sharded", action="store_true",
+                    help="skip the block-sharded layer's per-rank kernels (ranks emulated on one GPU)")
     ap.add_argument("--profile", choices=["phase1", "prefill", "decode"],
                     help="only launch this kernel `steps` times for an ncu capture (no bench line)")
     ap.add_argument("--blocks", type=int, default=0, help="--profile: keep the first N blocks")
@@ -800,6 +885,10 @@ def main():
             settle()
             long_dec_fp8_main = measure_long_decode(dev, flush, args.warmup, args.steps, world, kv_fp8=True,
                                                     name=w.name)
+    sharded = None
+    if not args.no_sharded and world == 1:
+        settle()
+        sharded = measure_sharded(dev, flush, w)
     rope = variants = None
     if not args.no_variants:
         settle()
@@ -859,6 +948,8 @@ def main():
         line["rope"] = rope
     if configs:
         line["configs"] = configs
+    if sharded:
+        line["sharded_emulated"] = sharded
     if variants:
         for v in variants.values():
             # burst peak for a launch of a few ms; a launch of 10+ ms runs under

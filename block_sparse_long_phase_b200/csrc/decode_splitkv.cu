@@ -72,11 +72,14 @@ struct DecodeArgs {
   int len0;                     // query-region rows before this step
   int ncta;
   int maxp;                     // partial slots per (batch, kv head)
-  long long rpb;                // cached rows per (batch, kv head): L + len0
+  long long rpb;                // rows attended per (batch, kv head): L - skip + len0
+  long long skip = 0;           // leading context rows of each (batch, kv head) left out
+  int with_token = 1;           // append the step's k, v and fold its own score in
   const bf16* q;                // [B][Hq][D]
-  const bf16* k;                // [B][Hkv][D]
+  const bf16* k;                // [B][Hkv][D] (unused without the token)
   const bf16* v;
-  bf16* o;                      // [B][Hq][D]
+  bf16* o;                      // [B][Hq][D] (null: not written)
+  float* o32 = nullptr;         // [B][Hq][D] float32 rows (null: not written)
   float* lse;                   // [B][Hq]
   float* partA;                 // [B*Hkv][maxp][G][D]
   float* partS;                 // [B*Hkv][maxp][G]
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         bool ctx = false;
         if (have) {
           bg = (int)((unsigned)x / (unsigned)a.rpb);
-          const long long off = x - (long long)bg * a.rpb;         // key index within bg
+          const long long off = x - (long long)bg * a.rpb + a.skip;   // key index within bg
           const long long run_end = ((long long)bg + 1) * a.rpb < x1 ? ((long long)bg + 1) * a.rpb : x1;
           long long region_end;
           if (off < c.L) {
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
             row = (int)((long long)seg * c.B * c.Hkv * c.b + (long long)bg * len + (off - (long long)seg * c.b));
             ctx = true;
           } else {
-            region_end = a.rpb;
+            region_end = a.rpb + a.skip;
             row = (int)((long long)bg * c.q_cap + (off - c.L));
           }
           n = FP8 ? KS8 : KS;
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     // this launch touches) and its FP8 copy for the steps after this one,
     // written by the whole warp once its last stage is issued: off the path
     // the step's time depends on.
-    if (!aborted()) {
+    if (!aborted() && a.with_token) {
       for (int bg = blockIdx.x; bg < c.B * c.Hkv; bg += a.ncta) {
         const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
         const long long qo = q_row_offset(c, bb, g, a.len0);
@@ -598,8 +601,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
     const long long R = (long long)c.B * c.Hkv * a.rpb;
     const int nspan = cta_of((long long)bg * a.rpb + a.rpb - 1, R, a.ncta) - cta_of((long long)bg * a.rpb, R, a.ncta) + 1;
     const int cnt = nspan;
-    const bf16* kn = a.k + (long long)bg * D;
-    const bf16* vn = a.v + (long long)bg * D;
+    const bool tok = a.with_token != 0;
+    const bf16* kn = tok ? a.k + (long long)bg * D : nullptr;
+    const bf16* vn = tok ? a.v + (long long)bg * D : nullptr;
     constexpr int NT = 32 * NCW;
     constexpr int KMAX = 11;
     const int nout = G * (D / 4);
@@ -619,7 +623,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       // the new token: this thread's 4 elements of q_r . k, and of v
       uint2 q2 = make_uint2(0u, 0u), k2 = make_uint2(0u, 0u), v2 = make_uint2(0u, 0u);
-      if (active) {
+      if (active && tok) {
         q2 = *reinterpret_cast<const uint2*>(a.q + ((long long)bb * c.Hq + (long long)g * G + r) * D + 4 * d4);
         k2 = *reinterpret_cast<const uint2*>(kn + 4 * d4);
         v2 = *reinterpret_cast<const uint2*>(vn + 4 * d4);
@@ -664,7 +668,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
                  __uint_as_float(q2.y & 0xffff0000u) * __uint_as_float(k2.y & 0xffff0000u);
 #pragma unroll
       for (int off = D / 8; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
-      if (active && pg == 0) {
+      if (active && pg == 0 && tok) {
         const float sn = qk * a.scale_log2 * kLn2;  // natural-log units, like s_h
         const float Mn = fmaxf(M, sn);
         const float al = M == -INFINITY ? 0.f : __expf(M - Mn);
@@ -701,10 +705,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
         const long long orow = (long long)bb * c.Hq + (long long)g * G + r;
         // (no early exit here: every consumer thread must reach the barrier below)
         if (STAR_STORE_OK(orow, (long long)c.B * c.Hq, a.err)) {
-          uint2 pk;
-          pk.x = pack_bf16(at.x * inv, at.y * inv);
-          pk.y = pack_bf16(at.z * inv, at.w * inv);
-          *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+          if (a.o) {
+            uint2 pk;
+            pk.x = pack_bf16(at.x * inv, at.y * inv);
+            pk.y = pack_bf16(at.z * inv, at.w * inv);
+            *reinterpret_cast<uint2*>(a.o + orow * D + 4 * d4) = pk;
+          }
+          if (a.o32)
+            *reinterpret_cast<float4*>(a.o32 + orow * D + 4 * d4) =
+                make_float4(at.x * inv, at.y * inv, at.z * inv, at.w * inv);
           if (d4 == 0) a.lse[orow] = Lt > 0.f ? Mt + __logf(Lt) : -INFINITY;
         }
       }
@@ -798,7 +807,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const __grid_consta
       const int bg0 = (int)((unsigned)x0 / (unsigned)a.rpb), bg1 = (int)((unsigned)(x1 - 1) / (unsigned)a.rpb);
       constexpr int kLine = 128;                       // bytes per L2 prefetch
       const int q_lines = G * D * 2 / kLine, kv_lines = D * 2 / kLine;
-      const int per_bg = q_lines + 2 * kv_lines;
+      const int per_bg = q_lines + (a.with_token ? 2 * kv_lines : 0);
       for (int i = ctid; i < (bg1 - bg0 + 1) * per_bg; i += 32 * NCW) {
         const int bg = bg0 + i / per_bg, l = i % per_bg;
         const int bb = bg / c.Hkv, g = bg - (bg / c.Hkv) * c.Hkv;
@@ -863,9 +872,9 @@ int decode_max_partials(const CacheView& c, int ncta) {
   return (ncta + bgs - 1) / bgs + 3;
 }
 
-DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms) {
+DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms, long long skip) {
   DecodePlan pl;
-  long long n = (long long)c.B * c.Hkv * (c.L + len0) / 512;   // at least 512 cached rows per CTA
+  long long n = (long long)c.B * c.Hkv * (c.L - skip + len0) / 512;   // at least 512 cached rows per CTA
   if (n < 1) n = 1;
   if (n > num_sms) n = num_sms;
   // A whole number of CTAs per (batch, kv head), if that idles at most 4 % of
@@ -931,7 +940,9 @@ void launch_decode_kernel(const DecodeArgs& a, int G, int ncta, cudaStream_t st)
 
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
                                const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,
-                               const DecodePlan& plan, const Scratch& s, cudaStream_t st) {
+                               const DecodePlan& plan, const Scratch& s, cudaStream_t st, long long skip,
+                               bool with_token, float* o32) {
+  if (skip < 0 || skip > c.L || c.L - skip + len0 < 1) return cudaErrorInvalidValue;
   DecodeArgs a;
   a.tk_ctx = maps.k_ctx;
   a.tv_ctx = maps.v_ctx;
@@ -950,7 +961,10 @@ cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float
   a.len0 = len0;
   a.ncta = plan.ncta;
   a.maxp = plan.maxp;
-  a.rpb = c.L + len0;
+  a.rpb = c.L - skip + len0;
+  a.skip = skip;
+  a.with_token = with_token ? 1 : 0;
+  a.o32 = o32;
   a.q = q;
   a.k = k;
   a.v = v;

@@ -679,6 +679,23 @@ int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query,
   if (with_query && c->q_len + lq > w.q_cap)
     return fail(STAR_ENOSPC, "query region full: %lld + %d > q_cap %d", c->q_len, lq, w.q_cap);
   if (lq > w.q_cap) return fail(STAR_EINVAL, "lq %d beyond q_cap %d (the scratch is sized by it)", lq, w.q_cap);
+  // One row over segments that run to the end of the context (a generation
+  // step of the block-sharded layer): the split-KV decode kernel streams them
+  // at the HBM rate, where the prefill tile kernel would fill 128-row tiles
+  // from G rows.  The bf16 cache only: on an FP8 cache the decode kernel reads
+  // the E4M3 copy, which is not this call's arithmetic.
+  const long long skip = (long long)first_seg * w.b;
+  const long long len0 = with_query ? c->q_len : 0;
+  if (lq == 1 && first_seg + n_seg == w.n_seg && !w.ctxK8 && w.L - skip + len0 >= 1) {
+    const star::DecodePlan dp = star::decode_plan(w, len0, c->num_sms, skip);
+    cudaError_t e = star::launch_decode_step(
+        w, c->dmaps, c->p.scale, (int)len0, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
+        static_cast<const bf16*>(V), nullptr, s, dp, c->scratch, static_cast<cudaStream_t>(stream), skip,
+        with_query != 0, A);
+    if (e != cudaSuccess) return cuda_fail(e, "star_partial_attend launch");
+    if (with_query) c->q_len += 1;
+    return STAR_OK;
+  }
   const star::PrefillPlan pl =
       star::plan_prefill(w, c->num_sms, lq, c->q_len, first_seg, first_seg + n_seg, with_query != 0);
   cudaError_t e = star::launch_query_prefill_tc(

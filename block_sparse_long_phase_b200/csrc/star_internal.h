@@ -205,7 +205,8 @@ struct DecodePlan {
   int maxp;   // part slots per (batch, kv head)
 };
 int decode_max_partials(const CacheView& c, int ncta);
-DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms);
+// skip: leading context rows of each (batch, kv head) the step leaves out
+DecodePlan decode_plan(const CacheView& c, long long len0, int num_sms, long long skip = 0);
 
 // Span of CTA i: rows [span_start(i), span_start(i + 1)) of the R cached rows
 // of all (batch, kv head) pairs laid end to end.  Row indices stay below 2^31
@@ -254,9 +255,14 @@ cudaError_t launch_quantize_qregion_fp8(const CacheView& c, const bf16* K, const
 // driver rejected.
 const char* decode_make_maps(const CacheView& c, DecodeMaps* m);
 cudaError_t decode_prepare(int D);   // one-time kernel attributes
+// One decode step over each (batch, kv head)'s cached rows past its first
+// `skip` context rows, then the query region's len0 rows and, with_token, the
+// step's own k, v (appended at region row len0).  o (bf16) and o32 (float32)
+// may each be null; lse is written.
 cudaError_t launch_decode_step(const CacheView& c, const DecodeMaps& maps, float scale, int len0,
                                const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse,
-                               const DecodePlan& plan, const Scratch& s, cudaStream_t st);
+                               const DecodePlan& plan, const Scratch& s, cudaStream_t st, long long skip = 0,
+                               bool with_token = true, float* o32 = nullptr);
 
 cudaError_t attn_tc_prepare(int D);   // one-time kernel attributes
 int prefill_row_pairs(const CacheView& c, int lq);   // 256-row pairs of packed query rows

@@ -54,8 +54,8 @@ TRAFFIC = {
     # anchored blocks: each anchored 64K-row block is an L2 group of its own)
     "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0cc8dda248e6e11f", 56290663552),
     "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0cc8dda248e6e11f", 1382001664),
-    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "b36c09b7fa823fac", 543239168),
-    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "b36c09b7fa823fac", 290013696),
+    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 543390976),
+    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 287083008),
 }
 
 

@@ -25,7 +25,8 @@ EXPORTS = (
     "star_cache_segment", "star_cache_segment_fp8", "star_cache_reset_query", "star_ctx_encode",
     "star_query_prefill", "star_query_prefill_partials", "star_decode_step", "star_lse_merge",
     "star_decode_step_noalloc", "star_last_error", "star_version",
-    "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_host",
+    "star_rope", "star_anchor_keys", "star_ctx_encode_anchored", "star_ctx_encode_after_anchor",
+    "star_ctx_encode_host",
     "star_selftest_wait_timeout", "star_noalloc_device_error", "star_ctx_encode_fp32",
     "star_decode_step_partials", "star_partial_attend",
     "star_lse_merge_bf16", "star_cache_check_guards", "star_plan_prefill", "star_prefill_span_tiles",
@@ -78,6 +79,7 @@ def load(path: str = LIB_PATH):
     lib.star_rope.argtypes = [i, i, ll, i, ctypes.c_double, vp, ll, vp, vp, vp]
     lib.star_anchor_keys.argtypes = [vp, i, vp, ctypes.c_double, vp, vp, vp]
     lib.star_ctx_encode_anchored.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.star_ctx_encode_after_anchor.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.star_decode_step_noalloc.argtypes = [ctypes.POINTER(StarParams), ll, vp, vp, vp, vp,
                                              vp, vp, vp, vp, vp, vp]
     lib.star_noalloc_device_error.argtypes = [ctypes.POINTER(i), vp]

@@ -166,6 +166,28 @@ class StarCache:
                                                      _ptr(LSE), _stream(Q.device)))
         return O, LSE
 
+    def star_ctx_encode_after_anchor(self, Q, K, V, Ka, Va, O=None, LSE=None):
+        """Phase 1 of blocks that all follow an anchor held outside this
+        context: every block, block 0 included, attends to ``Ka``, ``Va``
+        [B, Hkv, anchor, D] bf16 and causally to itself."""
+        B, Hq, Hkv, D, L = self.B, self.Hq, self.Hkv, self.D, self.L
+        _need(Q, (B, Hq, L, D), torch.bfloat16, "Q")
+        _need(K, (B, Hkv, L, D), torch.bfloat16, "K")
+        _need(V, (B, Hkv, L, D), torch.bfloat16, "V")
+        if self.anchor > 0:
+            _need(Ka, (B, Hkv, self.anchor, D), torch.bfloat16, "Ka")
+            _need(Va, (B, Hkv, self.anchor, D), torch.bfloat16, "Va")
+        if O is None:
+            O = torch.empty((B, Hq, L, D), dtype=torch.bfloat16, device=Q.device)
+        if LSE is None:
+            LSE = torch.empty((B, Hq, L), dtype=torch.float32, device=Q.device)
+        _need(O, (B, Hq, L, D), torch.bfloat16, "O")
+        _need(LSE, (B, Hq, L), torch.float32, "LSE")
+        _abi.check(self.lib.star_ctx_encode_after_anchor(
+            self.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(Ka) if self.anchor > 0 else None,
+            _ptr(Va) if self.anchor > 0 else None, _ptr(O), _ptr(LSE), _stream(Q.device)))
+        return O, LSE
+
     def star_ctx_encode_fp32(self, Q, K, V, O=None, LSE=None, O32=None):
         """Debug form of phase 1: also returns O32 [B, Hq, L, D] float32, the
         rows before their bf16 rounding.  Returns (O, LSE, O32)."""

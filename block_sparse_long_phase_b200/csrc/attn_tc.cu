@@ -74,8 +74,8 @@ struct CtxTcArgs {
   CUtensorMap tk;   // phase 1: K as [B*Hkv*L][D]; prefill: context cache as [B*Hkv*L][D]
   CUtensorMap tv;
   CUtensorMap tkq;  // prefill: query region as [B*Hkv*q_cap][D]; phase 1: anchor keys as
-                    // [(n-1)*B*Hkv*b_a][D] when anchor_keys is set
-  CUtensorMap tvq;
+                    // [(n-1)*B*Hkv*b_a][D] (anchor_keys 1) or [B*Hkv*b_a][D] (anchor_keys 2)
+  CUtensorMap tvq;  // prefill: query region V; phase 1, anchor_keys 2: anchor V [B*Hkv*b_a][D]
   CacheView c;
   float scale_log2;
   const bf16* K;
@@ -85,7 +85,9 @@ struct CtxTcArgs {
   float* O32;         // phase 1, debug: the rows before their bf16 rounding (null: none)
   const int4* work;   // phase 1: (b*Hkv + g, head pair, block, q tile)
   int* err;
-  int anchor_keys;    // phase 1: block i >= 1 reads its anchor's K tiles from tkq
+  int anchor_keys;    // phase 1: 1 -- block i >= 1 reads its anchor's K tiles from tkq;
+                      // 2 -- every block, 0 included, follows an anchor held outside this
+                      //      context: its K and V tiles from tkq and tvq
   // prefill
   int lq, len0, row_pairs;
   float* partA;
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
     const long long bend = bstart + c.b < c.L ? bstart + c.b : c.L;
     t0 = bstart + (long long)w.w * BM;
     n_rows0 = n_rows1 = (int)((bend - t0) < BM ? (bend - t0) : BM);
-    n_anchor = blk > 0 ? (c.b_a + BN - 1) / BN : 0;
+    n_anchor = (blk > 0 || a.anchor_keys == 2) ? (c.b_a + BN - 1) / BN : 0;
     n_kv = n_anchor + w.w + 1;
     kv_row0 = (long long)bg * c.L;                          // (b, g, token 0) in the K/V maps
     qrow0 = ((long long)bb * c.Hq + h0) * c.L + t0;         // Q0's first row; Q1 is one head later
@@ -238,8 +240,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
       }
       int pf_row = 0;
       bool pf_region = false, region_ready = false;
-      const bool own_anchor = !PF && a.anchor_keys && blk > 0;   // per-block anchor keys
-      if (own_anchor) prefetch_tmap(&a.tkq);
+      const bool own_anchor = !PF && a.anchor_keys == 1 && blk > 0;   // per-block anchor keys
+      const bool ext_anchor = !PF && a.anchor_keys == 2;                // anchor K, V outside
+      if (own_anchor || ext_anchor) prefetch_tmap(&a.tkq);
+      if (ext_anchor) prefetch_tmap(&a.tvq);
       if (PF && a.wait_first) {
         griddep_wait();                                 // inputs written by the kernel before this one
         region_ready = true;
@@ -279,6 +283,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) attn_tc_kernel(const __grid_const
           // K of block blk's anchor: rows of Ka[blk - 1] for this (batch, kv head)
           m = &a.tkq;
           row = (int)((((long long)(blk - 1) * c.B * c.Hkv) + bg) * c.b_a + tok);
+        }
+        if (ext_anchor && j < n_anchor) {
+          // the anchor's K / V rows for this (batch, kv head)
+          m = (i & 1) ? &a.tvq : &a.tkq;
+          row = (int)((long long)bg * c.b_a + tok);
         }
         const uint32_t fb = smem_u32(&bar_kv_full[slot]);
         mbar_arrive_expect_tx(fb, S::TILE);
@@ -662,7 +671,7 @@ cudaError_t attn_tc_prepare(int D) {
 
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
-                                 int* err, cudaStream_t st, const bf16* Ka, float* O32) {
+                                 int* err, cudaStream_t st, const bf16* Ka, float* O32, const bf16* Va) {
   if (n_work == 0) return cudaSuccess;
   CtxTcArgs a;
   memset(&a, 0, sizeof(a));
@@ -671,7 +680,15 @@ cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q,
   if (!make_tmap_bf16_2d(&a.tq, Q, qrows, c.D, BM, 64) || !make_tmap_bf16_2d(&a.tk, K, kvrows, c.D, BN, 64) ||
       !make_tmap_bf16_2d(&a.tv, V, kvrows, c.D, BN, 64))
     return cudaErrorInvalidValue;
-  if (Ka && c.n_seg > 1 && c.b_a > 0) {
+  if (Ka && Va) {
+    // every block follows the anchor Ka, Va [B][Hkv][b_a][D] (no anchor: plain blocks)
+    if (c.b_a > 0) {
+      const unsigned long long arows = (unsigned long long)c.B * c.Hkv * c.b_a;
+      if (!make_tmap_bf16_2d(&a.tkq, Ka, arows, c.D, BN, 64) || !make_tmap_bf16_2d(&a.tvq, Va, arows, c.D, BN, 64))
+        return cudaErrorInvalidValue;
+      a.anchor_keys = 2;
+    }
+  } else if (Ka && c.n_seg > 1 && c.b_a > 0) {
     const unsigned long long karows = (unsigned long long)(c.n_seg - 1) * c.B * c.Hkv * c.b_a;
     if (!make_tmap_bf16_2d(&a.tkq, Ka, karows, c.D, BN, 64)) return cudaErrorInvalidValue;
     a.anchor_keys = 1;

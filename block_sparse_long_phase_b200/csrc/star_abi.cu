@@ -452,16 +452,16 @@ namespace {
 // star_ctx_encode and its forms: per-block anchor keys (Ka) and the float32
 // debug rows (O32), either may be null.
 int ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, const void* Ka, void* O,
-               float* LSE, float* O32, void* stream) {
+               float* LSE, float* O32, void* stream, const void* Va = nullptr) {
   if (!c) return fail(STAR_EINVAL, "cache is NULL");
   if (!Q || !K || !V || !O || !LSE) return fail(STAR_EINVAL, "NULL tensor pointer");
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
-      (Ka && !aligned16(Ka)) || (O32 && !aligned16(O32)))
+      (Ka && !aligned16(Ka)) || (Va && !aligned16(Va)) || (O32 && !aligned16(O32)))
     return fail(STAR_EINVAL, "tensor pointers must be 16-byte aligned");
   cudaError_t e = star::launch_ctx_encode_tc(
       c->view, c->p.scale, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),
       static_cast<const bf16*>(V), static_cast<bf16*>(O), LSE, c->ctx_work, c->n_ctx_work, c->scratch.err,
-      static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka), O32);
+      static_cast<cudaStream_t>(stream), static_cast<const bf16*>(Ka), O32, static_cast<const bf16*>(Va));
   if (e == cudaErrorInvalidValue) return fail(STAR_EINVAL, "TMA tensor map rejected (alignment or size)");
   if (e == cudaSuccess && c->view.ctxK8) e = star::launch_quantize_ctx_fp8(c->view, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "star_ctx_encode launch");
@@ -480,6 +480,14 @@ int star_ctx_encode_anchored(star_cache* c, const void* Q, const void* K, const 
 int star_ctx_encode(star_cache* c, const void* Q, const void* K, const void* V, void* O,
                     float* LSE, void* stream) {
   return ctx_encode(c, Q, K, V, nullptr, O, LSE, nullptr, stream);
+}
+
+int star_ctx_encode_after_anchor(star_cache* c, const void* Q, const void* K, const void* V,
+                                 const void* Ka, const void* Va, void* O, float* LSE, void* stream) {
+  if (!c) return fail(STAR_EINVAL, "cache is NULL");
+  if (c->view.b_a > 0 && (!Ka || !Va)) return fail(STAR_EINVAL, "NULL anchor pointer");
+  if (c->view.b_a == 0) return ctx_encode(c, Q, K, V, nullptr, O, LSE, nullptr, stream);
+  return ctx_encode(c, Q, K, V, Ka, O, LSE, nullptr, stream, Va);
 }
 
 int star_ctx_encode_fp32(star_cache* c, const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -684,7 +692,7 @@ int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query,
   // at the HBM rate, where the prefill tile kernel would fill 128-row tiles
   // from G rows.  The bf16 cache only: on an FP8 cache the decode kernel reads
   // the E4M3 copy, which is not this call's arithmetic.
-  const long long skip = (long long)first_seg * w.b;
+  const long long skip = std::min<long long>((long long)first_seg * w.b, w.L);   // rows before first_seg
   const long long len0 = with_query ? c->q_len : 0;
   if (lq == 1 && first_seg + n_seg == w.n_seg && !w.ctxK8 && w.L - skip + len0 >= 1) {
     const star::DecodePlan dp = star::decode_plan(w, len0, c->num_sms, skip);

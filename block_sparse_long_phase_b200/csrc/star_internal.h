@@ -90,11 +90,13 @@ struct CtxUnit {
 void ctx_tc_fill_units(const CacheView& c, int num_sms, std::vector<CtxUnit>& units, int4* out);
 // Ka (may be null): anchor keys of blocks 1..n-1 as [n-1][B][Hkv][b_a][D];
 // block i >= 1 then reads its anchor keys from Ka[i-1] instead of K rows 0..b_a-1.
+// With Va too, Ka and Va are one anchor [B][Hkv][b_a][D] held outside this
+// context that every block, block 0 included, follows.
 // O32 (may be null): the phase-1 rows in float32 before their bf16 rounding.
 cudaError_t launch_ctx_encode_tc(const CacheView& c, float scale, const bf16* Q, const bf16* K,
                                  const bf16* V, bf16* O, float* LSE, const int4* work, int n_work,
                                  int* err, cudaStream_t st, const bf16* Ka = nullptr,
-                                 float* O32 = nullptr);
+                                 float* O32 = nullptr, const bf16* Va = nullptr);
 
 // Rotary embedding of rows: for group z < groups, batch b < B, head h < H and
 // t < n, row (z*x_grp + (b*H + h)*x_seq + t) of x is rotated at position

@@ -12,18 +12,17 @@ the query and generated tokens (Step 7).
 
 A host here is one process per GPU in a torch.distributed group.  Rank r
 holds the contiguous blocks ``block_ranges(n, world)[r]``; the last rank is
-the query host.  A rank whose blocks start after block 0 encodes the local
-context [anchor | zero rows up to one block | its own blocks] with the same
-block size: its local block 0 is then the anchor block (whose output is
-dropped, and which phase 2 never reads), and its local block j >= 1 is
-global block first + j - 1, whose mask -- the whole anchor, then itself
-causally -- is exactly the single-GPU one.  This costs each such rank one
-anchor block of causal attention, which the pages' hosts spend too (they
-encode the anchor tokens of their augmented block).
+the query host.  A rank's local context is its own rows, cut into blocks of
+the same size: the rank holding block 0 encodes them as a context of its own
+(star_ctx_encode), every other rank encodes each of its blocks behind the
+anchor rows it receives (star_ctx_encode_after_anchor), so local block j is
+global block first + j with exactly the single-GPU mask: the whole anchor,
+then itself causally.  A rank without blocks keeps a one-row placeholder
+context that is never encoded or attended.
 
 Everything arithmetic runs in libstar's kernels (star_ctx_encode,
-star_partial_attend, star_lse_merge_bf16); this module partitions, lays out
-inputs and moves the partials (one ``all_gather`` per call: B*Hq*lq*(D+1)
+star_ctx_encode_after_anchor, star_partial_attend, star_lse_merge_bf16); this
+module partitions, slices inputs and moves the partials (one ``all_gather`` per call: B*Hq*lq*(D+1)
 floats per rank, a few KB per decode step).  No remote memory is ever read by
 a kernel or a TMA copy: the partials land in each rank's own buffers first.
 
@@ -53,24 +52,19 @@ class LocalLayout:
     n_blocks: int        # how many (may be 0)
     rows0: int           # first global context row of the rank
     rows: int            # its context rows
-    pad: bool            # local context = [anchor | zeros | own rows]
-    L_local: int         # local context length
-    first_seg: int       # local segment of the first own block
-
-    @property
-    def offset(self) -> int:
-        """Local row of the rank's first own row."""
-        return self.L_local - self.rows
+    L_local: int         # local context length: its rows (a one-row placeholder when none)
+    first_seg: int       # local segment of the first own block (1, past the placeholder, when none)
+    after_anchor: bool   # its blocks follow an anchor it does not hold (the first block is not 0)
 
 
 def local_layout(rank: int, world: int, L: int, b: int) -> LocalLayout:
     n = -(-L // b)
     i0, i1 = block_ranges(n, world)[rank]
+    if i1 == i0:
+        return LocalLayout(i0, 0, min(i0 * b, L), 0, 1, 1, False)
     rows0 = i0 * b
-    rows = max(0, min(i1 * b, L) - rows0)
-    if i0 == 0 and i1 > 0:
-        return LocalLayout(i0, i1 - i0, 0, rows, False, rows, 0)
-    return LocalLayout(i0, i1 - i0, rows0, rows, True, b + rows, 1)
+    rows = min(i1 * b, L) - rows0
+    return LocalLayout(i0, i1 - i0, rows0, rows, rows, 0, i0 > 0)
 
 
 class LibstarOps:
@@ -83,15 +77,15 @@ class LibstarOps:
     def ctx_encode(self, cache, Q, K, V):
         return cache.star_ctx_encode(Q, K, V)
 
+    def ctx_encode_after_anchor(self, cache, Q, K, V, Ka, Va):
+        return cache.star_ctx_encode_after_anchor(Q, K, V, Ka, Va)
+
     def partial_attend(self, cache, Q, first_seg, n_seg, K=None, V=None):
         return cache.star_partial_attend(Q, first_seg, n_seg, K, V)
 
     def lse_merge(self, A, s):
         from .api import star_lse_merge_bf16
         return star_lse_merge_bf16(A, s)
-
-    def zeros(self, shape, dtype, device):
-        return torch.zeros(shape, dtype=dtype, device=device)
 
 
 class ShardedStarCache:
@@ -130,16 +124,12 @@ class ShardedStarCache:
         [B, Hkv, b_a, D] (the anchor block, copied to every rank once).
         Returns (O, LSE) of the rank's own rows."""
         lay = self.layout
-        if not lay.pad:
-            O, LSE = self.ops.ctx_encode(self.cache, Q_own, K_own, V_own)
-            return O, LSE
-        B, Hq, Hkv, D, b, ba = self.B, self.Hq, self.Hkv, self.D, self.block, self.anchor
-        dev, dt = Q_own.device, Q_own.dtype
-        Q = torch.cat([self.ops.zeros((B, Hq, b, D), dt, dev), Q_own], dim=2)
-        K = torch.cat([K_anchor, self.ops.zeros((B, Hkv, b - ba, D), dt, dev), K_own], dim=2)
-        V = torch.cat([V_anchor, self.ops.zeros((B, Hkv, b - ba, D), dt, dev), V_own], dim=2)
-        O, LSE = self.ops.ctx_encode(self.cache, Q, K, V)
-        return O[:, :, b:], LSE[:, :, b:]
+        if lay.n_blocks == 0:
+            return (Q_own.new_empty((self.B, self.Hq, 0, self.D)),
+                    Q_own.new_empty((self.B, self.Hq, 0), dtype=torch.float32))
+        if not lay.after_anchor:
+            return self.ops.ctx_encode(self.cache, Q_own, K_own, V_own)
+        return self.ops.ctx_encode_after_anchor(self.cache, Q_own, K_own, V_own, K_anchor, V_anchor)
 
     # -- phase 2 ---------------------------------------------------------------
     def local_partial(self, Q, K=None, V=None):

@@ -196,6 +196,19 @@ STAR_API int star_ctx_encode_host(star_cache* c, const void* hQ, const void* hK,
 STAR_API int star_anchor_keys(const star_cache* c, int mode, const int* pos, double theta,
                               const void* K, void* Ka, void* stream);
 
+/* Phase 1 of blocks that follow an anchor held outside this context ([P2]
+ * Phase 1 Steps 3-4, one host's blocks when the context is spread over
+ * several GPUs: every host but the first receives the anchor and encodes
+ * each of its blocks behind it).  Every block i of this cache -- block 0
+ * included -- attends to the anchor rows Ka, Va [B][Hkv][b_a][D] bf16
+ * (the longer context's rows 0..b_a-1, already rotated at their positions)
+ * with no mask, and to its own rows causally.  Q, K, V, O, LSE and the cache
+ * as star_ctx_encode; the anchor rows are only read.  With b_a = 0 the
+ * blocks are plain causal blocks (star_ctx_encode) and Ka, Va may be NULL. */
+STAR_API int star_ctx_encode_after_anchor(star_cache* c, const void* Q, const void* K, const void* V,
+                                          const void* Ka, const void* Va, void* O, float* LSE,
+                                          void* stream);
+
 /* Phase 1 as star_ctx_encode, except that block i >= 1 attends to the
  * anchor keys Ka[i-1] (from star_anchor_keys) instead of K rows
  * 0..b_a-1; the anchor's values are V rows 0..b_a-1 as before.  Q and K are

@@ -29,6 +29,28 @@ class OracleOps:
         c.q_len = 0
         return torch.from_numpy(O), torch.from_numpy(LSE)
 
+    def ctx_encode_after_anchor(self, c, Q, K, V, Ka, Va):
+        """Every block behind the anchor rows Ka, Va: the anchor with no mask,
+        then the block's own rows causally (the single-GPU mask of a block
+        i >= 1, written out block by block)."""
+        q, k, v, ka, va = (so._f64(t) for t in (Q, K, V, Ka, Va))
+        B, Hq, L, D = q.shape
+        G = Hq // c.Hkv
+        O = np.zeros((B, Hq, L, D))
+        LSE = np.zeros((B, Hq, L))
+        for s0, n in so.block_table(L, c.b):
+            mask = np.concatenate([np.ones((n, c.b_a), dtype=bool), np.tril(np.ones((n, n), dtype=bool))], axis=1)
+            for bi in range(B):
+                for h in range(Hq):
+                    g = h // G
+                    keys = np.concatenate([ka[bi, g], k[bi, g, s0:s0 + n]], axis=0)
+                    vals = np.concatenate([va[bi, g], v[bi, g, s0:s0 + n]], axis=0)
+                    O[bi, h, s0:s0 + n], LSE[bi, h, s0:s0 + n] = so.masked_attention(
+                        q[bi, h, s0:s0 + n], keys, vals, mask, c.scale)
+        c.segs = so.cache_segments(k, v, c.b)
+        c.q_len = 0
+        return torch.from_numpy(O), torch.from_numpy(LSE)
+
     def partial_attend(self, c, Q, first_seg, n_seg, K=None, V=None):
         q = so._f64(Q)
         B, Hq, lq, D = q.shape
@@ -40,8 +62,9 @@ class OracleOps:
         s = np.full((B, Hq, lq), -np.inf)
         for bi in range(B):
             for g in range(c.Hkv):
-                ks = [seg[2][bi, g] for seg in c.segs[first_seg:first_seg + n_seg]]
-                vs = [seg[3][bi, g] for seg in c.segs[first_seg:first_seg + n_seg]]
+                segs = (c.segs or [])[first_seg:first_seg + n_seg]   # a rank without blocks encodes none
+                ks = [seg[2][bi, g] for seg in segs]
+                vs = [seg[3][bi, g] for seg in segs]
                 n_ctx = sum(len(k) for k in ks)
                 nq = c.q_len + lq if K is not None else 0
                 ks.append(c.qk[bi, g, :nq])
@@ -59,6 +82,3 @@ class OracleOps:
     def lse_merge(self, A, s):
         O, L = so.lse_merge(A.numpy(), s.numpy())
         return torch.from_numpy(O), torch.from_numpy(L)
-
-    def zeros(self, shape, dtype, device):
-        return torch.zeros(shape, dtype=dtype, device=device)

@@ -102,3 +102,100 @@ def test_partial_attend_over_every_segment_equals_the_prefill():
     assert (A0 == 0).all() and torch.isinf(s0).all() and (s0 < 0).all()
     a.close()
     b.close()
+
+
+TAIL_SHAPES = {
+    "tiny": dict(L=1000, b=256, b_a=100, lq=5, T=0),
+    "d128-gqa8": dict(Hq=16, Hkv=2, D=128, L=700, b=128, b_a=128, lq=3, T=0),
+    "g16-batch2": dict(B=2, Hq=16, Hkv=1, L=600, b=200, b_a=50, lq=4, T=0),
+}
+
+
+@pytest.mark.parametrize("name", list(TAIL_SHAPES))
+def test_single_row_partials_over_tail_ranges(name):
+    """One row over segments [first, n) -- the sharded layer's generation
+    step, which runs on the split-KV decode kernel with the leading rows left
+    out -- against the oracle's local partial over the same keys: every
+    first segment (n: no context at all), without the query region, and with
+    it after a prefill (the token appended and attended)."""
+    from block_sparse_long_phase_b200 import StarCache
+    w = wl.get("tiny").with_(**TAIL_SHAPES[name])
+    cpu = wl.make_inputs(w, "cpu")
+    x = {k: v.cuda() for k, v in cpu.items()}
+    G = w.Hq // w.Hkv
+    n = -(-w.L // w.b)
+    Kc, Vc = so._f64(cpu["Kc"]), so._f64(cpu["Vc"])
+    q1 = (torch.randn((w.B, w.Hq, 1, w.D), generator=torch.Generator().manual_seed(11))).to(torch.bfloat16)
+    k1 = (torch.randn((w.B, w.Hkv, 1, w.D), generator=torch.Generator().manual_seed(12))).to(torch.bfloat16)
+    v1 = (torch.randn((w.B, w.Hkv, 1, w.D), generator=torch.Generator().manual_seed(13))).to(torch.bfloat16)
+    for first in range(n + 1):
+        for with_query in (0, 1):
+            c = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + 1, w.scale)
+            c.star_ctx_encode(x["Qc"], x["Kc"], x["Vc"])
+            c.star_query_prefill(x["Qq"], x["Kq"], x["Vq"])
+            if with_query:
+                A, s = c.star_partial_attend(q1.cuda(), first, n - first, k1.cuda(), v1.cuda())
+            else:
+                A, s = c.star_partial_attend(q1.cuda(), first, n - first)
+            torch.cuda.synchronize()
+            assert c.device_error() == 0
+            keys_k = [Kc[:, :, first * w.b:]]
+            keys_v = [Vc[:, :, first * w.b:]]
+            if with_query:
+                keys_k += [so._f64(cpu["Kq"]), so._f64(k1)]
+                keys_v += [so._f64(cpu["Vq"]), so._f64(v1)]
+                assert c.q_len == w.lq + 1
+            else:
+                assert c.q_len == w.lq
+            kk, vv = np.concatenate(keys_k, axis=2), np.concatenate(keys_v, axis=2)
+            q = so._f64(q1)
+            for bi in range(w.B):
+                for h in range(w.Hq):
+                    g = h // G
+                    a_ref, s_ref = so.local_partial(q[bi, h], kk[bi, g], vv[bi, g], w.scale)
+                    what = f"{name} first {first} query {with_query} b{bi} h{h}"
+                    got_a = A[bi, h].double().cpu().numpy()
+                    got_s = s[bi, h].double().cpu().numpy()
+                    if kk.shape[2] == 0:
+                        assert (got_a == 0).all() and np.isneginf(got_s).all(), what
+                        continue
+                    assert np.abs(got_a - a_ref).max() <= 1e-2, what
+                    assert np.abs(got_a - a_ref).mean() <= 1e-3, what
+                    assert np.abs(got_s - s_ref).max() <= 1e-3, what
+            c.close()
+
+
+AFTER_ANCHOR = {
+    "tiny": dict(L=1024, b=256, b_a=256),
+    "anchor-shorter-ragged": dict(L=1000, b=256, b_a=100),
+    "d128-gqa4": dict(Hq=16, Hkv=4, D=128, L=777, b=128, b_a=128),
+    "batch2-g1": dict(B=2, Hq=4, Hkv=4, L=600, b=200, b_a=37),
+    "many-blocks": dict(L=48 * 20, b=48, b_a=48),
+}
+
+
+@pytest.mark.parametrize("name", list(AFTER_ANCHOR))
+def test_ctx_encode_after_anchor_matches_the_oracle(name):
+    """Blocks 1..n-1 of a context encoded as a context of their own behind the
+    anchor rows (star_ctx_encode_after_anchor, every local block anchored)
+    give the single-device rows of those blocks, and the cache holds each
+    block's own K/V rows bit for bit."""
+    from block_sparse_long_phase_b200 import StarCache
+    w = wl.get("tiny").with_(**AFTER_ANCHOR[name])
+    cpu = wl.make_inputs(w, "cpu")
+    x = {k: v.cuda() for k, v in cpu.items()}
+    r0 = w.b
+    c = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L - r0, w.b, w.b_a, 1, w.scale)
+    O, LSE = c.star_ctx_encode_after_anchor(
+        x["Qc"][:, :, r0:].contiguous(), x["Kc"][:, :, r0:].contiguous(), x["Vc"][:, :, r0:].contiguous(),
+        x["Kc"][:, :, :w.b_a].contiguous(), x["Vc"][:, :, :w.b_a].contiguous())
+    torch.cuda.synchronize()
+    assert c.device_error() == 0
+    Oref, Lref = so.ctx_encode(cpu["Qc"], cpu["Kc"], cpu["Vc"], w.b, w.b_a, w.scale, rows=np.arange(r0, w.L))
+    assert_close(O, Oref, LSE, Lref, f"{name}: after-anchor phase 1")
+    for j in range(c.num_segments - 1):
+        k, v, seg = c.segment_tensors(j)
+        s0 = r0 + j * w.b
+        assert torch.equal(k.view(torch.int16), x["Kc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
+        assert torch.equal(v.view(torch.int16), x["Vc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
+    c.close()

@@ -41,11 +41,18 @@ def test_block_ranges_and_layouts():
             assert all(a[1] == b_[0] for a, b_ in zip(r, r[1:]))
             assert max(e - s for s, e in r) - min(e - s for s, e in r) <= 1
     lay = local_layout(0, 3, 1000, 256)            # 4 blocks over 3 ranks: [0,1) [1,2) [2,4)
-    assert (lay.pad, lay.L_local, lay.first_seg, lay.n_blocks) == (False, 256, 0, 1)
+    assert (lay.after_anchor, lay.L_local, lay.first_seg, lay.n_blocks) == (False, 256, 0, 1)
     lay = local_layout(2, 3, 1000, 256)
-    assert (lay.pad, lay.rows0, lay.rows, lay.L_local, lay.first_seg) == (True, 512, 488, 256 + 488, 1)
+    assert (lay.after_anchor, lay.rows0, lay.rows, lay.L_local, lay.first_seg) == (True, 512, 488, 488, 0)
     lay = local_layout(2, 3, 300, 256)             # 2 blocks over 3 ranks: rank 0 holds none
-    assert local_layout(0, 3, 300, 256).n_blocks == 0 and lay.n_blocks == 1
+    empty = local_layout(0, 3, 300, 256)
+    assert (empty.n_blocks, empty.rows, empty.L_local, empty.first_seg) == (0, 0, 1, 1)
+    assert (lay.n_blocks, lay.rows0, lay.rows, lay.after_anchor) == (1, 256, 44, True)
+    # every row of the context is held by exactly one rank
+    for L, b, world in ((1000, 256, 3), (300, 256, 3), (4096, 512, 8), (777, 100, 5)):
+        lays = [local_layout(r, world, L, b) for r in range(world)]
+        assert sum(x.rows for x in lays) == L
+        assert all(x.rows0 + x.rows == y.rows0 for x, y in zip(lays, lays[1:]) if x.n_blocks and y.n_blocks)
 
 
 def _worker(rank, world, port, shape, q):

@@ -23,7 +23,8 @@ context that is never encoded or attended.
 Everything arithmetic runs in libstar's kernels (star_ctx_encode,
 star_ctx_encode_after_anchor, star_partial_attend, star_lse_merge_bf16); this
 module partitions, slices inputs and moves the partials (one ``all_gather`` per call: B*Hq*lq*(D+1)
-floats per rank, a few KB per decode step).  No remote memory is ever read by
+floats per rank, a few KB per decode step, after one broadcast of the query
+rows).  No remote memory is ever read by
 a kernel or a TMA copy: the partials land in each rank's own buffers first.
 
 The kernel calls go through an ``ops`` object (``LibstarOps`` by default) so
@@ -149,22 +150,33 @@ class ShardedStarCache:
         return O.view(B, Hq, lq, D), LSE.view(B, Hq, lq)
 
     def _gather(self, A, s):
+        """Every rank's (A, s), stacked in rank order: one all_gather of the
+        partials packed as [A | s] float32 rows (the collective is
+        latency-bound at these sizes, so one call rather than two)."""
         if self.world == 1:
             return A[None], s[None]
         import torch.distributed as dist
-        As = [torch.empty_like(A) for _ in range(self.world)]
-        ss = [torch.empty_like(s) for _ in range(self.world)]
-        dist.all_gather(As, A.contiguous(), group=self.group)
-        dist.all_gather(ss, s.contiguous(), group=self.group)
-        return torch.stack(As), torch.stack(ss)
+        B, Hq, lq, D = A.shape
+        packed = torch.cat([A.reshape(B * Hq * lq, D), s.reshape(B * Hq * lq, 1)], dim=1).contiguous()
+        out = torch.empty((self.world * packed.shape[0], D + 1), dtype=packed.dtype, device=packed.device)
+        dist.all_gather_into_tensor(out, packed, group=self.group)
+        out = out.view(self.world, B * Hq * lq, D + 1)
+        return (out[:, :, :D].reshape(self.world, B, Hq, lq, D),
+                out[:, :, D].reshape(self.world, B, Hq, lq))
 
     def _broadcast(self, *xs):
+        """The query rank's tensors to every rank, in one broadcast of their
+        concatenated bytes."""
         if self.world == 1:
             return xs
         import torch.distributed as dist
+        flat = torch.cat([x.reshape(-1) for x in xs]).contiguous()
+        dist.broadcast(flat, src=self.query_rank, group=self.group)
+        out, o = [], 0
         for x in xs:
-            dist.broadcast(x, src=self.query_rank, group=self.group)
-        return xs
+            out.append(flat[o:o + x.numel()].view(x.shape))
+            o += x.numel()
+        return tuple(out)
 
     def query_prefill(self, Q, K, V):
         """Phase 2 for the query rows: Q [B, Hq, lq, D], K, V [B, Hkv, lq, D]

@@ -52,8 +52,8 @@ METRIC = "ctx-encode tok/s & decode tok/s per attn layer; % of bf16 TC / HBM roo
 TRAFFIC = {
     # the 1M launch scaled from captures at L = b and L = 3b (block 0, then two
     # anchored blocks: each anchored 64K-row block is an L2 group of its own)
-    "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0cc8dda248e6e11f", 56290663552),
-    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "0cc8dda248e6e11f", 1382001664),
+    "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3da1c828dfe05ede", 55308552448),
+    "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3da1c828dfe05ede", 1448725248),
     "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 543390976),
     "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 287083008),
 }

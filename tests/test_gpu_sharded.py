@@ -171,6 +171,7 @@ AFTER_ANCHOR = {
     "d128-gqa4": dict(Hq=16, Hkv=4, D=128, L=777, b=128, b_a=128),
     "batch2-g1": dict(B=2, Hq=4, Hkv=4, L=600, b=200, b_a=37),
     "many-blocks": dict(L=48 * 20, b=48, b_a=48),
+    "no-anchor": dict(L=500, b=128, b_a=0),
 }
 
 
@@ -186,9 +187,10 @@ def test_ctx_encode_after_anchor_matches_the_oracle(name):
     x = {k: v.cuda() for k, v in cpu.items()}
     r0 = w.b
     c = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L - r0, w.b, w.b_a, 1, w.scale)
+    Ka = x["Kc"][:, :, :w.b_a].contiguous() if w.b_a else None
+    Va = x["Vc"][:, :, :w.b_a].contiguous() if w.b_a else None
     O, LSE = c.star_ctx_encode_after_anchor(
-        x["Qc"][:, :, r0:].contiguous(), x["Kc"][:, :, r0:].contiguous(), x["Vc"][:, :, r0:].contiguous(),
-        x["Kc"][:, :, :w.b_a].contiguous(), x["Vc"][:, :, :w.b_a].contiguous())
+        x["Qc"][:, :, r0:].contiguous(), x["Kc"][:, :, r0:].contiguous(), x["Vc"][:, :, r0:].contiguous(), Ka, Va)
     torch.cuda.synchronize()
     assert c.device_error() == 0
     Oref, Lref = so.ctx_encode(cpu["Qc"], cpu["Kc"], cpu["Vc"], w.b, w.b_a, w.scale, rows=np.arange(r0, w.L))

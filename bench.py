@@ -54,8 +54,8 @@ TRAFFIC = {
     # anchored blocks: each anchored 64K-row block is an L2 group of its own)
     "phase1 8b-1m": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3da1c828dfe05ede", 55308552448),
     "phase1 8b-32k": ("block_sparse_long_phase_b200/csrc/attn_tc.cu", "3da1c828dfe05ede", 1448725248),
-    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 543390976),
-    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "14fda9e9e8c18cde", 287083008),
+    "decode 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "0bfa638da1bfd739", 543287808),
+    "decode fp8 8b-128k": ("block_sparse_long_phase_b200/csrc/decode_splitkv.cu", "0bfa638da1bfd739", 286823680),
 }
 
 

@@ -49,7 +49,6 @@ constexpr int KS8 = 256;                // keys per FP8 context stage (32 per co
 constexpr int NSTAGE = 3;
 constexpr int NCW = 8;                  // consumer warps
 constexpr int NTHREADS = 32 * (NCW + 1);
-constexpr int kMaxG = 16;
 
 struct StageMeta {
   int n;         // valid keys in the stage

@@ -58,8 +58,6 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-long long round_up(long long x, long long m) { return (x + m - 1) / m * m; }
-
 // Canary guard after each part of a cache's allocation.
 constexpr size_t kGuardBytes = 4096;
 constexpr int kCanary = 0xA5;

@@ -691,7 +691,10 @@ def measure_e2e(args, w, x, O, LSE, cache, flush, dev, world):
     except Exception:
         avail = None
     own = None
-    if avail is not None and need * local_world > avail // 2:
+    small = avail is not None and need * local_world > avail // 2
+    # every rank takes the same workload: the smaller one if any rank's node is short
+    (small_any,) = max_over_ranks([1.0 if small else 0.0], dev, world)
+    if small_any > 0:
         w = wl.get("8b-128k-needle")
         x = wl.make_inputs(w, dev, with_decode=False)
         own = StarCache(w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale)

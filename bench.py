@@ -340,11 +340,12 @@ def measure_long_decode(dev, flush, warmup, steps, world, kv_fp8=False, name="8b
 
 def measure_sharded(dev, flush, w, ranks=8, steps=8):
     """The block-sharded layer's per-rank work on one GPU, its ranks run one
-    after another: each rank's phase 1 on its local [anchor | zeros | own
-    blocks] context (input assembly included), its phase-2 partial of the query
-    rows and of ``steps`` decode tokens (star_partial_attend), each timed alone
-    after an L2 flush, and the merge of the gathered partials.  The all_gather
-    between ranks is not run (one GPU); its bytes are reported."""
+    after another: each rank's phase 1 on its own blocks behind the anchor rows
+    (input slicing included), its phase-2 partial of the query rows and of
+    ``steps`` decode tokens (star_partial_attend), each timed alone after an L2
+    flush, and the merge of the gathered partials; then the decode partials
+    again with FP8 rank caches.  The all_gather between ranks is not run (one
+    GPU); its bytes are reported."""
     import torch
     from block_sparse_long_phase_b200 import workloads as wl
     from block_sparse_long_phase_b200.api import star_lse_merge_bf16
@@ -356,45 +357,52 @@ def measure_sharded(dev, flush, w, ranks=8, steps=8):
     T = min(w.T, steps + 1)
     x = wl.make_inputs(w, dev)
     Ka, Va = x["Kc"][:, :, :w.b_a].contiguous(), x["Vc"][:, :, :w.b_a].contiguous()
-    enc, pre, dec, dec_bytes = [], [], [], []
-    parts = []
-    for r in range(R):
-        sc = ShardedStarCache(r, R, w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale, device=dev)
-        lay = sc.layout
-        r0, r1 = lay.rows0, lay.rows0 + lay.rows
-        own = [x[k][:, :, r0:r1].contiguous() for k in ("Qc", "Kc", "Vc")]
-        flush.flush(11.0)
-        a, b = ev(), ev()
-        a.record(stream)
-        sc.encode(*own, Ka, Va)
-        b.record(stream)
-        del own
-        qkv = (x["Qq"], x["Kq"], x["Vq"]) if sc.is_query_rank else (x["Qq"],)
-        flush.flush(12.0)
-        c, d = ev(), ev()
-        c.record(stream)
-        sc.local_partial(*qkv)
-        d.record(stream)
-        steps_ev = []
-        for t in range(T):
-            qkv = (x["qd"][t], x["kd"][t], x["vd"][t]) if sc.is_query_rank else (x["qd"][t],)
-            flush.flush(13.0)
-            e0, e1 = ev(), ev()
-            e0.record(stream)
-            A, s_ = sc.local_partial(*qkv)
-            e1.record(stream)
-            steps_ev.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        assert sc.cache.device_error() == 0, "a kernel gave up a bounded pipeline wait"
-        enc.append(a.elapsed_time(b))
-        pre.append(c.elapsed_time(d))
-        dec.append(sum(e0.elapsed_time(e1) for e0, e1 in steps_ev[1:]) / max(1, len(steps_ev) - 1) * 1e3)
-        rows = lay.rows + ((w.lq + T) if sc.is_query_rank else 0)
-        dec_bytes.append(w.B * w.Hkv * rows * w.D * 2 * 2)
-        parts.append((A, s_))
-        sc.close()
+
+    def ranks_pass(kv_fp8):
+        enc, pre, dec, dec_bytes, parts = [], [], [], [], []
+        for r in range(R):
+            sc = ShardedStarCache(r, R, w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale,
+                                  device=dev, kv_fp8=kv_fp8)
+            lay = sc.layout
+            r0, r1 = lay.rows0, lay.rows0 + lay.rows
+            own = [x[k][:, :, r0:r1].contiguous() for k in ("Qc", "Kc", "Vc")]
+            flush.flush(11.0)
+            a, b = ev(), ev()
+            a.record(stream)
+            sc.encode(*own, Ka, Va)
+            b.record(stream)
+            del own
+            qkv = (x["Qq"], x["Kq"], x["Vq"]) if sc.is_query_rank else (x["Qq"],)
+            flush.flush(12.0)
+            c, d = ev(), ev()
+            c.record(stream)
+            sc.local_partial(*qkv)
+            d.record(stream)
+            steps_ev = []
+            for t in range(T):
+                qkv = (x["qd"][t], x["kd"][t], x["vd"][t]) if sc.is_query_rank else (x["qd"][t],)
+                flush.flush(13.0)
+                e0, e1 = ev(), ev()
+                e0.record(stream)
+                A, s_ = sc.local_partial(*qkv)
+                e1.record(stream)
+                steps_ev.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            assert sc.cache.device_error() == 0, "a kernel gave up a bounded pipeline wait"
+            enc.append(a.elapsed_time(b))
+            pre.append(c.elapsed_time(d))
+            dec.append(sum(e0.elapsed_time(e1) for e0, e1 in steps_ev[1:]) / max(1, len(steps_ev) - 1) * 1e3)
+            rows = lay.rows + ((w.lq + T) if sc.is_query_rank else 0)
+            row_bytes = (w.D + 4) * 2 if kv_fp8 else w.D * 2 * 2   # K and V of one cached row
+            dec_bytes.append(w.B * w.Hkv * rows * row_bytes)
+            parts.append((A, s_))
+            sc.close()
+        return enc, pre, dec, dec_bytes, parts
+
+    enc, pre, dec, dec_bytes, parts = ranks_pass(False)
     A = torch.stack([p_[0] for p_ in parts]).reshape(R, w.B * w.Hq, w.D).contiguous()
     S = torch.stack([p_[1] for p_ in parts]).reshape(R, w.B * w.Hq).contiguous()
+    del parts
     m = []
     for _ in range(5):
         flush.flush(14.0)
@@ -405,10 +413,13 @@ def measure_sharded(dev, flush, w, ranks=8, steps=8):
         m.append((a, b))
     torch.cuda.synchronize(dev)
     merge_us = sum(a.elapsed_time(b) for a, b in m[1:]) / (len(m) - 1) * 1e3
-    del x, Ka, Va, parts, A, S
+    del A, S
+    _, _, dec8, dec8_bytes, parts8 = ranks_pass(True)
+    del x, Ka, Va, parts8
     torch.cuda.empty_cache()
     pk = peaks()
     gbs = [by / (us * 1e-6) / 1e9 for by, us in zip(dec_bytes, dec)]
+    gbs8 = [by / (us * 1e-6) / 1e9 for by, us in zip(dec8_bytes, dec8)]
     return {
         "workload": w.name, "ranks": R, "how": "ranks run one after another on one GPU; the all_gather "
         "of the partials between them is not run",
@@ -417,6 +428,8 @@ def measure_sharded(dev, flush, w, ranks=8, steps=8):
         "prefill_partial_ms_per_rank": pre,
         "decode_partial_us_per_rank": dec, "decode_partial_us_max": max(dec),
         "decode_partial_frac_per_rank": [g / pk["hbm_gbs"] for g in gbs],
+        "decode_partial_fp8_us_per_rank": dec8, "decode_partial_fp8_us_max": max(dec8),
+        "decode_partial_fp8_frac_per_rank": [g / pk["hbm_gbs"] for g in gbs8],
         "merge_us": merge_us,
         "gather_bytes_per_rank_per_step": w.B * w.Hq * (w.D + 1) * 4}
 

@@ -688,11 +688,11 @@ int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query,
   // One row over segments that run to the end of the context (a generation
   // step of the block-sharded layer): the split-KV decode kernel streams them
   // at the HBM rate, where the prefill tile kernel would fill 128-row tiles
-  // from G rows.  The bf16 cache only: on an FP8 cache the decode kernel reads
-  // the E4M3 copy, which is not this call's arithmetic.
+  // from G rows.  On an FP8 cache it reads the E4M3 copy, as star_decode_step
+  // does on that cache.
   const long long skip = std::min<long long>((long long)first_seg * w.b, w.L);   // rows before first_seg
   const long long len0 = with_query ? c->q_len : 0;
-  if (lq == 1 && first_seg + n_seg == w.n_seg && !w.ctxK8 && w.L - skip + len0 >= 1) {
+  if (lq == 1 && first_seg + n_seg == w.n_seg && w.L - skip + len0 >= 1) {
     const star::DecodePlan dp = star::decode_plan(w, len0, c->num_sms, skip);
     cudaError_t e = star::launch_decode_step(
         w, c->dmaps, c->p.scale, (int)len0, static_cast<const bf16*>(Q), static_cast<const bf16*>(K),

@@ -71,9 +71,9 @@ def local_layout(rank: int, world: int, L: int, b: int) -> LocalLayout:
 class LibstarOps:
     """The kernels behind a shard: libstar's C ABI on the rank's GPU."""
 
-    def create(self, B, Hq, Hkv, D, L, block, anchor, q_cap, scale):
+    def create(self, B, Hq, Hkv, D, L, block, anchor, q_cap, scale, kv_fp8=False):
         from .api import StarCache
-        return StarCache(B, Hq, Hkv, D, L, block, anchor, q_cap, scale)
+        return StarCache(B, Hq, Hkv, D, L, block, anchor, q_cap, scale, kv_fp8=kv_fp8)
 
     def ctx_encode(self, cache, Q, K, V):
         return cache.star_ctx_encode(Q, K, V)
@@ -95,11 +95,14 @@ class ShardedStarCache:
 
     ``group`` is a torch.distributed process group (None: the default one);
     with ``world = 1`` no collective is issued.  ``query_rank`` defaults to the
-    last rank.  Outputs of phase 2 are the merged rows on every rank.
+    last rank.  Outputs of phase 2 are the merged rows on every rank.  With
+    ``kv_fp8`` every rank's cache keeps the FP8 copy and the generation steps
+    read it (as star_decode_step on such a cache); phase 1 and the query
+    prefill read the bf16 rows.
     """
 
     def __init__(self, rank, world, B, Hq, Hkv, D, L, block, anchor, q_cap, scale=0.0,
-                 query_rank=None, group=None, ops=None, device=None):
+                 query_rank=None, group=None, ops=None, device=None, kv_fp8=False):
         if not (0 <= anchor <= block):
             raise ValueError("need 0 <= anchor <= block")
         self.rank, self.world = rank, world
@@ -112,7 +115,11 @@ class ShardedStarCache:
         self.device = device if device is not None else (
             torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else torch.device("cpu"))
         self.layout = local_layout(rank, world, L, block)
-        self.cache = self.ops.create(B, Hq, Hkv, D, self.layout.L_local, block, anchor, q_cap, scale)
+        if kv_fp8:
+            self.cache = self.ops.create(B, Hq, Hkv, D, self.layout.L_local, block, anchor, q_cap, scale,
+                                         kv_fp8=True)
+        else:
+            self.cache = self.ops.create(B, Hq, Hkv, D, self.layout.L_local, block, anchor, q_cap, scale)
 
     @property
     def is_query_rank(self) -> bool:

@@ -267,9 +267,10 @@ STAR_API int star_decode_step(star_cache* c, const void* q, const void* k, const
  * the normalised local attention output, s [B][Hq][lq] its natural-log LSE
  * of the scaled logits (A = 0, s = -inf for a row that sees no key).
  * 1 <= lq <= q_cap.  STAR_ENOSPC if with_query and the region is full.
- * On a bf16 cache, lq = 1 over segments that reach the last one runs the
- * split-KV decode kernel (as star_decode_step over those rows); other calls
- * run the prefill tile kernel on a span plan of the range. */
+ * lq = 1 over segments that reach the last one runs the split-KV decode
+ * kernel (as star_decode_step over those rows: on a kv_fp8 cache it reads
+ * the E4M3 copy of the cached rows, the token exact); other calls run the
+ * prefill tile kernel on a span plan of the range, on the bf16 rows. */
 STAR_API int star_partial_attend(star_cache* c, int first_seg, int n_seg, int with_query, int lq,
                                  const void* Q, const void* K, const void* V, float* A, float* s,
                                  void* stream);

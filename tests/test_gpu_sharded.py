@@ -201,3 +201,48 @@ def test_ctx_encode_after_anchor_matches_the_oracle(name):
         assert torch.equal(k.view(torch.int16), x["Kc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
         assert torch.equal(v.view(torch.int16), x["Vc"][:, :, s0:s0 + seg.len].contiguous().view(torch.int16))
     c.close()
+
+
+FP8_CASES = [
+    (3, dict(L=1000, b=256, b_a=100, lq=4, T=3)),
+    (4, dict(L=4096, b=512, b_a=512, Hq=16, Hkv=4, D=128, lq=8, T=3)),
+]
+
+
+@pytest.mark.parametrize("world,shape", FP8_CASES)
+def test_sharded_fp8_decode_matches_the_dequantised_oracle(world, shape):
+    """Ranks with FP8 caches: the query prefill reads the bf16 rows (exact
+    oracle); each generation step's partials read the E4M3 copies, so the
+    merged step equals the single-device FP8 decode: the oracle on the
+    dequantised context and query region, the step's own token exact."""
+    from test_gpu_fp8 import decode_reference, dequantised
+    w = wl.get("tiny").with_(**shape)
+    cpu = wl.make_inputs(w, "cpu")
+    x = {k: v.cuda() for k, v in cpu.items()}
+    ranks = [ShardedStarCache(r, world, w.B, w.Hq, w.Hkv, w.D, w.L, w.b, w.b_a, w.lq + w.T, w.scale,
+                              kv_fp8=True) for r in range(world)]
+    for sc in ranks:
+        lay = sc.layout
+        r0, r1 = lay.rows0, lay.rows0 + lay.rows
+        sc.encode(x["Qc"][:, :, r0:r1].contiguous(), x["Kc"][:, :, r0:r1].contiguous(),
+                  x["Vc"][:, :, r0:r1].contiguous(), x["Kc"][:, :, :w.b_a].contiguous(),
+                  x["Vc"][:, :, :w.b_a].contiguous())
+
+    def step(Q, K, V):
+        parts = [sc.local_partial(Q, K, V) for sc in ranks]
+        return ranks[-1].merge(torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts]))
+
+    Oq, Lq = step(x["Qq"], x["Kq"], x["Vq"])
+    dec = [step(x["qd"][t], x["kd"][t], x["vd"][t]) for t in range(w.T)]
+    torch.cuda.synchronize()
+    segs = so.cache_segments(cpu["Kc"], cpu["Vc"], w.b)
+    region = np.zeros((w.B, w.Hkv, w.lq + w.T, w.D))
+    ref, lref, _, _ = so.query_prefill(cpu["Qq"], cpu["Kq"], cpu["Vq"], segs, region, region, 0, w.scale)
+    assert_close(Oq, ref, Lq, lref, f"sharded fp8 x{world} prefill")
+    segs_deq = so.cache_segments(dequantised(cpu["Kc"]), dequantised(cpu["Vc"]), w.b)
+    for t in range(w.T):
+        o_ref, l_ref = decode_reference(cpu, segs_deq, t, w.lq, w.scale)
+        assert_close(dec[t][0], o_ref, dec[t][1][:, :, 0], l_ref[:, :, 0], f"sharded fp8 x{world} decode {t}")
+    for sc in ranks:
+        assert sc.cache.device_error() == 0
+        sc.close()
